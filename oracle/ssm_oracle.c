@@ -1,0 +1,221 @@
+/*
+ * ssm_oracle.c -- plain, sequential, double-precision CPU restatement of the
+ * selective state-space scan.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may call this code:
+ * only tests/, __graft_entry__.smoke() and bench.py's CPU-baseline / reference
+ * leg may load, call or link it.  It shares no code, header, table or helper
+ * with the CUDA library; the two only ever see the same seeded inputs.
+ *
+ * Sources (page title, then section):
+ *  [P1] "Selective Scan trong Mamba toi uu chuoi dai the nao?" (thecsnote.cc)
+ *       - "Tai sao Mamba can Selective Scan?": h_t = Abar h_{t-1} + Bbar x_t,
+ *         y_t = C h_t.
+ *       - "Selection pha vo convolution kernel co dinh": B_t, C_t and
+ *         Delta_t = softplus(theta + s(x_t)) vary per token, giving the
+ *         time-varying recurrence h_t = Abar_t h_{t-1} + Bbar_t x_t.
+ *       - "Vi du Python": diagonal A, Abar = exp(Delta*A); its zero-order-hold
+ *         input matrix Bbar = expm1(Delta*A)/A * B (kept here as an option).
+ *       - "Selective Scan thay doi inference chuoi dai nhu the nao?": decoding
+ *         updates a fixed-size state one token at a time.
+ *  [P3] "Selective (Data-Dependent) SSM Scan" (cartesia-pytorch, problem 15)
+ *       - "Step-by-Step Approach" 3-4: elementwise update h = A_t*h + B_t*x_t,
+ *         readout y_t = C_t*h taken from the UPDATED state.
+ *  The default input coefficient is Bbar_t = Delta_t * B_t (the simplified
+ *  discretisation the library targets: "(Delta_t*B_t)*x_t"); the output is
+ *  y_t = C_t . h_t + D*x_t, optionally multiplied by silu(z_t), with
+ *  silu(z) = z * sigmoid(z).  Every floating-point step is done in double.
+ *
+ * Layouts (row-major, contiguous): x, delta, z, y: (B, L, D); Bm, Cm:
+ * (B, L, N); A: (D, N); D, bias: (D); h0, h_last, state: (B, D, N).
+ * In the elementwise variant x, A, B, C, y are (B, L, D) and h0, h_last are
+ * (B, D).
+ *
+ * ORACLE_MUTANT (compile-time, tests only) plants one deliberate mistake so a
+ * test can show that the pins catch it.  The default build has none.
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdint.h>
+#include <stdlib.h>
+
+#ifndef ORACLE_MUTANT
+#define ORACLE_MUTANT 0
+#endif
+
+/* Option bits understood by the oracle.  They are the oracle's own
+ * definitions; the Python wrapper maps keyword arguments onto them. */
+#define ORC_HAS_Z 1u
+#define ORC_HAS_D 2u
+#define ORC_SOFTPLUS 4u
+#define ORC_HAS_BIAS 8u
+#define ORC_HAS_H0 16u
+#define ORC_ZOH 128u
+
+/* softplus(v) = log(1 + e^v), written in the overflow-free form
+ * max(v, 0) + log1p(e^{-|v|}).  [P1] "Selection ...": Delta = softplus(.). */
+double ssm_oracle_softplus(double v) {
+#if ORACLE_MUTANT == 5
+  return log(1.0 + exp(v)) + 1e-3; /* biased softplus */
+#else
+  return (v > 0.0 ? v : 0.0) + log1p(exp(-fabs(v)));
+#endif
+}
+
+/* silu(z) = z * sigmoid(z) = z / (1 + e^{-z}). */
+double ssm_oracle_silu(double z) {
+#if ORACLE_MUTANT == 6
+  return 1.0 / (1.0 + exp(-z)); /* sigmoid instead of silu */
+#else
+  return z / (1.0 + exp(-z));
+#endif
+}
+
+/* One token of the Mamba-form recurrence for one channel (b, d).
+ * h[0..N) is updated in place; returns y for this token.  [P1] "Selection
+ * ...": Abar_t = exp(Delta_t*A), Bbar_t = Delta_t*B_t (or ZOH), h updated
+ * first, readout from the updated state ([P3] step 4). */
+static double token_update(int64_t N, uint32_t flags, double xv, double dv,
+                           double bias, const double *Arow, const double *Bt,
+                           const double *Ct, double Dd, double zv, double *h) {
+  double v = dv + bias;
+  double dt = (flags & ORC_SOFTPLUS) ? ssm_oracle_softplus(v) : v;
+#if ORACLE_MUTANT == 7
+  dt = (flags & ORC_SOFTPLUS) ? ssm_oracle_softplus(dv) : dv; /* bias dropped */
+#endif
+  double acc = 0.0;
+  for (int64_t n = 0; n < N; ++n) {
+    double a = Arow[n];
+    double abar = exp(dt * a);
+#if ORACLE_MUTANT == 1
+    abar = exp(-dt * a); /* sign flip */
+#endif
+    double bbar;
+    if (flags & ORC_ZOH)
+      bbar = (a != 0.0 ? expm1(dt * a) / a : dt) * Bt[n];
+    else
+      bbar = dt * Bt[n];
+#if ORACLE_MUTANT == 2
+    acc += Ct[n] * h[n]; /* readout from the state before the update */
+#endif
+    h[n] = abar * h[n] + bbar * xv;
+#if ORACLE_MUTANT == 8
+    h[n] = abar * h[n] + bbar; /* input x dropped */
+#endif
+#if ORACLE_MUTANT != 2
+#if ORACLE_MUTANT == 9
+    acc += Bt[n] * h[n]; /* B used as readout instead of C */
+#else
+    acc += Ct[n] * h[n];
+#endif
+#endif
+  }
+  if (flags & ORC_HAS_D) {
+#if ORACLE_MUTANT != 3
+    acc += Dd * xv;
+#endif
+  }
+  if (flags & ORC_HAS_Z) {
+#if ORACLE_MUTANT == 4
+    acc = (acc - Dd * xv) * ssm_oracle_silu(zv) + ((flags & ORC_HAS_D) ? Dd * xv : 0.0);
+#else
+    acc *= ssm_oracle_silu(zv);
+#endif
+  }
+  return acc;
+}
+
+/* Full-sequence forward pass: for every channel (b, d) run t = 0..L-1 in
+ * order.  Returns 0, or -1 on a bad argument / allocation failure.  h_last
+ * may be NULL. */
+int ssm_oracle_fwd(int64_t Bsz, int64_t L, int64_t D, int64_t N, uint32_t flags,
+                   const double *x, const double *delta, const double *bias,
+                   const double *A, const double *Bm, const double *Cm,
+                   const double *Dv, const double *z, const double *h0,
+                   double *y, double *h_last) {
+  if (Bsz < 0 || L < 0 || D < 0 || N < 1) return -1;
+  if (!x || !delta || !A || !Bm || !Cm || !y) return -1;
+  if ((flags & ORC_HAS_Z) && !z) return -1;
+  if ((flags & ORC_HAS_D) && !Dv) return -1;
+  if ((flags & ORC_HAS_BIAS) && !bias) return -1;
+  if ((flags & ORC_HAS_H0) && !h0) return -1;
+  double *h = (double *)malloc((size_t)N * sizeof(double));
+  if (!h) return -1;
+  for (int64_t b = 0; b < Bsz; ++b) {
+    for (int64_t d = 0; d < D; ++d) {
+      for (int64_t n = 0; n < N; ++n) {
+        h[n] = (flags & ORC_HAS_H0) ? h0[(b * D + d) * N + n] : 0.0;
+#if ORACLE_MUTANT == 10
+        h[n] = 0.0; /* h0 ignored */
+#endif
+      }
+      for (int64_t t = 0; t < L; ++t) {
+        size_t i = (size_t)((b * L + t) * D + d);
+        size_t j = (size_t)((b * L + t) * N);
+#if ORACLE_MUTANT == 11
+        /* B and C taken from the previous token */
+        if (t > 0) j -= (size_t)N;
+#endif
+        y[i] = token_update(N, flags, x[i], delta[i],
+                            (flags & ORC_HAS_BIAS) ? bias[d] : 0.0, A + d * N,
+                            Bm + j, Cm + j, (flags & ORC_HAS_D) ? Dv[d] : 0.0,
+                            (flags & ORC_HAS_Z) ? z[i] : 0.0, h);
+      }
+      if (h_last)
+        for (int64_t n = 0; n < N; ++n) h_last[(b * D + d) * N + n] = h[n];
+    }
+  }
+  free(h);
+  return 0;
+}
+
+/* One decode step ([P1] inference section): state (B, D, N) is read, updated
+ * with one token and written back; y is (B, D).  x, delta, z: (B, D);
+ * Bm, Cm: (B, N). */
+int ssm_oracle_step(int64_t Bsz, int64_t D, int64_t N, uint32_t flags,
+                    const double *x, const double *delta, const double *bias,
+                    const double *A, const double *Bm, const double *Cm,
+                    const double *Dv, const double *z, double *state, double *y) {
+  if (Bsz < 0 || D < 0 || N < 1) return -1;
+  if (!x || !delta || !A || !Bm || !Cm || !state || !y) return -1;
+  if ((flags & ORC_HAS_Z) && !z) return -1;
+  if ((flags & ORC_HAS_D) && !Dv) return -1;
+  if ((flags & ORC_HAS_BIAS) && !bias) return -1;
+  for (int64_t b = 0; b < Bsz; ++b) {
+    for (int64_t d = 0; d < D; ++d) {
+      size_t i = (size_t)(b * D + d);
+      y[i] = token_update(N, flags, x[i], delta[i],
+                          (flags & ORC_HAS_BIAS) ? bias[d] : 0.0, A + d * N,
+                          Bm + b * N, Cm + b * N,
+                          (flags & ORC_HAS_D) ? Dv[d] : 0.0,
+                          (flags & ORC_HAS_Z) ? z[i] : 0.0, state + i * N);
+    }
+  }
+  return 0;
+}
+
+/* Elementwise variant ([P3] steps 2-5): A_t is the transition itself,
+ * h = A_t*h + B_t*x_t, y_t = C_t*h (after the update).  All of x, A, B, C, y
+ * are (B, L, D); h0 and h_last are (B, D) and may be NULL (h0 = 0). */
+int ssm_oracle_direct(int64_t Bsz, int64_t L, int64_t D, const double *x,
+                      const double *A, const double *Bm, const double *Cm,
+                      const double *h0, double *y, double *h_last) {
+  if (Bsz < 0 || L < 0 || D < 0) return -1;
+  if (!x || !A || !Bm || !Cm || !y) return -1;
+  for (int64_t b = 0; b < Bsz; ++b) {
+    for (int64_t d = 0; d < D; ++d) {
+      double h = h0 ? h0[b * D + d] : 0.0;
+      for (int64_t t = 0; t < L; ++t) {
+        size_t i = (size_t)((b * L + t) * D + d);
+#if ORACLE_MUTANT == 12
+        h = Bm[i] * x[i] + (t > 0 ? A[i - D] : A[i]) * h; /* A from previous token */
+#else
+        h = A[i] * h + Bm[i] * x[i];
+#endif
+        y[i] = Cm[i] * h;
+      }
+      if (h_last) h_last[b * D + d] = h;
+    }
+  }
+  return 0;
+}
