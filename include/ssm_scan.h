@@ -1,0 +1,188 @@
+/*
+ * ssm_scan.h -- C ABI of the B200 (sm_100a) selective state-space scan.
+ *
+ * The operation (page titles and sections cited):
+ *   "Selective Scan trong Mamba toi uu chuoi dai the nao?" (thecsnote.cc)
+ *     - "Tai sao Mamba can Selective Scan?": the discrete recurrence
+ *       h_t = Abar h_{t-1} + Bbar x_t, y_t = C h_t.
+ *     - "Selection pha vo convolution kernel co dinh": B_t, C_t and
+ *       Delta_t = softplus(theta + s(x_t)) change per token, so
+ *       h_t = Abar_t h_{t-1} + Bbar_t x_t, y_t = C_t h_t.
+ *     - "Vi du Python": diagonal A, Abar_t = exp(Delta_t * A).
+ *     - "Scan bien recurrence thanh phep toan co the song song hoa ra sao?":
+ *       the per-token affine maps compose associatively,
+ *       (A2, b2) (x) (A1, b1) = (A2 A1, A2 b1 + b2).
+ *     - "Tai sao chi parallel scan van chua du nhanh?" / "Kernel fusion":
+ *       the (B, L, D, N) state is never written to HBM.
+ *     - "Selective Scan thay doi inference chuoi dai nhu the nao?": decode
+ *       keeps one fixed-size state per layer and updates it per token.
+ *   "Selective (Data-Dependent) SSM Scan" (cartesia-pytorch, problem 15)
+ *     - "Step-by-Step Approach" 2-6 and the reference solution: elementwise
+ *       variant h = A_t*h + B_t*x_t, y_t = C_t*h read after the update
+ *       (flag SSM_A_DIRECT).
+ *
+ * Computed per channel (b, d), for t = 0 .. L-1, per state n < N:
+ *   Delta   = softplus(delta[b,t,d] + delta_bias[d])   (softplus if flagged)
+ *   h[n]    = exp(Delta * A[d,n]) * h[n] + (Delta * B[b,t,n]) * x[b,t,d]
+ *   y[b,t,d]= (sum_n C[b,t,n] * h[n] + D[d] * x[b,t,d]) * silu(z[b,t,d])
+ * with h starting at h0 (or 0) and h_last = h after the last token.  The
+ * skip and gate terms are present only when flagged; silu(z) = z*sigmoid(z).
+ *
+ * Layouts (row-major, contiguous, element strides implied by the shape):
+ *   x, delta, z, y : (batch, seqlen, dim)         in_dtype / out_dtype
+ *   B, C           : (batch, seqlen, dstate)      in_dtype
+ *   A              : (dim, dstate) fp32           (SSM_A_DIRECT: (batch, seqlen, dim) in_dtype)
+ *   D, delta_bias  : (dim) fp32
+ *   h0, h_last     : (batch, dim, dstate) fp32    (SSM_A_DIRECT: (batch, dim))
+ *   state (step)   : (batch, dim, dstate) fp32, read and written in place
+ *   step inputs    : x, delta, z, y (batch, dim); B, C (batch, dstate)
+ *
+ * Ownership: the caller owns every tensor; all data pointers are DEVICE
+ * pointers on the plan's device.  The plan owns a small workspace allocated
+ * by ssm_scan_create; ssm_scan_fwd / ssm_scan_step allocate nothing and are
+ * asynchronous on the caller's stream.  Calls on one plan must not overlap
+ * in time (issue them on one stream, or order them): they share the
+ * workspace.  y must not alias any input; only `state` is updated in place.
+ *
+ * Errors: argument checks are synchronous and launch nothing.  A failed
+ * launch returns SSM_ERR_CUDA.  The only device-side wait (a chunk waiting
+ * for the carried state of the previous chunk of the same channels) is
+ * bounded; if it expires the kernel records SSM_ERR_TIMEOUT, finishes without
+ * hanging, and y/h_last of that call are unspecified.  ssm_scan_get_status
+ * synchronises the device and returns (and clears) that record.
+ *
+ * Alignment: the fast path needs 16-byte aligned pointers, dim*sizeof(in)
+ * and dstate*sizeof(in) multiples of 16 bytes, and dstate in {8, 16} (bf16)
+ * or {4, 8, 16} (fp32).  Any other valid shape runs on a slower general
+ * kernel of the same library (never on the CPU).
+ */
+#ifndef SSM_SCAN_H
+#define SSM_SCAN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SSM_API __attribute__((visibility("default")))
+#else
+#define SSM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *ssm_stream_t; /* same object as cudaStream_t */
+
+typedef enum {
+  SSM_OK = 0,
+  SSM_ERR_INVALID_ARG = 1, /* null/negative/inconsistent argument or flags */
+  SSM_ERR_UNSUPPORTED = 2, /* valid but not supported (e.g. dstate > 64) */
+  SSM_ERR_MISALIGNED = 3,  /* reserved: misaligned data takes the general kernel */
+  SSM_ERR_CUDA = 4,        /* CUDA runtime error (no device, launch failure) */
+  SSM_ERR_TIMEOUT = 5,     /* a bounded device-side wait expired */
+  SSM_ERR_OOM = 6          /* workspace allocation failed in ssm_scan_create */
+} ssm_status;
+
+typedef enum { SSM_F32 = 0, SSM_BF16 = 1 } ssm_dtype;
+
+enum {
+  SSM_HAS_Z = 1,            /* multiply y by silu(z) */
+  SSM_HAS_D = 2,            /* add D[d] * x */
+  SSM_DELTA_SOFTPLUS = 4,   /* Delta = softplus(delta + bias) (else delta + bias) */
+  SSM_HAS_DELTA_BIAS = 8,   /* add delta_bias[d] before softplus */
+  SSM_HAS_H0 = 16,          /* start from h0 (else from 0) */
+  SSM_WANT_HLAST = 32,      /* write h_last */
+  SSM_A_DIRECT = 64         /* elementwise variant: N = 1, A/B/C per (b,t,d), no delta/D/z */
+};
+
+typedef struct {
+  int64_t batch, seqlen, dim, dstate;
+  ssm_dtype in_dtype;  /* x, delta, z, B, C (and A in SSM_A_DIRECT) */
+  ssm_dtype out_dtype; /* y; states are always fp32 */
+  uint32_t flags;
+} ssm_scan_desc;
+
+typedef struct ssm_scan_plan ssm_scan_plan;
+
+/* Plan details chosen by ssm_scan_create (read-only; for tests and tuning). */
+typedef struct {
+  int path;            /* 0 = TMA chunked kernel, 1 = general kernel, 2 = elementwise, 3 = step */
+  int lanes_per_chan;  /* lanes sharing one channel's dstate states */
+  int warps_per_cta;
+  int tile_t;          /* timesteps per pipeline stage */
+  int stages;          /* pipeline depth */
+  int seg_len;         /* timesteps per work item (chunk) */
+  int chans_per_cta;
+  int grid;            /* persistent CTAs launched */
+  int64_t rows;        /* independent (batch, channel-tile) rows */
+  int64_t items;       /* work items = rows * chunks */
+  size_t smem_bytes;
+  size_t workspace_bytes;
+} ssm_scan_info;
+
+/* Optional overrides of the launch shape (0 = keep the default). */
+typedef struct {
+  int lanes_per_chan; /* 1, 2, 4, 8 (<= dstate) */
+  int warps_per_cta;  /* 2, 4, 8 */
+  int seg_len;        /* multiple of the stage length */
+  int grid;           /* persistent CTAs (clamped to what fits on the device) */
+} ssm_scan_config;
+
+/* Create a plan for one problem shape on `device`; allocates the workspace.
+ * Returns SSM_ERR_INVALID_ARG / SSM_ERR_UNSUPPORTED for a bad desc (checked
+ * before any CUDA call), SSM_ERR_CUDA if the device is unusable,
+ * SSM_ERR_OOM if the workspace cannot be allocated. */
+SSM_API ssm_status ssm_scan_create(ssm_scan_plan **plan, const ssm_scan_desc *desc, int device);
+
+/* Free the plan and its workspace (synchronises the device first). */
+SSM_API ssm_status ssm_scan_destroy(ssm_scan_plan *plan);
+
+/* Full-sequence forward pass (prefill / training forward), the fused
+ * discretise + scan + readout + skip + gate of the pages' "Kernel fusion"
+ * section.  Optional pointers (delta_bias, D, z, h0, h_last) must be NULL
+ * exactly when their flag is clear.  In SSM_A_DIRECT mode pass A, B, C, x,
+ * y (and h0/h_last of shape (batch, dim)); delta, delta_bias, D, z must be
+ * NULL. */
+SSM_API ssm_status ssm_scan_fwd(ssm_scan_plan *plan, const void *x, const void *delta,
+                        const float *delta_bias, const void *A, const void *B,
+                        const void *C, const float *D, const void *z,
+                        const float *h0, void *y, float *h_last, ssm_stream_t stream);
+
+/* One decode step per the pages' inference section: reads `state`
+ * (batch, dim, dstate), applies one token, writes it back and writes y
+ * (batch, dim).  desc.seqlen is ignored; SSM_HAS_H0 / SSM_WANT_HLAST /
+ * SSM_A_DIRECT are not used. */
+SSM_API ssm_status ssm_scan_step(ssm_scan_plan *plan, const void *x, const void *delta,
+                         const float *delta_bias, const float *A, const void *B,
+                         const void *C, const float *D, const void *z, float *state,
+                         void *y, ssm_stream_t stream);
+
+/* Synchronise the plan's device, return the device-side status recorded by
+ * the last calls (SSM_OK or SSM_ERR_TIMEOUT) and reset it to SSM_OK. */
+SSM_API ssm_status ssm_scan_get_status(ssm_scan_plan *plan);
+
+/* Fill *info with the plan's launch shape. */
+SSM_API ssm_status ssm_scan_get_info(const ssm_scan_plan *plan, ssm_scan_info *info);
+
+/* Override the launch shape (tuning); takes effect on the next call.  May
+ * reallocate the workspace, so call it between calls, not during one. */
+SSM_API ssm_status ssm_scan_set_config(ssm_scan_plan *plan, const ssm_scan_config *cfg);
+
+/* Test hook: set the bound of device-side waits (nanoseconds, 0 = default
+ * of 2 s) and make work item `drop_item` (-1 = none) skip publishing its
+ * carried state, so the next chunk's bounded wait expires.  Used to test
+ * the timeout path without hanging the device. */
+SSM_API ssm_status ssm_scan_set_debug(ssm_scan_plan *plan, uint64_t wait_timeout_ns, int64_t drop_item);
+
+/* Static description of a status code. */
+SSM_API const char *ssm_status_string(ssm_status s);
+
+/* Library version as 10000*major + 100*minor + patch. */
+SSM_API int ssm_scan_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSM_SCAN_H */

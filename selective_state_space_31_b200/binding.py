@@ -1,0 +1,287 @@
+"""ctypes binding of ``libssm_scan_b200.so`` (C ABI: ``include/ssm_scan.h``).
+
+Argument marshalling only: tensors are checked for device, dtype, shape and
+contiguity, their data pointers and the current CUDA stream are passed to
+the library, and every step of the scan runs in the library's kernels.
+There is no fallback: if the library is missing, loading fails loudly.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libssm_scan_b200.so")
+
+# ssm_status
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_MISALIGNED, ERR_CUDA, ERR_TIMEOUT, ERR_OOM = range(7)
+# ssm_dtype
+F32, BF16 = 0, 1
+# flags
+HAS_Z, HAS_D, DELTA_SOFTPLUS, HAS_DELTA_BIAS, HAS_H0, WANT_HLAST, A_DIRECT = 1, 2, 4, 8, 16, 32, 64
+
+_TORCH_TO_SSM = {torch.float32: F32, torch.bfloat16: BF16}
+
+
+class SsmError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+
+
+class Desc(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64), ("dim", ctypes.c_int64),
+                ("dstate", ctypes.c_int64), ("in_dtype", ctypes.c_int), ("out_dtype", ctypes.c_int),
+                ("flags", ctypes.c_uint32)]
+
+
+class Info(ctypes.Structure):
+    _fields_ = [("path", ctypes.c_int), ("lanes_per_chan", ctypes.c_int),
+                ("warps_per_cta", ctypes.c_int), ("tile_t", ctypes.c_int), ("stages", ctypes.c_int),
+                ("seg_len", ctypes.c_int), ("chans_per_cta", ctypes.c_int), ("grid", ctypes.c_int),
+                ("rows", ctypes.c_int64), ("items", ctypes.c_int64),
+                ("smem_bytes", ctypes.c_size_t), ("workspace_bytes", ctypes.c_size_t)]
+
+    def as_dict(self):
+        return {k: getattr(self, k) for k, _ in self._fields_}
+
+
+class Config(ctypes.Structure):
+    _fields_ = [("lanes_per_chan", ctypes.c_int), ("warps_per_cta", ctypes.c_int),
+                ("seg_len", ctypes.c_int), ("grid", ctypes.c_int)]
+
+
+_lib = None
+_lib_lock = threading.Lock()
+_vp = ctypes.c_void_p
+
+
+def load_library(path: str | None = None):
+    """Load the CUDA library (once).  Raises if it has not been built."""
+    global _lib
+    with _lib_lock:
+        if _lib is not None:
+            return _lib
+        path = path or LIB_PATH
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} is missing: build it with "
+                               "`python -m selective_state_space_31_b200.build`")
+        lib = ctypes.CDLL(path)
+        st = ctypes.c_int
+        lib.ssm_scan_create.argtypes = [ctypes.POINTER(_vp), ctypes.POINTER(Desc), ctypes.c_int]
+        lib.ssm_scan_create.restype = st
+        lib.ssm_scan_destroy.argtypes = [_vp]
+        lib.ssm_scan_destroy.restype = st
+        lib.ssm_scan_fwd.argtypes = [_vp] * 13
+        lib.ssm_scan_fwd.restype = st
+        lib.ssm_scan_step.argtypes = [_vp] * 12
+        lib.ssm_scan_step.restype = st
+        lib.ssm_scan_get_status.argtypes = [_vp]
+        lib.ssm_scan_get_status.restype = st
+        lib.ssm_scan_get_info.argtypes = [_vp, ctypes.POINTER(Info)]
+        lib.ssm_scan_get_info.restype = st
+        lib.ssm_scan_set_config.argtypes = [_vp, ctypes.POINTER(Config)]
+        lib.ssm_scan_set_config.restype = st
+        lib.ssm_scan_set_debug.argtypes = [_vp, ctypes.c_uint64, ctypes.c_int64]
+        lib.ssm_scan_set_debug.restype = st
+        lib.ssm_status_string.argtypes = [ctypes.c_int]
+        lib.ssm_status_string.restype = ctypes.c_char_p
+        lib.ssm_scan_version.argtypes = []
+        lib.ssm_scan_version.restype = ctypes.c_int
+        _lib = lib
+        return lib
+
+
+def status_string(s: int) -> str:
+    return load_library().ssm_status_string(int(s)).decode()
+
+
+def _check(rc: int, what: str):
+    if rc != OK:
+        raise SsmError(rc, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _need(t, name, shape, dtype, device):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+class Plan:
+    """One problem shape on one device (wraps ``ssm_scan_plan``)."""
+
+    def __init__(self, batch, seqlen, dim, dstate, in_dtype=torch.bfloat16, out_dtype=None,
+                 flags=0, device=None):
+        self._lib = load_library()
+        self.device = torch.device(device if device is not None else "cuda", )
+        if self.device.index is None:
+            self.device = torch.device("cuda", torch.cuda.current_device())
+        out_dtype = out_dtype or in_dtype
+        self.desc = Desc(int(batch), int(seqlen), int(dim), int(dstate),
+                         _TORCH_TO_SSM[in_dtype], _TORCH_TO_SSM[out_dtype], int(flags))
+        self.in_dtype, self.out_dtype, self.flags = in_dtype, out_dtype, int(flags)
+        h = _vp()
+        _check(self._lib.ssm_scan_create(ctypes.byref(h), ctypes.byref(self.desc),
+                                         self.device.index), "ssm_scan_create")
+        self._h = h
+
+    def close(self):
+        if getattr(self, "_h", None) is not None and self._h.value:
+            self._lib.ssm_scan_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def info(self) -> dict:
+        i = Info()
+        _check(self._lib.ssm_scan_get_info(self._h, ctypes.byref(i)), "ssm_scan_get_info")
+        return i.as_dict()
+
+    def set_config(self, lanes_per_chan=0, warps_per_cta=0, seg_len=0, grid=0):
+        c = Config(lanes_per_chan, warps_per_cta, seg_len, grid)
+        _check(self._lib.ssm_scan_set_config(self._h, ctypes.byref(c)), "ssm_scan_set_config")
+
+    def set_debug(self, wait_timeout_ns=0, drop_item=-1):
+        _check(self._lib.ssm_scan_set_debug(self._h, int(wait_timeout_ns), int(drop_item)),
+               "ssm_scan_set_debug")
+
+    def status(self) -> int:
+        """Synchronise and return (and clear) the device-side status."""
+        return self._lib.ssm_scan_get_status(self._h)
+
+    # -- calls -------------------------------------------------------------
+    def fwd(self, x, delta, A, B, C, D=None, z=None, delta_bias=None, h0=None, y=None,
+            h_last=None):
+        d, f, dev = self.desc, self.flags, self.device
+        Bz, L, Dm, N = d.batch, d.seqlen, d.dim, d.dstate
+        if f & A_DIRECT:
+            _need(A, "A", (Bz, L, Dm), self.in_dtype, dev)
+            _need(h0, "h0", (Bz, Dm), torch.float32, dev)
+            hshape = (Bz, Dm)
+        else:
+            _need(delta, "delta", (Bz, L, Dm), self.in_dtype, dev)
+            _need(A, "A", (Dm, N), torch.float32, dev)
+            _need(D, "D", (Dm,), torch.float32, dev)
+            _need(z, "z", (Bz, L, Dm), self.in_dtype, dev)
+            _need(delta_bias, "delta_bias", (Dm,), torch.float32, dev)
+            _need(h0, "h0", (Bz, Dm, N), torch.float32, dev)
+            hshape = (Bz, Dm, N)
+        _need(x, "x", (Bz, L, Dm), self.in_dtype, dev)
+        bshape = (Bz, L, Dm) if f & A_DIRECT else (Bz, L, N)
+        _need(B, "B", bshape, self.in_dtype, dev)
+        _need(C, "C", bshape, self.in_dtype, dev)
+        if y is None:
+            y = torch.empty((Bz, L, Dm), dtype=self.out_dtype, device=dev)
+        _need(y, "y", (Bz, L, Dm), self.out_dtype, dev)
+        if f & WANT_HLAST and h_last is None:
+            h_last = torch.empty(hshape, dtype=torch.float32, device=dev)
+        _need(h_last, "h_last", hshape, torch.float32, dev)
+        rc = self._lib.ssm_scan_fwd(self._h, _ptr(x), _ptr(delta), _ptr(delta_bias), _ptr(A),
+                                    _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(h0), _ptr(y),
+                                    _ptr(h_last), _stream(dev))
+        _check(rc, "ssm_scan_fwd")
+        return y, h_last
+
+    def step(self, state, x, delta, A, B, C, D=None, z=None, delta_bias=None, y=None):
+        d, dev = self.desc, self.device
+        Bz, Dm, N = d.batch, d.dim, d.dstate
+        _need(state, "state", (Bz, Dm, N), torch.float32, dev)
+        for name, t in (("x", x), ("delta", delta), ("z", z)):
+            _need(t, name, (Bz, Dm), self.in_dtype, dev)
+        _need(A, "A", (Dm, N), torch.float32, dev)
+        _need(B, "B", (Bz, N), self.in_dtype, dev)
+        _need(C, "C", (Bz, N), self.in_dtype, dev)
+        _need(D, "D", (Dm,), torch.float32, dev)
+        _need(delta_bias, "delta_bias", (Dm,), torch.float32, dev)
+        if y is None:
+            y = torch.empty((Bz, Dm), dtype=self.out_dtype, device=dev)
+        _need(y, "y", (Bz, Dm), self.out_dtype, dev)
+        rc = self._lib.ssm_scan_step(self._h, _ptr(x), _ptr(delta), _ptr(delta_bias), _ptr(A),
+                                     _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(state), _ptr(y),
+                                     _stream(dev))
+        _check(rc, "ssm_scan_step")
+        return y
+
+
+def flags_for(*, z=None, D=None, delta_bias=None, h0=None, delta_softplus=True,
+              want_h_last=True) -> int:
+    return ((HAS_Z if z is not None else 0) | (HAS_D if D is not None else 0)
+            | (DELTA_SOFTPLUS if delta_softplus else 0)
+            | (HAS_DELTA_BIAS if delta_bias is not None else 0)
+            | (HAS_H0 if h0 is not None else 0) | (WANT_HLAST if want_h_last else 0))
+
+
+_plans: dict = {}
+_plans_lock = threading.Lock()
+
+
+def _plan_for(key, make):
+    with _plans_lock:
+        p = _plans.get(key)
+        if p is None:
+            p = make()
+            _plans[key] = p
+        return p
+
+
+def fwd(x, delta, A, B, C, D=None, z=None, delta_bias=None, h0=None, delta_softplus=True,
+        want_h_last=True, out_dtype=None):
+    """Selective-scan forward.  x, delta, z: (B, L, D); B, C: (B, L, N);
+    A: (D, N) fp32; D, delta_bias: (D,) fp32; h0: (B, D, N) fp32.
+    Returns (y, h_last) (h_last is None when not requested)."""
+    Bz, L, Dm = x.shape
+    N = A.shape[1]
+    flags = flags_for(z=z, D=D, delta_bias=delta_bias, h0=h0, delta_softplus=delta_softplus,
+                      want_h_last=want_h_last)
+    out_dtype = out_dtype or x.dtype
+    key = ("fwd", Bz, L, Dm, N, x.dtype, out_dtype, flags, x.device)
+    plan = _plan_for(key, lambda: Plan(Bz, L, Dm, N, x.dtype, out_dtype, flags, x.device))
+    return plan.fwd(x, delta, A, B, C, D=D, z=z, delta_bias=delta_bias, h0=h0)
+
+
+def step(state, x, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True,
+         out_dtype=None):
+    """One decode step: updates ``state`` (B, D, N) fp32 in place, returns y (B, D)."""
+    Bz, Dm, N = state.shape
+    flags = flags_for(z=z, D=D, delta_bias=delta_bias, delta_softplus=delta_softplus,
+                      want_h_last=False)
+    out_dtype = out_dtype or x.dtype
+    key = ("step", Bz, Dm, N, x.dtype, out_dtype, flags, x.device)
+    plan = _plan_for(key, lambda: Plan(Bz, 1, Dm, N, x.dtype, out_dtype, flags, x.device))
+    return plan.step(state, x, delta, A, B, C, D=D, z=z, delta_bias=delta_bias)
+
+
+def direct(x, A, B, C, h0=None, want_h_last=True, out_dtype=None):
+    """Elementwise variant (N = 1, transition A_t given): all of x, A, B, C
+    are (B, L, D); h0 (B, D) fp32.  Returns (y, h_last)."""
+    Bz, L, Dm = x.shape
+    flags = A_DIRECT | (HAS_H0 if h0 is not None else 0) | (WANT_HLAST if want_h_last else 0)
+    out_dtype = out_dtype or x.dtype
+    key = ("direct", Bz, L, Dm, x.dtype, out_dtype, flags, x.device)
+    plan = _plan_for(key, lambda: Plan(Bz, L, Dm, 1, x.dtype, out_dtype, flags, x.device))
+    return plan.fwd(x, None, A, B, C, h0=h0)

@@ -1,0 +1,110 @@
+// scan_general.cu -- general-shape kernels of the selective scan.
+//
+// fwd_general_kernel: same arithmetic as the chunked TMA kernel for shapes
+// the fast path does not take (misaligned pointers, dim not a multiple of
+// the vector width, dstate outside {4, 8, 16}, seqlen = 0).  One thread owns
+// one channel (b, d) and all of its states and walks t = 0..L-1 in order
+// ("Selective Scan trong Mamba ...", "Selection pha vo convolution kernel
+// co dinh"); B_t / C_t reads are warp-uniform broadcasts.
+//
+// direct_kernel: the elementwise variant of "Selective (Data-Dependent) SSM
+// Scan" (steps 2-5): h = A_t*h + B_t*x_t, y_t = C_t*h after the update,
+// N = 1, every operand per (b, t, d).  It is bandwidth-bound (no
+// transcendental work): one thread per channel, loads coalesced along d.
+#include "device_common.cuh"
+#include "scan_params.h"
+
+namespace ssm {
+
+template <typename T>
+__device__ __forceinline__ float ldf(const void *base, size_t i) {
+  return to_f32(reinterpret_cast<const T *>(base)[i]);
+}
+
+template <typename InT, typename OutT, int NMAX>
+__global__ void __launch_bounds__(128) fwd_general_kernel(const GenericParams p) {
+  const long long chn = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (chn >= (long long)p.Bsz * p.D) return;
+  const int b = (int)(chn / p.D), d = (int)(chn % p.D);
+  const int N = p.N;
+  float h[NMAX], A2[NMAX];
+#pragma unroll
+  for (int n = 0; n < NMAX; ++n) {
+    const bool on = n < N;
+    h[n] = (on && p.has_h0) ? p.h0[((size_t)b * p.D + d) * N + n] : 0.f;
+    A2[n] = on ? p.A[(size_t)d * N + n] * kLog2e : 0.f;
+  }
+  const float Dd = p.has_D ? p.Dv[d] : 0.f;
+  const float bias = p.has_bias ? p.bias[d] : 0.f;
+  for (int t = 0; t < p.L; ++t) {
+    const size_t i = ((size_t)b * p.L + t) * p.D + d;
+    const size_t j = ((size_t)b * p.L + t) * N;
+    const float xv = ldf<InT>(p.x, i);
+    const float v = ldf<InT>(p.dt, i) + bias;
+    const float dlt = p.softplus ? softplus_f(v) : v;
+    const float dtx = dlt * xv;
+    float acc = 0.f;
+#pragma unroll
+    for (int n = 0; n < NMAX; ++n) {
+      if (n < N) {
+        const float a = ex2_approx(dlt * A2[n]);
+        h[n] = fmaf(a, h[n], dtx * ldf<InT>(p.B, j + n));
+        acc = fmaf(ldf<InT>(p.C, j + n), h[n], acc);
+      }
+    }
+    float yv = fmaf(Dd, xv, acc);
+    if (p.has_z) yv *= silu_f(ldf<InT>(p.z, i));
+    reinterpret_cast<OutT *>(p.y)[i] = from_f32<OutT>(yv);
+  }
+  if (p.want_hlast) {
+#pragma unroll
+    for (int n = 0; n < NMAX; ++n)
+      if (n < N) p.h_last[((size_t)b * p.D + d) * N + n] = h[n];
+  }
+}
+
+template <typename InT, typename OutT>
+static cudaError_t general_by_n(const GenericParams &p, cudaStream_t stream) {
+  const long long chans = (long long)p.Bsz * p.D;
+  if (chans == 0) return cudaSuccess;
+  const unsigned grid = (unsigned)((chans + 127) / 128);
+  if (p.N <= 4) fwd_general_kernel<InT, OutT, 4><<<grid, 128, 0, stream>>>(p);
+  else if (p.N <= 16) fwd_general_kernel<InT, OutT, 16><<<grid, 128, 0, stream>>>(p);
+  else fwd_general_kernel<InT, OutT, 64><<<grid, 128, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fwd_general(const GenericParams &p, cudaStream_t stream) {
+  if (!p.in_bf16 && !p.out_bf16) return general_by_n<float, float>(p, stream);
+  if (p.in_bf16 && p.out_bf16) return general_by_n<__nv_bfloat16, __nv_bfloat16>(p, stream);
+  if (p.in_bf16 && !p.out_bf16) return general_by_n<__nv_bfloat16, float>(p, stream);
+  return general_by_n<float, __nv_bfloat16>(p, stream);
+}
+
+template <typename InT, typename OutT>
+__global__ void __launch_bounds__(256) direct_kernel(const DirectParams p) {
+  const long long chn = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (chn >= (long long)p.Bsz * p.D) return;
+  const int b = (int)(chn / p.D), d = (int)(chn % p.D);
+  float h = p.h0 ? p.h0[(size_t)b * p.D + d] : 0.f;
+  for (int t = 0; t < p.L; ++t) {
+    const size_t i = ((size_t)b * p.L + t) * p.D + d;
+    h = fmaf(ldf<InT>(p.A, i), h, ldf<InT>(p.B, i) * ldf<InT>(p.x, i));
+    reinterpret_cast<OutT *>(p.y)[i] = from_f32<OutT>(ldf<InT>(p.C, i) * h);
+  }
+  if (p.h_last) p.h_last[(size_t)b * p.D + d] = h;
+}
+
+cudaError_t launch_direct(const DirectParams &p, cudaStream_t stream) {
+  const long long chans = (long long)p.Bsz * p.D;
+  if (chans == 0) return cudaSuccess;
+  const unsigned grid = (unsigned)((chans + 255) / 256);
+  if (!p.in_bf16 && !p.out_bf16) direct_kernel<float, float><<<grid, 256, 0, stream>>>(p);
+  else if (p.in_bf16 && p.out_bf16)
+    direct_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, 256, 0, stream>>>(p);
+  else if (p.in_bf16) direct_kernel<__nv_bfloat16, float><<<grid, 256, 0, stream>>>(p);
+  else direct_kernel<float, __nv_bfloat16><<<grid, 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace ssm

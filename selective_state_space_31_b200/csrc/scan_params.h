@@ -1,0 +1,95 @@
+// scan_params.h -- parameter blocks passed from the C-ABI layer to the
+// kernel launchers (internal to the library).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ssm {
+
+// Device-resident control block of one plan.  The last CTA of each chunked
+// launch resets `tile` and `done` and advances `epoch`, so consecutive calls
+// need no memset and work under stream capture.
+struct Control {
+  unsigned long long tile;  // next work item to claim
+  unsigned int done;        // CTAs finished in the current launch
+  unsigned int epoch;       // launch counter, tags the carry flags
+  int status;               // 0 or a timeout code, sticky until read
+  int pad[3];
+};
+
+struct FwdParams {
+  int Bsz, L, D, N;
+  int DT;       // channels per CTA (row tile)
+  int nDT;      // row tiles per batch
+  int Tseg;     // timesteps per work item
+  int nseg;     // work items per row
+  int rows;     // Bsz * nDT
+  long long total_items;
+  bool softplus, has_z, has_D, has_bias, has_h0, want_hlast;
+  const float *A;      // (D, N)
+  const float *Dv;     // (D) or null
+  const float *bias;   // (D) or null
+  const float *h0;     // (B, D, N) or null
+  float *h_last;       // (B, D, N) or null
+  float *ws_state;     // rows * DT * NS carried states
+  unsigned long long *ws_flags;  // rows * warps carry flags
+  Control *ctl;
+  unsigned long long timeout_ns;
+  long long drop_item;
+};
+
+struct TmaMaps {
+  CUtensorMap x, dt, z, B, C, y;
+};
+
+struct LaunchShape {
+  int lpc, warps, tt, stages, ns;
+  int grid;
+  size_t smem;
+};
+
+// Chunked TMA forward kernel (scan_fwd_tma.cu).
+cudaError_t launch_fwd_tma(int in_dtype, int out_dtype, const LaunchShape &ls,
+                           const TmaMaps &maps, const FwdParams &p, cudaStream_t stream);
+// Dynamic shared memory and per-SM residency of one chunked-kernel variant.
+cudaError_t fwd_tma_smem_and_occupancy(int in_dtype, int out_dtype, const LaunchShape &ls,
+                                       size_t *smem, int *blocks_per_sm);
+
+struct GenericParams {
+  int Bsz, L, D, N;
+  bool softplus, has_z, has_D, has_bias, has_h0, want_hlast;
+  int in_bf16, out_bf16;
+  const void *x, *dt, *z, *B, *C;
+  const float *A, *Dv, *bias, *h0;
+  void *y;
+  float *h_last;
+};
+// General forward kernel: any shape and alignment (scan_general.cu).
+cudaError_t launch_fwd_general(const GenericParams &p, cudaStream_t stream);
+
+struct DirectParams {
+  int Bsz, L, D;
+  int in_bf16, out_bf16;
+  const void *x, *A, *B, *C;
+  const float *h0;
+  void *y;
+  float *h_last;
+};
+// Elementwise (N = 1, A given per token) variant (scan_general.cu).
+cudaError_t launch_direct(const DirectParams &p, cudaStream_t stream);
+
+struct StepParams {
+  int Bsz, D, N;
+  bool softplus, has_z, has_D, has_bias;
+  int in_bf16, out_bf16;
+  const void *x, *dt, *z, *B, *C;
+  const float *A, *Dv, *bias;
+  float *state;
+  void *y;
+};
+// Decode step (scan_step.cu).
+cudaError_t launch_step(const StepParams &p, cudaStream_t stream);
+
+}  // namespace ssm

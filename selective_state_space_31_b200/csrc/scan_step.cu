@@ -1,0 +1,120 @@
+// scan_step.cu -- single-token decode step ("Selective Scan trong Mamba ...",
+// section "Selective Scan thay doi inference chuoi dai nhu the nao?": the
+// fixed-size state of a layer is updated once per new token, no re-scan).
+//
+// The step is bandwidth-bound: the (B, D, N) fp32 state is read and written
+// once per token (2 x 4 bytes per state) while the per-token inputs are
+// (B, D) and (B, N) vectors.  Threads own NPT consecutive states of one
+// channel (128-bit loads/stores of the state), TPC = N / NPT threads share a
+// channel and combine their partial readouts with xor shuffles.  The
+// per-channel scalars (x, delta, z) are re-read by the TPC threads of a
+// channel from the same cache line and softplus/silu are recomputed by each;
+// both are free next to the state traffic.
+#include "device_common.cuh"
+#include "scan_params.h"
+
+namespace ssm {
+
+template <typename T>
+__device__ __forceinline__ float ld1(const void *base, size_t i) {
+  return to_f32(reinterpret_cast<const T *>(base)[i]);
+}
+
+template <typename InT, typename OutT, int NPT, int TPC>
+__global__ void __launch_bounds__(256) step_kernel(const StepParams p) {
+  const long long gt = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long chn = gt / TPC;
+  const int q = (int)(gt % TPC);
+  const bool active = chn < (long long)p.Bsz * p.D;
+  const int N = NPT * TPC;
+  float acc = 0.f, xv = 0.f, zv = 0.f, Dd = 0.f;
+  int b = 0, d = 0;
+  float h[NPT];
+  float *sp = nullptr;
+  if (active) {
+    b = (int)(chn / p.D);
+    d = (int)(chn % p.D);
+    xv = ld1<InT>(p.x, (size_t)chn);
+    const float v = ld1<InT>(p.dt, (size_t)chn) + (p.has_bias ? __ldg(p.bias + d) : 0.f);
+    const float dlt = p.softplus ? softplus_f(v) : v;
+    const float dtx = dlt * xv;
+    if (p.has_z) zv = ld1<InT>(p.z, (size_t)chn);
+    if (p.has_D) Dd = __ldg(p.Dv + d);
+    sp = p.state + (size_t)chn * N + q * NPT;
+#pragma unroll
+    for (int i = 0; i < NPT; i += 4) {
+      const float4 s4 = __ldcs(reinterpret_cast<const float4 *>(sp + i));
+      h[i] = s4.x; h[i + 1] = s4.y; h[i + 2] = s4.z; h[i + 3] = s4.w;
+    }
+    const float *Ar = p.A + (size_t)d * N + q * NPT;
+    const size_t bc = (size_t)b * N + q * NPT;
+#pragma unroll
+    for (int n = 0; n < NPT; ++n) {
+      const float a = ex2_approx(dlt * (__ldg(Ar + n) * kLog2e));
+      h[n] = fmaf(a, h[n], dtx * ld1<InT>(p.B, bc + n));
+      acc = fmaf(ld1<InT>(p.C, bc + n), h[n], acc);
+    }
+#pragma unroll
+    for (int i = 0; i < NPT; i += 4)
+      __stcs(reinterpret_cast<float4 *>(sp + i), make_float4(h[i], h[i + 1], h[i + 2], h[i + 3]));
+  }
+#pragma unroll
+  for (int m = TPC / 2; m >= 1; m >>= 1) acc += __shfl_xor_sync(FULL_MASK, acc, m);
+  if (active && q == 0) {
+    float yv = fmaf(Dd, xv, acc);
+    if (p.has_z) yv *= silu_f(zv);
+    reinterpret_cast<OutT *>(p.y)[chn] = from_f32<OutT>(yv);
+  }
+}
+
+// Any dstate: one thread per channel, plain loads.
+template <typename InT, typename OutT>
+__global__ void __launch_bounds__(128) step_general_kernel(const StepParams p) {
+  const long long chn = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (chn >= (long long)p.Bsz * p.D) return;
+  const int b = (int)(chn / p.D), d = (int)(chn % p.D), N = p.N;
+  const float xv = ld1<InT>(p.x, (size_t)chn);
+  const float v = ld1<InT>(p.dt, (size_t)chn) + (p.has_bias ? p.bias[d] : 0.f);
+  const float dlt = p.softplus ? softplus_f(v) : v;
+  const float dtx = dlt * xv;
+  float acc = 0.f;
+  for (int n = 0; n < N; ++n) {
+    float *sp = p.state + (size_t)chn * N + n;
+    const float a = ex2_approx(dlt * (p.A[(size_t)d * N + n] * kLog2e));
+    const float hn = fmaf(a, *sp, dtx * ld1<InT>(p.B, (size_t)b * N + n));
+    *sp = hn;
+    acc = fmaf(ld1<InT>(p.C, (size_t)b * N + n), hn, acc);
+  }
+  float yv = fmaf(p.has_D ? p.Dv[d] : 0.f, xv, acc);
+  if (p.has_z) yv *= silu_f(ld1<InT>(p.z, (size_t)chn));
+  reinterpret_cast<OutT *>(p.y)[chn] = from_f32<OutT>(yv);
+}
+
+template <typename InT, typename OutT>
+static cudaError_t step_typed(const StepParams &p, bool vec_ok, cudaStream_t stream) {
+  const long long chans = (long long)p.Bsz * p.D;
+  if (chans == 0) return cudaSuccess;
+  auto grid_for = [&](int tpc) { return (unsigned)((chans * tpc + 255) / 256); };
+  if (vec_ok) {
+    switch (p.N) {
+      case 4: step_kernel<InT, OutT, 4, 1><<<grid_for(1), 256, 0, stream>>>(p); return cudaGetLastError();
+      case 8: step_kernel<InT, OutT, 8, 1><<<grid_for(1), 256, 0, stream>>>(p); return cudaGetLastError();
+      case 16: step_kernel<InT, OutT, 8, 2><<<grid_for(2), 256, 0, stream>>>(p); return cudaGetLastError();
+      case 32: step_kernel<InT, OutT, 8, 4><<<grid_for(4), 256, 0, stream>>>(p); return cudaGetLastError();
+      case 64: step_kernel<InT, OutT, 8, 8><<<grid_for(8), 256, 0, stream>>>(p); return cudaGetLastError();
+      default: break;
+    }
+  }
+  step_general_kernel<InT, OutT><<<(unsigned)((chans + 127) / 128), 128, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_step(const StepParams &p, cudaStream_t stream) {
+  const bool vec_ok = (reinterpret_cast<uintptr_t>(p.state) % 16) == 0;
+  if (!p.in_bf16 && !p.out_bf16) return step_typed<float, float>(p, vec_ok, stream);
+  if (p.in_bf16 && p.out_bf16) return step_typed<__nv_bfloat16, __nv_bfloat16>(p, vec_ok, stream);
+  if (p.in_bf16) return step_typed<__nv_bfloat16, float>(p, vec_ok, stream);
+  return step_typed<float, __nv_bfloat16>(p, vec_ok, stream);
+}
+
+}  // namespace ssm

@@ -1,0 +1,213 @@
+"""GPU parity of the CUDA library against the CPU oracle on seeded inputs of
+sizes the oracle finishes in seconds: several chunks and pipeline stages, a
+ragged tail, every kernel variant and option, edge cases."""
+import numpy as np
+import pytest
+import torch
+
+import gpu_util as gu
+from selective_state_space_31_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def _case(inp, cfg=None, expect_path=None):
+    plan = gu.make_plan(inp)
+    if cfg:
+        plan.set_config(**cfg)
+    info = plan.info()
+    if expect_path is not None:
+        assert info["path"] == expect_path, info
+    gy, gh = gu.run_gpu(inp, plan)
+    ry, rh = gu.run_oracle(inp)
+    gu.assert_parity(gy, ry, gh, rh, gu.TOL[inp.in_dtype if inp.out_dtype == inp.in_dtype
+                                             else "bf16"], f"{inp.name} {cfg} {info}")
+    assert plan.status() == 0
+    return plan
+
+
+def test_tiny_fp32_workload():
+    """The tiny fp32 case (B=1, L=512, D=64, N=16), fp32 tolerance 1e-5."""
+    _case(synth.tiny_fp32(), expect_path=0)
+
+
+@pytest.mark.parametrize("lpc", [1, 2, 4, 8])
+@pytest.mark.parametrize("warps", [2, 4, 8])
+def test_bf16_all_options_every_variant(lpc, warps):
+    """bf16 in/out, gate, skip, bias, h0; ragged L (not a multiple of the
+    stage) and chunks of one stage so the carry crosses many work items."""
+    inp = synth.make_fwd(3, 389, 64, 16, seed=21, has_h0=True)
+    if lpc == 1 and warps == 8:   # 256 bf16 channels x 3 stages does not fit in shared memory
+        from selective_state_space_31_b200 import binding as bnd
+        plan = gu.make_plan(inp)
+        with pytest.raises(bnd.SsmError):
+            plan.set_config(lanes_per_chan=lpc, warps_per_cta=warps, seg_len=64)
+        gy, gh = gu.run_gpu(inp, plan)   # the previous shape stays in force
+        ry, rh = gu.run_oracle(inp)
+        gu.assert_parity(gy, ry, gh, rh, gu.TOL["bf16"], "after rejected config")
+        return
+    _case(inp, dict(lanes_per_chan=lpc, warps_per_cta=warps, seg_len=64), expect_path=0)
+
+
+@pytest.mark.parametrize("seg_len,grid", [(64, 1), (128, 2), (192, 0), (0, 0), (64, 500)])
+def test_chunking_and_grid(seg_len, grid):
+    """A single CTA walking every item (grid=1), small grids that must wait
+    for predecessors, default and oversize grids."""
+    inp = synth.make_fwd(2, 1000, 128, 16, seed=22, has_h0=True)
+    _case(inp, dict(seg_len=seg_len, grid=grid), expect_path=0)
+
+
+@pytest.mark.parametrize("N", [4, 8, 16])
+def test_fp32_fast_path_dstate(N):
+    inp = synth.make_fwd(2, 200, 32, N, in_dtype="f32", seed=23, has_h0=True)
+    _case(inp, expect_path=0)
+
+
+@pytest.mark.parametrize("N", [8, 16])
+def test_bf16_in_fp32_out(N):
+    inp = synth.make_fwd(2, 257, 48, N, in_dtype="bf16", out_dtype="f32", seed=24)
+    _case(inp, expect_path=0)
+
+
+@pytest.mark.parametrize("shape,dt", [((2, 77, 37, 16), "bf16"), ((1, 130, 24, 1), "f32"),
+                                      ((2, 64, 16, 2), "f32"), ((1, 65, 40, 12), "bf16"),
+                                      ((1, 33, 8, 32), "f32"), ((1, 20, 8, 64), "bf16"),
+                                      ((2, 50, 16, 4), "bf16")])
+def test_general_path(shape, dt):
+    """Shapes the fast path does not take run on the general kernel."""
+    Bz, L, D, N = shape
+    inp = synth.make_fwd(Bz, L, D, N, in_dtype=dt, seed=25, has_h0=True)
+    _case(inp, expect_path=1)
+
+
+@pytest.mark.parametrize("softplus,z,bias,D,h0", [(False, False, False, False, False),
+                                                  (True, False, True, False, True),
+                                                  (False, True, False, True, False)])
+def test_option_combinations(softplus, z, bias, D, h0):
+    inp = synth.make_fwd(2, 150, 64, 16, seed=26, has_z=z, has_bias=bias, has_D=D, has_h0=h0,
+                         delta_softplus=softplus)
+    if not softplus:
+        inp.delta = np.abs(inp.delta) * np.float32(0.1)   # keep Delta positive and small
+        inp.delta = synth.round_bf16(inp.delta)
+    _case(inp, expect_path=0)
+
+
+def test_misaligned_pointers_take_general_kernel():
+    inp = synth.make_fwd(1, 100, 64, 16, seed=27)
+    plan = gu.make_plan(inp)
+    dev = gu.upload(inp)
+    # views that start 2 bytes into a buffer: valid, but not 16-byte aligned
+    for k in ("x", "delta", "z"):
+        buf = torch.empty(dev[k].numel() + 1, dtype=dev[k].dtype, device="cuda")
+        buf[1:].copy_(dev[k].reshape(-1))
+        dev[k] = buf[1:].view(dev[k].shape)
+        assert dev[k].data_ptr() % 16 != 0
+    gy, gh = gu.run_gpu(inp, plan, dev)
+    ry, rh = gu.run_oracle(inp)
+    gu.assert_parity(gy, ry, gh, rh, gu.TOL["bf16"], "misaligned")
+
+
+def test_zero_length_and_empty():
+    inp = synth.make_fwd(2, 0, 16, 16, in_dtype="f32", seed=28, has_h0=True)
+    gy, gh = gu.run_gpu(inp)
+    assert gy.shape == (2, 0, 16)
+    np.testing.assert_array_equal(gh, inp.h0.astype(np.float64))
+    inp = synth.make_fwd(0, 10, 16, 16, in_dtype="f32", seed=28)
+    gy, gh = gu.run_gpu(inp)
+    assert gy.shape == (0, 10, 16)
+
+
+def test_deterministic():
+    inp = synth.make_fwd(2, 700, 128, 16, seed=29, has_h0=True)
+    plan = gu.make_plan(inp)
+    plan.set_config(seg_len=64)
+    dev = gu.upload(inp)
+    a = gu.run_gpu(inp, plan, dev)
+    b = gu.run_gpu(inp, plan, dev)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+def test_h0_split_matches_full_run():
+    """Resuming from h_last of [0, k) reproduces the full run on [k, L)."""
+    inp = synth.make_fwd(2, 512, 64, 16, in_dtype="f32", seed=30, has_h0=True)
+    full_y, full_h = gu.run_gpu(inp)
+    k = 200
+    first = synth.make_fwd(2, k, 64, 16, in_dtype="f32", seed=30, has_h0=True)
+    for f in ("x", "delta", "z", "B", "C"):
+        setattr(first, f, getattr(inp, f)[:, :k].copy())
+    y1, h1 = gu.run_gpu(first)
+    second = synth.make_fwd(2, 512 - k, 64, 16, in_dtype="f32", seed=30, has_h0=True)
+    for f in ("x", "delta", "z", "B", "C"):
+        setattr(second, f, getattr(inp, f)[:, k:].copy())
+    second.h0 = h1.astype(np.float32)
+    y2, h2 = gu.run_gpu(second)
+    assert gu.normwise(np.concatenate([y1, y2], axis=1), full_y) < 1e-5
+    assert gu.normwise(h2, full_h) < 1e-5
+
+
+def test_elementwise_variant_page_example():
+    """The elementwise example's shapes (batch=2, seq_len=6, d=4, A in (0,1),
+    h0 = 0): output (2, 6, 4), values against the oracle."""
+    import oracle
+    from selective_state_space_31_b200 import binding as bnd
+    d = synth.make_direct(2, 6, 4, seed=31, has_h0=False)
+    dev = {k: gu.dev_tensor(d[k]) for k in ("x", "A", "B", "C")}
+    y, hl = bnd.direct(dev["x"], dev["A"], dev["B"], dev["C"])
+    assert tuple(y.shape) == (2, 6, 4)
+    ry, rh = oracle.get().direct(d["x"], d["A"], d["B"], d["C"])
+    gu.assert_parity(y.cpu().numpy(), ry, hl.cpu().numpy(), rh, 1e-5, "direct")
+
+
+@pytest.mark.parametrize("dt,a_zero", [("bf16", False), ("f32", True), ("f32", False)])
+def test_elementwise_variant(dt, a_zero):
+    import oracle
+    from selective_state_space_31_b200 import binding as bnd
+    d = synth.make_direct(3, 777, 96, seed=32, in_dtype=dt, a_zero=a_zero)
+    dev = {k: gu.dev_tensor(d[k], dt) for k in ("x", "A", "B", "C")}
+    h0 = gu.dev_tensor(d["h0"])
+    y, hl = bnd.direct(dev["x"], dev["A"], dev["B"], dev["C"], h0=h0)
+    ry, rh = oracle.get().direct(d["x"], d["A"], d["B"], d["C"], h0=d["h0"])
+    gu.assert_parity(y.float().cpu().numpy(), ry, hl.cpu().numpy(), rh, gu.TOL[dt], "direct")
+    if a_zero:   # memoryless: y_t = C_t B_t x_t
+        np.testing.assert_allclose(y.cpu().numpy(), d["C"] * d["B"] * d["x"], rtol=1e-6, atol=1e-6)
+
+
+@pytest.mark.parametrize("N,dt", [(16, "bf16"), (16, "f32"), (8, "bf16"), (4, "f32"),
+                                  (32, "f32"), (12, "f32")])
+def test_decode_steps_match_full_sequence(N, dt):
+    """L decode steps reproduce the oracle's full-sequence outputs and state."""
+    import oracle
+    from selective_state_space_31_b200 import binding as bnd
+    inp = synth.make_fwd(4, 40, 96, N, in_dtype=dt, seed=33, has_h0=True)
+    dev = gu.upload(inp)
+    state = dev["h0"].clone()
+    ys = []
+    for t in range(inp.L):
+        ys.append(bnd.step(state, dev["x"][:, t].contiguous(), dev["delta"][:, t].contiguous(),
+                           dev["A"], dev["B"][:, t].contiguous(), dev["C"][:, t].contiguous(),
+                           D=dev["D"], z=dev["z"][:, t].contiguous(),
+                           delta_bias=dev["delta_bias"]))
+    y = torch.stack(ys, dim=1).float().cpu().numpy()
+    ry, rh = oracle.get().fwd(inp.x, inp.delta, inp.A, inp.B, inp.C, D=inp.Dskip, z=inp.z,
+                              delta_bias=inp.delta_bias, h0=inp.h0)
+    gu.assert_parity(y, ry, state.cpu().numpy(), rh, gu.TOL[dt], f"decode N={N}")
+
+
+def test_timeout_is_reported_without_hanging():
+    """A work item that never hands its state on makes the next chunk's
+    bounded wait expire: the kernel records SSM_ERR_TIMEOUT and returns; the
+    plan stays usable and the next call is exact again."""
+    inp = synth.make_fwd(1, 512, 32, 16, seed=34)
+    plan = gu.make_plan(inp)
+    plan.set_config(seg_len=128)
+    info = plan.info()
+    assert info["items"] >= 2
+    plan.set_debug(wait_timeout_ns=50_000_000, drop_item=0)
+    dev = gu.upload(inp)
+    gu.run_gpu(inp, plan, dev)
+    assert plan.status() == 5  # SSM_ERR_TIMEOUT
+    plan.set_debug(0, -1)
+    gy, gh = gu.run_gpu(inp, plan, dev)
+    ry, rh = gu.run_oracle(inp)
+    gu.assert_parity(gy, ry, gh, rh, gu.TOL["bf16"], "after timeout")
+    assert plan.status() == 0
