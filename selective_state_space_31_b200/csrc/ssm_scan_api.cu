@@ -356,17 +356,25 @@ ssm_status ssm_scan_fwd(ssm_scan_plan *pl, const void *x, const void *delta,
   const ssm_scan_desc &d = pl->desc;
   const uint32_t f = d.flags;
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-  const bool empty = d.batch * d.seqlen * d.dim == 0;
-  if ((f & SSM_HAS_H0) != (h0 != nullptr)) return SSM_ERR_INVALID_ARG;
-  if ((f & SSM_WANT_HLAST) != (h_last != nullptr)) return SSM_ERR_INVALID_ARG;
-  if (!empty && (!x || !A || !B || !C || !y)) return SSM_ERR_INVALID_ARG;
+  // Pointer checks apply to tensors that have elements: a zero-size tensor
+  // may legitimately be passed as NULL.
+  const bool has_tokens = d.batch * d.seqlen * d.dim != 0;  // x, delta, z, y, B, C
+  const bool has_chans = d.batch * d.dim != 0;              // h0, h_last, A, D, bias
+  if (has_chans) {
+    if (((f & SSM_HAS_H0) != 0) != (h0 != nullptr)) return SSM_ERR_INVALID_ARG;
+    if (((f & SSM_WANT_HLAST) != 0) != (h_last != nullptr)) return SSM_ERR_INVALID_ARG;
+  }
+  if (has_tokens && (!x || !A || !B || !C || !y)) return SSM_ERR_INVALID_ARG;
   if (f & SSM_A_DIRECT) {
     if (delta || delta_bias || D || z) return SSM_ERR_INVALID_ARG;
   } else {
-    if (!empty && !delta) return SSM_ERR_INVALID_ARG;
-    if ((f & SSM_HAS_Z) != (z != nullptr)) return SSM_ERR_INVALID_ARG;
-    if ((f & SSM_HAS_D) != (D != nullptr)) return SSM_ERR_INVALID_ARG;
-    if ((f & SSM_HAS_DELTA_BIAS) != (delta_bias != nullptr)) return SSM_ERR_INVALID_ARG;
+    if (has_tokens && !delta) return SSM_ERR_INVALID_ARG;
+    if (has_tokens && (((f & SSM_HAS_Z) != 0) != (z != nullptr))) return SSM_ERR_INVALID_ARG;
+    if (has_chans) {
+      if (!A) return SSM_ERR_INVALID_ARG;
+      if (((f & SSM_HAS_D) != 0) != (D != nullptr)) return SSM_ERR_INVALID_ARG;
+      if (((f & SSM_HAS_DELTA_BIAS) != 0) != (delta_bias != nullptr)) return SSM_ERR_INVALID_ARG;
+    }
   }
   if (d.batch == 0 || d.dim == 0) return SSM_OK;
   DeviceGuard guard(pl->device);
@@ -438,9 +446,9 @@ ssm_status ssm_scan_step(ssm_scan_plan *pl, const void *x, const void *delta,
   if (f & SSM_A_DIRECT) return SSM_ERR_INVALID_ARG;
   const bool empty = d.batch * d.dim == 0;
   if (!empty && (!x || !delta || !A || !B || !C || !state || !y)) return SSM_ERR_INVALID_ARG;
-  if ((f & SSM_HAS_Z) != (z != nullptr)) return SSM_ERR_INVALID_ARG;
-  if ((f & SSM_HAS_D) != (D != nullptr)) return SSM_ERR_INVALID_ARG;
-  if ((f & SSM_HAS_DELTA_BIAS) != (delta_bias != nullptr)) return SSM_ERR_INVALID_ARG;
+  if (((f & SSM_HAS_Z) != 0) != (z != nullptr)) return SSM_ERR_INVALID_ARG;
+  if (((f & SSM_HAS_D) != 0) != (D != nullptr)) return SSM_ERR_INVALID_ARG;
+  if (((f & SSM_HAS_DELTA_BIAS) != 0) != (delta_bias != nullptr)) return SSM_ERR_INVALID_ARG;
   if (empty) return SSM_OK;
   DeviceGuard guard(pl->device);
   if (!guard.ok) return SSM_ERR_CUDA;
