@@ -158,6 +158,32 @@ SSM_API ssm_status ssm_scan_step(ssm_scan_plan *plan, const void *x, const void 
                          const void *C, const float *D, const void *z, float *state,
                          void *y, ssm_stream_t stream);
 
+/* Allocation-free forward pass.  The pages have no counterpart: this entry
+ * exists for callers that cannot allocate device memory (no cudaMalloc):
+ * code running under an allocator that owns all device memory up front,
+ * plugins that must not bypass their host's allocator, paths that must not
+ * risk the device synchronisation an allocation can cause.  Same operation,
+ * layouts and flags as ssm_scan_fwd (SSM_A_DIRECT excluded), on the CALLER'S
+ * CURRENT DEVICE, without a plan: the kernel's scratch (carried states,
+ * per-chunk flags, work counter) lives in a fixed 4 MiB device array inside
+ * the library, which every device that loads the library holds until the
+ * process exits.  Limits: the fast-path shape rules above (otherwise
+ * SSM_ERR_UNSUPPORTED; misaligned pointers give SSM_ERR_MISALIGNED), and
+ * about 4*dstate bytes of scratch per channel of batch*dim (rounded up to the
+ * kernel's channel tile): a problem whose scratch exceeds 4 MiB is rejected
+ * with SSM_ERR_UNSUPPORTED before anything is launched.  All calls share the
+ * scratch, so calls that overlap on the GPU (other streams or threads) race
+ * and give wrong results.  The first call on a device looks the scratch
+ * address up (cudaGetSymbolAddress); make that first call before any stream
+ * capture.  A device-side wait timeout is not reported by this entry point
+ * (outputs are then unspecified).  Nothing is allocated; inputs and outputs
+ * are the caller's device buffers. */
+SSM_API ssm_status ssm_scan_fwd_noalloc(const ssm_scan_desc *desc, const void *x,
+                                        const void *delta, const float *delta_bias,
+                                        const float *A, const void *B, const void *C,
+                                        const float *D, const void *z, const float *h0,
+                                        void *y, float *h_last, ssm_stream_t stream);
+
 /* Synchronise the plan's device, return the device-side status recorded by
  * the last calls (SSM_OK or SSM_ERR_TIMEOUT) and reset it to SSM_OK. */
 SSM_API ssm_status ssm_scan_get_status(ssm_scan_plan *plan);

@@ -1,0 +1,197 @@
+// scan_fwd_noalloc.cu -- ssm_scan_fwd_noalloc: the chunked forward scan for
+// callers that cannot allocate device memory.
+//
+// Some callers cannot call cudaMalloc at all: code that runs inside a
+// memory-capped or pre-partitioned allocator (an inference server that owns
+// every byte of the device up front), plugins loaded into a host process
+// whose allocator must not be bypassed, and code paths that must not
+// synchronise the device (cudaMalloc/cudaFree can).  They cannot create an
+// ssm_scan_plan, whose workspace is allocated by ssm_scan_create.  This entry
+// point runs the same chunked forward kernel with its scratch (the carried
+// states between chunks, the per-chunk flags and the work counter) in a
+// fixed file-scope device array instead, so it allocates nothing.
+//
+// The scratch array lives in every device that loads this library, until
+// the process exits: kNoAllocScratchBytes (4 MiB).  All calls share it and it
+// keeps the previous call's contents, so:
+//   * calls that overlap on the GPU (two streams, or two host threads) race
+//     on it and give wrong results: order them;
+//   * the work counters start at zero (static initialisation) and every
+//     launch of the kernel returns them to zero when its last CTA finishes;
+//     the per-chunk flags carry a launch counter, so stale flags from an
+//     earlier call never match.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/ssm_scan.h"
+#include "scan_params.h"
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
+constexpr size_t kCtlBytes = 256;
+constexpr int kMaxDevices = 64;
+constexpr int kTTna = 64;
+constexpr int kStagesNa = 3;
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch, looked up once per device with that
+// device current (host code must not use the symbol itself as an address).
+void *scratch_address(int device) {
+  static std::mutex mu;
+  static void *addr[kMaxDevices] = {};
+  if (device < 0 || device >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[device]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    addr[device] = p;
+  }
+  return addr[device];
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encoder_na() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool encode_na(CUtensorMap *m, ssm_dtype dt, const void *base, uint64_t d0, uint64_t d1,
+               uint64_t d2, uint32_t box0, uint32_t box1) {
+  auto enc = encoder_na();
+  if (!enc) return false;
+  const uint64_t es = dt == SSM_BF16 ? 2 : 4;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0 * es, d0 * d1 * es};
+  cuuint32_t box[3] = {box0, box1, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, dt == SSM_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+             3, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool al16(const void *p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+}  // namespace
+
+extern "C" SSM_API ssm_status ssm_scan_fwd_noalloc(
+    const ssm_scan_desc *desc, const void *x, const void *delta, const float *delta_bias,
+    const float *A, const void *B, const void *C, const float *D, const void *z,
+    const float *h0, void *y, float *h_last, ssm_stream_t stream_) {
+  if (!desc) return SSM_ERR_INVALID_ARG;
+  const ssm_scan_desc &d = *desc;
+  const uint32_t f = d.flags;
+  if (d.batch < 1 || d.seqlen < 1 || d.dim < 1) return SSM_ERR_INVALID_ARG;
+  if (d.batch > INT32_MAX || d.seqlen > INT32_MAX || d.dim > INT32_MAX) return SSM_ERR_UNSUPPORTED;
+  if ((d.in_dtype != SSM_F32 && d.in_dtype != SSM_BF16) ||
+      (d.out_dtype != SSM_F32 && d.out_dtype != SSM_BF16))
+    return SSM_ERR_INVALID_ARG;
+  constexpr uint32_t known = SSM_HAS_Z | SSM_HAS_D | SSM_DELTA_SOFTPLUS | SSM_HAS_DELTA_BIAS |
+                             SSM_HAS_H0 | SSM_WANT_HLAST;
+  if (f & ~known) return SSM_ERR_INVALID_ARG;
+  // the fast-path shape rules of the chunked kernel
+  const int ns = (int)d.dstate;
+  const size_t ei = d.in_dtype == SSM_BF16 ? 2 : 4, eo = d.out_dtype == SSM_BF16 ? 2 : 4;
+  if (ns != 4 && ns != 8 && ns != 16) return SSM_ERR_UNSUPPORTED;
+  if (ns == 4 && d.in_dtype == SSM_BF16) return SSM_ERR_UNSUPPORTED;
+  if (d.in_dtype == SSM_F32 && d.out_dtype == SSM_BF16) return SSM_ERR_UNSUPPORTED;
+  if ((d.dim * ei) % 16 || (ns * ei) % 16 || (d.dim * eo) % 16) return SSM_ERR_UNSUPPORTED;
+  if (!x || !delta || !A || !B || !C || !y) return SSM_ERR_INVALID_ARG;
+  if (((f & SSM_HAS_Z) != 0) != (z != nullptr) || ((f & SSM_HAS_D) != 0) != (D != nullptr) ||
+      ((f & SSM_HAS_DELTA_BIAS) != 0) != (delta_bias != nullptr) ||
+      ((f & SSM_HAS_H0) != 0) != (h0 != nullptr) ||
+      ((f & SSM_WANT_HLAST) != 0) != (h_last != nullptr))
+    return SSM_ERR_INVALID_ARG;
+  if (!al16(x) || !al16(delta) || !al16(z) || !al16(B) || !al16(C) || !al16(y))
+    return SSM_ERR_MISALIGNED;
+
+  int device = 0, num_sms = 0;
+  if (cudaGetDevice(&device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess) {
+    cudaGetLastError();
+    return SSM_ERR_CUDA;
+  }
+  // launch shape: same heuristic as a plan's default
+  const int64_t chans = d.batch * d.dim;
+  int lpc = 1;
+  while (lpc < 8 && lpc * 2 <= ns && chans * lpc / 32 < 8LL * num_sms) lpc *= 2;
+  const int warps = 4;
+  const int DT = warps * 32 / lpc;
+  if ((DT * (int)ei) % 16 || (DT * (int)eo) % 16) return SSM_ERR_UNSUPPORTED;
+  const int nDT = (int)((d.dim + DT - 1) / DT);
+  const int64_t rows = d.batch * nDT;
+  // scratch layout: [Control | flags rows*warps u64 | states rows*DT*N f32]
+  const size_t fl_bytes = (size_t)rows * warps * sizeof(unsigned long long);
+  const size_t st_off = (kCtlBytes + fl_bytes + 255) / 256 * 256;
+  const size_t need = st_off + (size_t)rows * DT * ns * sizeof(float);
+  if (need > kNoAllocScratchBytes) return SSM_ERR_UNSUPPORTED;  // beyond the fixed scratch
+
+  ssm::LaunchShape ls{lpc, warps, kTTna, kStagesNa, ns, 0, 0};
+  int bps = 0;
+  size_t smem = 0;
+  if (ssm::fwd_tma_smem_and_occupancy((int)d.in_dtype, (int)d.out_dtype, ls, &smem, &bps) !=
+          cudaSuccess ||
+      bps < 1) {
+    cudaGetLastError();
+    return SSM_ERR_UNSUPPORTED;
+  }
+  const int64_t grid = std::min<int64_t>((int64_t)bps * num_sms, rows);
+  const int64_t tiles = (d.seqlen + kTTna - 1) / kTTna;
+  int64_t nseg = std::min(std::max<int64_t>(1, (8 * grid + rows - 1) / rows), tiles);
+  const int Tseg = (int)(((d.seqlen + nseg - 1) / nseg + kTTna - 1) / kTTna * kTTna);
+  nseg = (d.seqlen + Tseg - 1) / Tseg;
+  if (rows * nseg > INT32_MAX) return SSM_ERR_UNSUPPORTED;
+  ls.grid = (int)std::max<int64_t>(1, std::min<int64_t>(grid, rows * nseg));
+  ls.smem = smem;
+
+  unsigned char *base = static_cast<unsigned char *>(scratch_address(device));
+  if (!base) return SSM_ERR_CUDA;
+
+  ssm::TmaMaps maps;
+  const uint64_t Bn = d.batch, L = d.seqlen, Dm = d.dim, N = d.dstate;
+  if (!encode_na(&maps.x, d.in_dtype, x, Dm, L, Bn, DT, kTTna) ||
+      !encode_na(&maps.dt, d.in_dtype, delta, Dm, L, Bn, DT, kTTna) ||
+      !encode_na(&maps.z, d.in_dtype, z ? z : x, Dm, L, Bn, DT, kTTna) ||
+      !encode_na(&maps.B, d.in_dtype, B, N, L, Bn, (uint32_t)N, kTTna) ||
+      !encode_na(&maps.C, d.in_dtype, C, N, L, Bn, (uint32_t)N, kTTna) ||
+      !encode_na(&maps.y, d.out_dtype, y, Dm, L, Bn, DT, kTTna))
+    return SSM_ERR_CUDA;
+
+  ssm::FwdParams p{};
+  p.Bsz = (int)d.batch; p.L = (int)d.seqlen; p.D = (int)d.dim; p.N = ns;
+  p.DT = DT; p.nDT = nDT; p.Tseg = Tseg; p.nseg = (int)nseg;
+  p.rows = (int)rows; p.total_items = rows * nseg;
+  p.softplus = (f & SSM_DELTA_SOFTPLUS) != 0;
+  p.has_z = (f & SSM_HAS_Z) != 0;
+  p.has_D = (f & SSM_HAS_D) != 0;
+  p.has_bias = (f & SSM_HAS_DELTA_BIAS) != 0;
+  p.has_h0 = (f & SSM_HAS_H0) != 0;
+  p.want_hlast = (f & SSM_WANT_HLAST) != 0;
+  p.A = A; p.Dv = D; p.bias = delta_bias; p.h0 = h0; p.h_last = h_last;
+  p.ctl = reinterpret_cast<ssm::Control *>(base);
+  p.ws_flags = reinterpret_cast<unsigned long long *>(base + kCtlBytes);
+  p.ws_state = reinterpret_cast<float *>(base + st_off);
+  p.timeout_ns = 2000000000ull;
+  p.drop_item = -1;
+  const cudaError_t e = ssm::launch_fwd_tma((int)d.in_dtype, (int)d.out_dtype, ls, maps, p,
+                                            reinterpret_cast<cudaStream_t>(stream_));
+  return e == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
