@@ -45,15 +45,16 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mamba130m_layer",
-                    choices=["tiny_fp32", "mamba130m_layer", "mamba1p4b_layer", "long_seq"])
+                    choices=["tiny_fp32", "mamba130m_layer", "mamba1p4b_layer", "long_seq",
+                             "decode"])
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--cpu-budget-s", type=float, default=60.0,
                     help="CPU seconds (summed over threads) for the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--lpc", type=int, default=0)
     ap.add_argument("--warps", type=int, default=0)
-    ap.add_argument("--seg-len", type=int, default=0)
     ap.add_argument("--grid", type=int, default=0)
+    ap.add_argument("--tile-t", type=int, default=0)
     return ap.parse_args()
 
 
@@ -103,6 +104,28 @@ def profiled_traffic(workload):
         return int(float(kv["dram_bytes_per_launch"]))
     except (KeyError, ValueError):
         return None
+
+
+# ---------------------------------------------------------------------------
+# multi-GPU replicas: slowest rank decides, work adds up
+# ---------------------------------------------------------------------------
+
+def max_over_ranks(values, device=None):
+    """Max of each value over all ranks (identity when not distributed).
+    Works with NCCL (CUDA tensors) and gloo (CPU tensors)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def replica_throughput(updates_per_rank, world, ms_per_step_max):
+    """Whole-job state-updates/s: every rank runs its own replica of the
+    workload, so the work adds up and the slowest rank's time counts."""
+    return updates_per_rank * world / (ms_per_step_max * 1e-3)
 
 
 # ---------------------------------------------------------------------------
@@ -251,8 +274,8 @@ def run_ours(args, rank, world, device):
                           delta_softplus=inp.delta_softplus, want_h_last=True)
     plan = bnd.Plan(inp.Bsz, inp.L, inp.D, inp.N, tdt[inp.in_dtype], tdt[inp.out_dtype], flags,
                     device)
-    if args.lpc or args.warps or args.seg_len or args.grid:
-        plan.set_config(args.lpc, args.warps, args.seg_len, args.grid)
+    if args.lpc or args.warps or args.grid or args.tile_t:
+        plan.set_config(args.lpc, args.warps, args.grid, args.tile_t)
     outs = [(torch.empty((inp.Bsz, inp.L, inp.D), dtype=tdt[inp.out_dtype], device=device),
              torch.empty((inp.Bsz, inp.D, inp.N), dtype=torch.float32, device=device))
             for _ in range(2)]
@@ -292,14 +315,11 @@ def run_ours(args, rank, world, device):
     st = plan.status()
     if st != 0:
         raise RuntimeError(f"device status {st} after the timed region")
-    if world > 1:
-        t = torch.tensor([total_ms, kern_ms], device=device, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms, kern_ms = t.tolist()
+    total_ms, kern_ms = max_over_ranks([total_ms, kern_ms], device)
     ms_per_step = total_ms / K
 
     counts = algorithmic_counts(inp)
-    value = counts["updates"] * world / (ms_per_step * 1e-3)
+    value = replica_throughput(counts["updates"], world, ms_per_step)
 
     # e2e through the public API: pinned host inputs copied in, y/h_last copied out
     e2e = None
@@ -340,11 +360,8 @@ def run_ours(args, rank, world, device):
         b.record(stream)
         torch.cuda.synchronize(device)
         e_ms = a.elapsed_time(b) / args.e2e_steps
-        if world > 1:
-            t = torch.tensor([e_ms], device=device, dtype=torch.float64)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e_ms = t.item()
-        e2e = {"value": counts["updates"] * world / (e_ms * 1e-3), "unit": "state-updates/s",
+        e_ms = max_over_ranks([e_ms], device)[0]
+        e2e = {"value": replica_throughput(counts["updates"], world, e_ms), "unit": "state-updates/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms,
                "steps": args.e2e_steps}
 
@@ -381,8 +398,8 @@ def run_ours(args, rank, world, device):
                    "l2": "two input sets alternate between steps (2x inputs > 126 MB L2)",
                    "parallelism": f"replicas x{world}",
                    "launch": {k: info[k] for k in ("lanes_per_chan", "warps_per_cta",
-                                                    "seg_len", "chans_per_cta", "grid",
-                                                    "items")}},
+                                                    "tile_t", "chans_per_cta", "grid",
+                                                    "rows", "units")}},
         "roofline": {"bound": "alu", "achieved": achieved_mufu / 1e9, "peak": peak_mufu / 1e9,
                      "unit": "G MUFU-op/s (ex2, lg2, rcp)", "frac": achieved_mufu / peak_mufu,
                      "traffic": traffic,
@@ -407,14 +424,177 @@ def run_ours(args, rank, world, device):
 
 
 # ---------------------------------------------------------------------------
+# decode: one token step over a (256, 5120, 16) fp32 state
+# ---------------------------------------------------------------------------
+
+def run_decode(args, rank, world, device):
+    """One step = one ssm_scan_step over the whole (B, D, N) state.  Three
+    independent states (3 x 84 MB, more than the 126 MB L2) take turns and
+    32 distinct token inputs rotate, so every step streams its state from
+    HBM.  96 steps (all combinations) are captured in one CUDA graph."""
+    import numpy as np
+    import torch
+
+    from selective_state_space_31_b200 import binding as bnd
+    from selective_state_space_31_b200 import synth
+
+    torch.cuda.set_device(device)
+    dec = synth.make_decode(steps=32, seed=4 + rank)
+    bf, f32 = torch.bfloat16, torch.float32
+    up = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a)).to(device, dt)
+    toks = [dec.token(t) for t in range(32)]
+    tin = [{k: up(v, bf) for k, v in tk.items()} for tk in toks]
+    A, D, bias = up(dec.A, f32), up(dec.Dskip, f32), up(dec.delta_bias, f32)
+    states = [up(dec.h0, f32) for _ in range(3)]
+    ys = [torch.empty((dec.Bsz, dec.D), dtype=bf, device=device) for _ in range(3)]
+    flags = bnd.flags_for(z=1, D=1, delta_bias=1, delta_softplus=True, want_h_last=False)
+    plan = bnd.Plan(dec.Bsz, 1, dec.D, dec.N, bf, bf, flags, device)
+
+    def step(i):
+        t, s = tin[i % 32], i % 3
+        plan.step(states[s], t["x"], t["delta"], A, t["B"], t["C"], D=D, z=t["z"],
+                  delta_bias=bias, y=ys[s])
+
+    G = 96
+    stream = torch.cuda.Stream(device)
+    with torch.cuda.stream(stream):
+        for i in range(G):   # warm-up outside capture (also loads the module)
+            step(i)
+    torch.cuda.synchronize(device)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(G):
+            step(i)
+    reps = max(1, args.steps // G)
+    for _ in range(max(1, args.warmup // G)):
+        graph.replay()
+    torch.cuda.synchronize(device)
+    sampler = ClockSampler(device)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    sampler.start()
+    a.record(torch.cuda.current_stream(device))
+    for _ in range(reps):
+        graph.replay()
+    b.record(torch.cuda.current_stream(device))
+    torch.cuda.synchronize(device)
+    sampler.stop()
+    if world > 1:
+        torch.distributed.barrier()
+    steps = reps * G
+    ms_per_step = max_over_ranks([a.elapsed_time(b) / steps], device)[0]
+    upd = dec.Bsz * dec.D * dec.N
+    Bz, Dm, N = dec.Bsz, dec.D, dec.N
+    byt = 8 * Bz * Dm * N + 3 * 2 * Bz * Dm + 2 * 2 * Bz * N + 2 * Bz * Dm + 4 * Dm * N + 8 * Dm
+    peaks = {}
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peaks = json.load(f)
+    except Exception:
+        pass
+    hbm_peak = peaks.get("hbm_gbs", 6650.0)
+    gbs = byt / (ms_per_step * 1e-3) / 1e9
+    # e2e: a token's inputs come from pinned host memory, y goes back
+    host = [{k: v.to(bf).cpu().pin_memory() for k, v in t.items()} for t in tin[:4]]
+    y_h = torch.empty((Bz, Dm), dtype=bf).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host[0].values())
+    d2h = y_h.numel() * y_h.element_size()
+    s0 = torch.cuda.current_stream(device)
+    e1, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    E = max(8, min(args.e2e_steps, 200))
+    e1.record(s0)
+    for i in range(E):
+        for k, v in host[i % 4].items():
+            tin[0][k].copy_(v, non_blocking=True)
+        step(0)
+        y_h.copy_(ys[0], non_blocking=True)
+    e2.record(s0)
+    torch.cuda.synchronize(device)
+    e_ms = max_over_ranks([e1.elapsed_time(e2) / E], device)[0]
+    res = {
+        "metric": "selective-scan state-updates/s (B*L*D*N)",
+        "value": replica_throughput(upd, world, ms_per_step),
+        "unit": "state-updates/s", "n_gpus": world, "steps": steps,
+        "warmup": max(1, args.warmup // G) * G, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded normal draws, shapes and distributions of the workload)",
+        "config": {"workload": "decode", "batch": Bz, "dim": Dm, "dstate": N,
+                   "step": "one token for the whole state", "graph": f"{G} steps per CUDA graph",
+                   "l2": "3 independent 84 MB states take turns (252 MB > 126 MB L2)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": gbs / hbm_peak, "traffic": None, "algorithmic_bytes": byt},
+        "gpu_launches": steps,
+        "clocks": sampler.summary(),
+        "e2e": {"value": replica_throughput(upd, world, e_ms), "unit": "state-updates/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms},
+    }
+    del graph
+    plan.close()
+    return res
+
+
+# ---------------------------------------------------------------------------
 # reference arm: the CPU oracle on a bounded sample of the same workload
 # ---------------------------------------------------------------------------
 
+def oracle_decode_rate(dec, budget_cpu_s, threads):
+    """Time the fp64 oracle's decode step on the first channels of the
+    (B, D, N) state, sized to the CPU-seconds budget, on all host cores."""
+    import concurrent.futures as cf
+
+    import oracle
+    orc = oracle.get()
+    tok = dec.token(0)
+    t0 = time.perf_counter()
+    orc.step(dec.h0[:1, :64], tok["x"][:1, :64], tok["delta"][:1, :64], dec.A[:64], tok["B"][:1],
+             tok["C"][:1], D=dec.Dskip[:64], z=tok["z"][:1, :64], delta_bias=dec.delta_bias[:64])
+    per_chan = max((time.perf_counter() - t0) / 64, 1e-9)
+    n_b = int(min(dec.Bsz, max(threads, budget_cpu_s / per_chan / dec.D)))
+
+    def work(b):
+        orc.step(dec.h0[b:b + 1], tok["x"][b:b + 1], tok["delta"][b:b + 1], dec.A, tok["B"][b:b + 1],
+                 tok["C"][b:b + 1], D=dec.Dskip, z=tok["z"][b:b + 1], delta_bias=dec.delta_bias)
+
+    t0 = time.perf_counter()
+    with cf.ThreadPoolExecutor(max_workers=threads) as ex:
+        list(ex.map(work, range(n_b)))
+    dt = time.perf_counter() - t0
+    upd = n_b * dec.D * dec.N
+    return upd / dt, upd, (f"{n_b} of {dec.Bsz} batch rows of one decode step "
+                           f"(D={dec.D}, N={dec.N}), fp64 oracle, {threads} threads")
+
+
 def run_reference(args):
     from selective_state_space_31_b200 import synth
+    if args.workload == "decode":
+        dec = synth.make_decode(steps=1)
+        threads = os.cpu_count() or 1
+        per_step = args.cpu_budget_s * threads / max(1, args.steps + args.warmup)
+        for _ in range(args.warmup):
+            oracle_decode_rate(dec, per_step, threads)
+        upd_total, t_total, desc = 0, 0.0, ""
+        for _ in range(args.steps):
+            rate, upd, desc = oracle_decode_rate(dec, per_step, threads)
+            upd_total += upd
+            t_total += upd / rate
+        value = upd_total / t_total
+        return {"impl": "reference", "metric": "selective-scan state-updates/s (B*L*D*N)",
+                "value": value, "unit": "state-updates/s", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": t_total / max(1, args.steps) * 1e3, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic (seeded normal draws, shapes and distributions of the workload)",
+                "config": {"workload": "decode", "batch": dec.Bsz, "dim": dec.D, "dstate": dec.N},
+                "cpu_baseline": {"value": value, "unit": "state-updates/s", "cores": threads,
+                                 "kind": "oracle", "sample": "per step: " + desc},
+                "e2e": {"value": value, "unit": "state-updates/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
     inp = synth.FWD_WORKLOADS[args.workload]()
     threads = os.cpu_count() or 1
-    total_budget = 90.0 * threads   # CPU-seconds for warmup + timed steps
+    total_budget = args.cpu_budget_s * threads   # CPU-seconds for warmup + timed steps
     per_step = total_budget / max(1, args.steps + args.warmup)
     for _ in range(args.warmup):
         oracle_sample_rate(inp, per_step, threads)
@@ -465,7 +645,7 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=device)
     try:
-        res = run_ours(args, rank, world, device)
+        res = (run_decode if args.workload == "decode" else run_ours)(args, rank, world, device)
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:

@@ -45,9 +45,9 @@
  * workspace.  y must not alias any input; only `state` is updated in place.
  *
  * Errors: argument checks are synchronous and launch nothing.  A failed
- * launch returns SSM_ERR_CUDA.  The only device-side wait (a chunk waiting
- * for the carried state of the previous chunk of the same channels) is
- * bounded; if it expires the kernel records SSM_ERR_TIMEOUT, finishes without
+ * launch returns SSM_ERR_CUDA.  Device-side waits (a CTA waiting for the
+ * carried state of the earlier part of a row that another CTA ran, and for
+ * its own TMA loads) are bounded; if it expires the kernel records SSM_ERR_TIMEOUT, finishes without
  * hanging, and y/h_last of that call are unspecified.  ssm_scan_get_status
  * synchronises the device and returns (and clears) that record.
  *
@@ -107,16 +107,16 @@ typedef struct ssm_scan_plan ssm_scan_plan;
 
 /* Plan details chosen by ssm_scan_create (read-only; for tests and tuning). */
 typedef struct {
-  int path;            /* 0 = TMA chunked kernel, 1 = general kernel, 2 = elementwise, 3 = step */
+  int path;            /* 0 = fused chunked kernel, 1 = general kernel, 2 = elementwise */
   int lanes_per_chan;  /* lanes sharing one channel's dstate states */
   int warps_per_cta;
-  int tile_t;          /* timesteps per pipeline stage */
+  int tile_t;          /* tokens per pipeline stage (one work unit) */
   int stages;          /* pipeline depth */
-  int seg_len;         /* timesteps per work item (chunk) */
-  int chans_per_cta;
-  int grid;            /* persistent CTAs launched */
+  int stages_per_row;  /* work units per row = ceil(seqlen / tile_t) */
+  int chans_per_cta;   /* channels per row tile */
+  int grid;            /* CTAs launched (each takes an equal share of the units) */
   int64_t rows;        /* independent (batch, channel-tile) rows */
-  int64_t items;       /* work items = rows * chunks */
+  int64_t units;       /* work units = rows * stages_per_row */
   size_t smem_bytes;
   size_t workspace_bytes;
 } ssm_scan_info;
@@ -124,9 +124,9 @@ typedef struct {
 /* Optional overrides of the launch shape (0 = keep the default). */
 typedef struct {
   int lanes_per_chan; /* 1, 2, 4, 8 (<= dstate) */
-  int warps_per_cta;  /* 2, 4, 8 */
-  int seg_len;        /* multiple of the stage length */
-  int grid;           /* persistent CTAs (clamped to what fits on the device) */
+  int warps_per_cta;  /* 2 or 4 */
+  int grid;           /* CTAs (clamped to what is co-resident on the device) */
+  int tile_t;         /* tokens per pipeline stage: 16, 32 or 64 */
 } ssm_scan_config;
 
 /* Create a plan for one problem shape on `device`; allocates the workspace.
@@ -196,10 +196,11 @@ SSM_API ssm_status ssm_scan_get_info(const ssm_scan_plan *plan, ssm_scan_info *i
 SSM_API ssm_status ssm_scan_set_config(ssm_scan_plan *plan, const ssm_scan_config *cfg);
 
 /* Test hook: set the bound of device-side waits (nanoseconds, 0 = default
- * of 2 s) and make work item `drop_item` (-1 = none) skip publishing its
- * carried state, so the next chunk's bounded wait expires.  Used to test
- * the timeout path without hanging the device. */
-SSM_API ssm_status ssm_scan_set_debug(ssm_scan_plan *plan, uint64_t wait_timeout_ns, int64_t drop_item);
+ * of 2 s) and make the run of work units that ends at unit `drop_unit`
+ * (-1 = none) skip handing on its carried state, so the CTA that continues
+ * that row waits until the bound expires.  Used to test the timeout path
+ * without hanging the device. */
+SSM_API ssm_status ssm_scan_set_debug(ssm_scan_plan *plan, uint64_t wait_timeout_ns, int64_t drop_unit);
 
 /* Static description of a status code. */
 SSM_API const char *ssm_status_string(ssm_status s);

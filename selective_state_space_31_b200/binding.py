@@ -41,8 +41,8 @@ class Desc(ctypes.Structure):
 class Info(ctypes.Structure):
     _fields_ = [("path", ctypes.c_int), ("lanes_per_chan", ctypes.c_int),
                 ("warps_per_cta", ctypes.c_int), ("tile_t", ctypes.c_int), ("stages", ctypes.c_int),
-                ("seg_len", ctypes.c_int), ("chans_per_cta", ctypes.c_int), ("grid", ctypes.c_int),
-                ("rows", ctypes.c_int64), ("items", ctypes.c_int64),
+                ("stages_per_row", ctypes.c_int), ("chans_per_cta", ctypes.c_int),
+                ("grid", ctypes.c_int), ("rows", ctypes.c_int64), ("units", ctypes.c_int64),
                 ("smem_bytes", ctypes.c_size_t), ("workspace_bytes", ctypes.c_size_t)]
 
     def as_dict(self):
@@ -51,7 +51,7 @@ class Info(ctypes.Structure):
 
 class Config(ctypes.Structure):
     _fields_ = [("lanes_per_chan", ctypes.c_int), ("warps_per_cta", ctypes.c_int),
-                ("seg_len", ctypes.c_int), ("grid", ctypes.c_int)]
+                ("grid", ctypes.c_int), ("tile_t", ctypes.c_int)]
 
 
 _lib = None
@@ -162,12 +162,12 @@ class Plan:
         _check(self._lib.ssm_scan_get_info(self._h, ctypes.byref(i)), "ssm_scan_get_info")
         return i.as_dict()
 
-    def set_config(self, lanes_per_chan=0, warps_per_cta=0, seg_len=0, grid=0):
-        c = Config(lanes_per_chan, warps_per_cta, seg_len, grid)
+    def set_config(self, lanes_per_chan=0, warps_per_cta=0, grid=0, tile_t=0):
+        c = Config(lanes_per_chan, warps_per_cta, grid, tile_t)
         _check(self._lib.ssm_scan_set_config(self._h, ctypes.byref(c)), "ssm_scan_set_config")
 
-    def set_debug(self, wait_timeout_ns=0, drop_item=-1):
-        _check(self._lib.ssm_scan_set_debug(self._h, int(wait_timeout_ns), int(drop_item)),
+    def set_debug(self, wait_timeout_ns=0, drop_unit=-1):
+        _check(self._lib.ssm_scan_set_debug(self._h, int(wait_timeout_ns), int(drop_unit)),
                "ssm_scan_set_debug")
 
     def status(self) -> int:

@@ -25,14 +25,85 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// softplus(v) = log(1 + e^v) = max(v, 0) + log1p(e^{-|v|}); log1pf keeps the
-// small-Delta end accurate (the rounding of 1 + e^{-|v|} is never taken).
+// --- packed fp32 pairs (sm_100 f32x2 instructions: two lanes of fp32 work per
+// issued instruction; round-to-nearest like the scalar forms) -------------
+
+// float2 is an 8-byte aligned pair: pass it to PTX as one 64-bit register.
+#define SSM_U64(v) (*reinterpret_cast<unsigned long long *>(&(v)))
+#define SSM_CU64(v) (*reinterpret_cast<const unsigned long long *>(&(v)))
+
+// a * b + c, elementwise on the pair
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(SSM_U64(d)) : "l"(SSM_CU64(a)), "l"(SSM_CU64(b)), "l"(SSM_CU64(c)));
+  return d;
+}
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  float2 d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(SSM_U64(d)) : "l"(SSM_CU64(a)), "l"(SSM_CU64(b)));
+  return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(SSM_U64(d)) : "l"(SSM_CU64(a)), "l"(SSM_CU64(b)));
+  return d;
+}
+
+// log1p(u) for u in [0, 1] as u * P(u), P of degree 8 fitted to log1p(u)/u
+// by least squares on Chebyshev nodes (csrc/fit_log1p.py derives and checks
+// the coefficients: max relative error 1.9e-7 in float32).  Never forms
+// 1 + u, so small u keeps full relative accuracy.
+__device__ __forceinline__ float log1p_unit(float u) {
+  float p = 0.00525345793f;
+  p = fmaf(p, u, -0.0295885075f);
+  p = fmaf(p, u, 0.0783616677f);
+  p = fmaf(p, u, -0.136747703f);
+  p = fmaf(p, u, 0.191114306f);
+  p = fmaf(p, u, -0.248443693f);
+  p = fmaf(p, u, 0.333192706f);
+  p = fmaf(p, u, -0.499995023f);
+  p = fmaf(p, u, 1.0f);
+  return u * p;
+}
+
+// 1/x on the special-function unit (rcp.approx, flush-to-zero).
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// softplus(v) = log(1 + e^v) = max(v, 0) + log1p(e^{-|v|}), e^{-|v|} in (0, 1]
+// on the special-function unit, log1p by the fitted polynomial.
 __device__ __forceinline__ float softplus_f(float v) {
-  return fmaxf(v, 0.f) + log1pf(__expf(-fabsf(v)));
+  return fmaxf(v, 0.f) + log1p_unit(ex2_approx(-fabsf(v) * kLog2e));
 }
 
 // silu(z) = z * sigmoid(z) = z / (1 + e^{-z}).
 __device__ __forceinline__ float silu_f(float z) { return __fdividef(z, 1.f + __expf(-z)); }
+
+// The same two functions on a pair of channels, with packed arithmetic.
+__device__ __forceinline__ float2 log1p_unit2(float2 u) {
+  float2 p = make_float2(0.00525345793f, 0.00525345793f);
+  p = ffma2(p, u, make_float2(-0.0295885075f, -0.0295885075f));
+  p = ffma2(p, u, make_float2(0.0783616677f, 0.0783616677f));
+  p = ffma2(p, u, make_float2(-0.136747703f, -0.136747703f));
+  p = ffma2(p, u, make_float2(0.191114306f, 0.191114306f));
+  p = ffma2(p, u, make_float2(-0.248443693f, -0.248443693f));
+  p = ffma2(p, u, make_float2(0.333192706f, 0.333192706f));
+  p = ffma2(p, u, make_float2(-0.499995023f, -0.499995023f));
+  p = ffma2(p, u, make_float2(1.0f, 1.0f));
+  return fmul2(u, p);
+}
+__device__ __forceinline__ float2 softplus_f2(float2 v) {
+  const float2 u = make_float2(ex2_approx(-fabsf(v.x) * kLog2e), ex2_approx(-fabsf(v.y) * kLog2e));
+  return fadd2(make_float2(fmaxf(v.x, 0.f), fmaxf(v.y, 0.f)), log1p_unit2(u));
+}
+__device__ __forceinline__ float2 silu_f2(float2 z) {
+  const float2 e = make_float2(ex2_approx(-z.x * kLog2e), ex2_approx(-z.y * kLog2e));
+  const float2 den = fadd2(e, make_float2(1.f, 1.f));
+  return fmul2(z, make_float2(rcp_approx(den.x), rcp_approx(den.y)));
+}
 
 template <typename T> __device__ __forceinline__ float to_f32(T v);
 template <> __device__ __forceinline__ float to_f32<float>(float v) { return v; }

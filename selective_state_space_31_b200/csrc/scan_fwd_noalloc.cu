@@ -16,10 +16,10 @@
 // keeps the previous call's contents, so:
 //   * calls that overlap on the GPU (two streams, or two host threads) race
 //     on it and give wrong results: order them;
-//   * the work counters start at zero (static initialisation) and every
-//     launch of the kernel returns them to zero when its last CTA finishes;
-//     the per-chunk flags carry a launch counter, so stale flags from an
-//     earlier call never match.
+//   * the finished-CTA counter starts at zero (static initialisation) and
+//     every launch returns it to zero when its last CTA finishes; the
+//     per-chunk flags carry a launch counter that the same CTA advances, so
+//     stale flags from an earlier call never match.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -28,7 +28,7 @@
 #include <cstdint>
 #include <mutex>
 
-#include "../../include/ssm_scan.h"
+#include "ssm_scan.h"
 #include "scan_params.h"
 
 namespace {
@@ -36,8 +36,8 @@ namespace {
 constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
 constexpr size_t kCtlBytes = 256;
 constexpr int kMaxDevices = 64;
-constexpr int kTTna = 64;
-constexpr int kStagesNa = 3;
+constexpr int kTTna = 16;
+constexpr int kStagesNa = 2;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
@@ -129,38 +129,48 @@ extern "C" SSM_API ssm_status ssm_scan_fwd_noalloc(
     cudaGetLastError();
     return SSM_ERR_CUDA;
   }
-  // launch shape: same heuristic as a plan's default
-  const int64_t chans = d.batch * d.dim;
-  int lpc = 1;
-  while (lpc < 8 && lpc * 2 <= ns && chans * lpc / 32 < 8LL * num_sms) lpc *= 2;
-  const int warps = 4;
-  const int DT = warps * 32 / lpc;
-  if ((DT * (int)ei) % 16 || (DT * (int)eo) % 16) return SSM_ERR_UNSUPPORTED;
+  // launch shape: the same choice a plan makes by default (most busy warps
+  // per SM, capped at 12 and weighted by the cost of splitting channels)
+  struct Cand { int lpc, warps, DT, grid; int64_t rows; size_t smem; double score; };
+  Cand best{};
+  best.score = -1.0;
+  for (int lpc : {1, 2, 4, 8}) {
+    if (lpc > ns) continue;
+    const double eff = lpc == 1 ? 1.0 : lpc == 2 ? 0.95 : lpc == 4 ? 0.9 : 0.55;
+    for (int warps : {2, 4}) {
+      const int DT = warps * 32 / lpc;
+      if ((DT * (int)ei) % 16 || (DT * (int)eo) % 16) continue;
+      ssm::LaunchShape probe{lpc, warps, kTTna, kStagesNa, ns, 0, 0};
+      int occ = 0;
+      size_t smem = 0;
+      if (ssm::fwd_tma_smem_and_occupancy((int)d.in_dtype, (int)d.out_dtype, probe, &smem,
+                                          &occ) != cudaSuccess ||
+          occ < 1) {
+        cudaGetLastError();
+        continue;
+      }
+      const int64_t rows = d.batch * ((d.dim + DT - 1) / DT);
+      const int64_t grid = std::min<int64_t>(rows, (int64_t)occ * num_sms);
+      const int64_t per_sm = (grid + num_sms - 1) / num_sms;
+      const double busy = (double)grid * warps / num_sms;
+      const double balance = (double)grid / (double)(per_sm * num_sms);
+      const double score = std::min(busy, 12.0) * balance * eff + 1e-3 * warps;
+      if (score > best.score) best = Cand{lpc, warps, DT, (int)grid, rows, smem, score};
+    }
+  }
+  if (best.score < 0) return SSM_ERR_UNSUPPORTED;
+  const int DT = best.DT, warps = best.warps;
   const int nDT = (int)((d.dim + DT - 1) / DT);
-  const int64_t rows = d.batch * nDT;
+  const int64_t rows = best.rows;
+  const int64_t S = (d.seqlen + kTTna - 1) / kTTna;
+  if (rows * S > INT32_MAX) return SSM_ERR_UNSUPPORTED;
   // scratch layout: [Control | flags rows*warps u64 | states rows*DT*N f32]
   const size_t fl_bytes = (size_t)rows * warps * sizeof(unsigned long long);
   const size_t st_off = (kCtlBytes + fl_bytes + 255) / 256 * 256;
   const size_t need = st_off + (size_t)rows * DT * ns * sizeof(float);
   if (need > kNoAllocScratchBytes) return SSM_ERR_UNSUPPORTED;  // beyond the fixed scratch
-
-  ssm::LaunchShape ls{lpc, warps, kTTna, kStagesNa, ns, 0, 0};
-  int bps = 0;
-  size_t smem = 0;
-  if (ssm::fwd_tma_smem_and_occupancy((int)d.in_dtype, (int)d.out_dtype, ls, &smem, &bps) !=
-          cudaSuccess ||
-      bps < 1) {
-    cudaGetLastError();
-    return SSM_ERR_UNSUPPORTED;
-  }
-  const int64_t grid = std::min<int64_t>((int64_t)bps * num_sms, rows);
-  const int64_t tiles = (d.seqlen + kTTna - 1) / kTTna;
-  int64_t nseg = std::min(std::max<int64_t>(1, (8 * grid + rows - 1) / rows), tiles);
-  const int Tseg = (int)(((d.seqlen + nseg - 1) / nseg + kTTna - 1) / kTTna * kTTna);
-  nseg = (d.seqlen + Tseg - 1) / Tseg;
-  if (rows * nseg > INT32_MAX) return SSM_ERR_UNSUPPORTED;
-  ls.grid = (int)std::max<int64_t>(1, std::min<int64_t>(grid, rows * nseg));
-  ls.smem = smem;
+  ssm::LaunchShape ls{best.lpc, warps, kTTna, kStagesNa, ns,
+                      (int)std::max<int64_t>(1, std::min<int64_t>(best.grid, rows * S)), best.smem};
 
   unsigned char *base = static_cast<unsigned char *>(scratch_address(device));
   if (!base) return SSM_ERR_CUDA;
@@ -171,26 +181,24 @@ extern "C" SSM_API ssm_status ssm_scan_fwd_noalloc(
       !encode_na(&maps.dt, d.in_dtype, delta, Dm, L, Bn, DT, kTTna) ||
       !encode_na(&maps.z, d.in_dtype, z ? z : x, Dm, L, Bn, DT, kTTna) ||
       !encode_na(&maps.B, d.in_dtype, B, N, L, Bn, (uint32_t)N, kTTna) ||
-      !encode_na(&maps.C, d.in_dtype, C, N, L, Bn, (uint32_t)N, kTTna) ||
-      !encode_na(&maps.y, d.out_dtype, y, Dm, L, Bn, DT, kTTna))
+      !encode_na(&maps.C, d.in_dtype, C, N, L, Bn, (uint32_t)N, kTTna))
     return SSM_ERR_CUDA;
 
   ssm::FwdParams p{};
   p.Bsz = (int)d.batch; p.L = (int)d.seqlen; p.D = (int)d.dim; p.N = ns;
-  p.DT = DT; p.nDT = nDT; p.Tseg = Tseg; p.nseg = (int)nseg;
-  p.rows = (int)rows; p.total_items = rows * nseg;
+  p.DT = DT; p.nDT = nDT; p.rows = (int)rows; p.S = (int)S;
   p.softplus = (f & SSM_DELTA_SOFTPLUS) != 0;
   p.has_z = (f & SSM_HAS_Z) != 0;
   p.has_D = (f & SSM_HAS_D) != 0;
   p.has_bias = (f & SSM_HAS_DELTA_BIAS) != 0;
   p.has_h0 = (f & SSM_HAS_H0) != 0;
   p.want_hlast = (f & SSM_WANT_HLAST) != 0;
-  p.A = A; p.Dv = D; p.bias = delta_bias; p.h0 = h0; p.h_last = h_last;
+  p.A = A; p.Dv = D; p.bias = delta_bias; p.h0 = h0; p.h_last = h_last; p.y = y;
   p.ctl = reinterpret_cast<ssm::Control *>(base);
   p.ws_flags = reinterpret_cast<unsigned long long *>(base + kCtlBytes);
   p.ws_state = reinterpret_cast<float *>(base + st_off);
   p.timeout_ns = 2000000000ull;
-  p.drop_item = -1;
+  p.drop_unit = -1;
   const cudaError_t e = ssm::launch_fwd_tma((int)d.in_dtype, (int)d.out_dtype, ls, maps, p,
                                             reinterpret_cast<cudaStream_t>(stream_));
   return e == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;

@@ -9,10 +9,10 @@
 namespace ssm {
 
 // Device-resident control block of one plan.  The last CTA of each chunked
-// launch resets `tile` and `done` and advances `epoch`, so consecutive calls
+// launch resets `done` and advances `epoch`, so consecutive calls
 // need no memset and work under stream capture.
 struct Control {
-  unsigned long long tile;  // next work item to claim
+  unsigned long long reserved;
   unsigned int done;        // CTAs finished in the current launch
   unsigned int epoch;       // launch counter, tags the carry flags
   int status;               // 0 or a timeout code, sticky until read
@@ -21,27 +21,26 @@ struct Control {
 
 struct FwdParams {
   int Bsz, L, D, N;
-  int DT;       // channels per CTA (row tile)
-  int nDT;      // row tiles per batch
-  int Tseg;     // timesteps per work item
-  int nseg;     // work items per row
+  int DT;       // channels per row tile
+  int nDT;      // row tiles per batch element
   int rows;     // Bsz * nDT
-  long long total_items;
+  int S;        // stages (of the kernel's stage length) per row
   bool softplus, has_z, has_D, has_bias, has_h0, want_hlast;
   const float *A;      // (D, N)
   const float *Dv;     // (D) or null
   const float *bias;   // (D) or null
   const float *h0;     // (B, D, N) or null
   float *h_last;       // (B, D, N) or null
-  float *ws_state;     // rows * DT * NS carried states
+  void *y;             // (B, L, D) output
+  float *ws_state;     // rows * DT * N carried states
   unsigned long long *ws_flags;  // rows * warps carry flags
   Control *ctl;
   unsigned long long timeout_ns;
-  long long drop_item;
+  long long drop_unit;  // test hook: the run ending at this unit does not hand on its state
 };
 
 struct TmaMaps {
-  CUtensorMap x, dt, z, B, C, y;
+  CUtensorMap x, dt, z, B, C;
 };
 
 struct LaunchShape {
@@ -50,7 +49,7 @@ struct LaunchShape {
   size_t smem;
 };
 
-// Chunked TMA forward kernel (scan_fwd_tma.cu).
+// Fused forward kernel (scan_fwd_kernel.cuh, instantiated per dtype pair).
 cudaError_t launch_fwd_tma(int in_dtype, int out_dtype, const LaunchShape &ls,
                            const TmaMaps &maps, const FwdParams &p, cudaStream_t stream);
 // Dynamic shared memory and per-SM residency of one chunked-kernel variant.

@@ -12,7 +12,7 @@
 #include <mutex>
 #include <new>
 
-#include "../../include/ssm_scan.h"
+#include "ssm_scan.h"
 #include "scan_params.h"
 
 namespace {
@@ -20,8 +20,8 @@ namespace {
 constexpr uint32_t kKnownFlags = SSM_HAS_Z | SSM_HAS_D | SSM_DELTA_SOFTPLUS | SSM_HAS_DELTA_BIAS |
                                  SSM_HAS_H0 | SSM_WANT_HLAST | SSM_A_DIRECT;
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
-constexpr int kTT = 64;       // stage length of the chunked kernel
-constexpr int kStages = 3;    // pipeline depth of the chunked kernel
+constexpr int kTTDefault = 32;  // default stage length (work unit) of the fused kernel
+constexpr int kStages = 2;      // TMA slots of the fused kernel
 constexpr int kMaxDstate = 64;
 
 enum Path { PATH_TMA = 0, PATH_GENERAL = 1, PATH_DIRECT = 2 };
@@ -82,15 +82,15 @@ struct ssm_scan_plan {
   int num_sms = 0;
   int path = PATH_GENERAL;
   ssm::LaunchShape ls{};
-  int DT = 0, nDT = 0, Tseg = 0, nseg = 0;
-  int64_t rows = 0, items = 0;
+  int DT = 0, nDT = 0, S = 0;
+  int64_t rows = 0, units = 0;
   ssm_scan_config cfg{};  // user overrides
   ssm::Control *ctl = nullptr;
   float *ws_state = nullptr;
   unsigned long long *ws_flags = nullptr;
   size_t ws_state_bytes = 0, ws_flag_bytes = 0;
   uint64_t timeout_ns = kDefaultTimeoutNs;
-  int64_t drop_item = -1;
+  int64_t drop_unit = -1;
 };
 
 namespace {
@@ -124,58 +124,73 @@ bool tma_eligible(const ssm_scan_desc &d) {
   return true;
 }
 
-// Choose the launch shape of the chunked kernel and size the workspace.
+// Measured relative efficiency of each lanes-per-channel choice (B200,
+// consumer scan loop at equal warps per SM): splitting a channel's states over
+// more lanes adds shuffles and shared loads per update.
+double lpc_efficiency(int lpc) {
+  switch (lpc) {
+    case 1: return 1.0;
+    case 2: return 0.95;
+    case 4: return 0.9;
+    default: return 0.55;
+  }
+}
+
+// Choose the launch shape of the fused kernel and size the workspace.  Rows
+// (batch x channel tiles) are the only independent chains, so at most `rows`
+// CTAs can be busy: grid = min(rows, CTAs resident on the device), which
+// keeps every CTA's range starting at a row head (no CTA waits for another at
+// its start).  Among the variants, pick the most busy consumer warps per SM
+// (capped at 12), discounted for uneven CTAs per SM and for the instruction
+// cost of splitting channels across lanes.
 ssm_status plan_tma(ssm_scan_plan *pl) {
   const ssm_scan_desc &d = pl->desc;
   const int ns = (int)d.dstate;
-  const int64_t chans = d.batch * d.dim;
-  // lanes per channel: enough warps for ~2 per SM sub-partition, within N
-  int lpc = pl->cfg.lanes_per_chan;
-  if (lpc == 0) {
-    const int64_t target_warps = 8LL * pl->num_sms;
-    lpc = 1;
-    while (lpc < 8 && lpc * 2 <= ns && chans * lpc / 32 < target_warps) lpc *= 2;
-  }
-  if (lpc != 1 && lpc != 2 && lpc != 4 && lpc != 8) return SSM_ERR_INVALID_ARG;
-  if (lpc > ns) return SSM_ERR_INVALID_ARG;
-  int warps = pl->cfg.warps_per_cta ? pl->cfg.warps_per_cta : 4;
-  if (warps != 2 && warps != 4 && warps != 8) return SSM_ERR_INVALID_ARG;
-  const int DT = warps * 32 / lpc;
-  // keep TMA boxes 16-byte granular
-  if ((DT * (int)dtype_size(d.in_dtype)) % 16 || (DT * (int)dtype_size(d.out_dtype)) % 16)
+  const int sms = pl->num_sms;
+  const int ei = (int)dtype_size(d.in_dtype), eo = (int)dtype_size(d.out_dtype);
+  if (pl->cfg.tile_t && pl->cfg.tile_t != 16 && pl->cfg.tile_t != 32 && pl->cfg.tile_t != 64)
     return SSM_ERR_INVALID_ARG;
-  ssm::LaunchShape ls{lpc, warps, kTT, kStages, ns, 0, 0};
-  int bps = 0;
-  size_t smem = 0;
-  if (ssm::fwd_tma_smem_and_occupancy((int)d.in_dtype, (int)d.out_dtype, ls, &smem, &bps) !=
-          cudaSuccess ||
-      bps < 1) {
-    cudaGetLastError();
-    return SSM_ERR_UNSUPPORTED;  // this launch shape does not fit the device
+  struct Cand { int lpc, warps, tt, DT, occ, grid; int64_t rows; size_t smem; double score; };
+  Cand best{};
+  best.score = -1.0;
+  for (int lpc : {1, 2, 4, 8}) {
+    if (lpc > ns) continue;
+    if (pl->cfg.lanes_per_chan && lpc != pl->cfg.lanes_per_chan) continue;
+    for (int warps : {2, 4})
+    for (int tt : {kTTDefault, 16}) {
+      if (pl->cfg.warps_per_cta && warps != pl->cfg.warps_per_cta) continue;
+      if (pl->cfg.tile_t ? tt != pl->cfg.tile_t : false) continue;
+      const int DT = warps * 32 / lpc;
+      if ((DT * ei) % 16 || (DT * eo) % 16) continue;
+      ssm::LaunchShape ls{lpc, warps, tt, kStages, ns, 0, 0};
+      int occ = 0;
+      size_t smem = 0;
+      if (ssm::fwd_tma_smem_and_occupancy((int)d.in_dtype, (int)d.out_dtype, ls, &smem, &occ) !=
+              cudaSuccess ||
+          occ < 1) {
+        cudaGetLastError();
+        continue;
+      }
+      const int64_t rows = d.batch * ((d.dim + DT - 1) / DT);
+      int64_t grid = std::min<int64_t>(rows, (int64_t)occ * sms);
+      if (pl->cfg.grid > 0) grid = std::min<int64_t>(pl->cfg.grid, (int64_t)occ * sms);
+      const int64_t per_sm = (grid + sms - 1) / sms;                 // CTAs on the busiest SM
+      const double busy = (double)std::min<int64_t>(grid, rows) * warps / sms;
+      const double balance = (double)grid / (double)(per_sm * sms);
+      const double score =
+          std::min(busy, 12.0) * balance * lpc_efficiency(lpc) + 1e-3 * warps - 1e-4 * tt;
+      if (score > best.score) best = Cand{lpc, warps, tt, DT, occ, (int)grid, rows, smem, score};
+    }
   }
-  const int64_t cap = (int64_t)bps * pl->num_sms;
-  const int nDT = (int)((d.dim + DT - 1) / DT);
-  const int64_t rows = d.batch * nDT;
-  // persistent CTAs: no more than rows, so a chunk's predecessor is normally done
-  int64_t grid = std::min(cap, rows);
-  if (pl->cfg.grid > 0) grid = std::min<int64_t>(pl->cfg.grid, cap);
-  // chunk length: ~8 work items per CTA for dynamic balance
-  int Tseg = pl->cfg.seg_len;
-  if (Tseg == 0) {
-    const int64_t tiles = (d.seqlen + kTT - 1) / kTT;
-    int64_t nseg = std::max<int64_t>(1, (8 * grid + rows - 1) / rows);
-    nseg = std::min(nseg, tiles);
-    const int64_t per = (d.seqlen + nseg - 1) / nseg;
-    Tseg = (int)((per + kTT - 1) / kTT * kTT);
-  }
-  if (Tseg <= 0 || Tseg % kTT) return SSM_ERR_INVALID_ARG;
-  const int64_t nseg = (d.seqlen + Tseg - 1) / Tseg;
-  if (rows * nseg > INT32_MAX) return SSM_ERR_UNSUPPORTED;
-  ls.grid = (int)std::max<int64_t>(1, std::min<int64_t>(grid, rows * nseg));
-  ls.smem = smem;
+  if (best.score < 0) return SSM_ERR_UNSUPPORTED;  // no variant fits (or bad override)
+  const int64_t S = (d.seqlen + best.tt - 1) / best.tt;
+  if (best.rows * S > INT32_MAX) return SSM_ERR_UNSUPPORTED;
+  ssm::LaunchShape ls{best.lpc, best.warps, best.tt, kStages, ns,
+                      (int)std::max<int64_t>(1, std::min<int64_t>(best.grid, best.rows * S)),
+                      best.smem};
   // workspace: carried state per (row, channel, n) and a flag per (row, warp)
-  const size_t st_bytes = (size_t)rows * DT * ns * sizeof(float);
-  const size_t fl_bytes = (size_t)rows * warps * sizeof(unsigned long long);
+  const size_t st_bytes = (size_t)best.rows * best.DT * ns * sizeof(float);
+  const size_t fl_bytes = (size_t)best.rows * best.warps * sizeof(unsigned long long);
   if (st_bytes > pl->ws_state_bytes) {
     if (pl->ws_state) cudaFree(pl->ws_state);
     pl->ws_state = nullptr;
@@ -193,12 +208,11 @@ ssm_status plan_tma(ssm_scan_plan *pl) {
   // flags start below every epoch tag (epochs start at 1)
   if (cudaMemset(pl->ws_flags, 0, pl->ws_flag_bytes) != cudaSuccess) return SSM_ERR_CUDA;
   pl->ls = ls;
-  pl->DT = DT;
-  pl->nDT = nDT;
-  pl->Tseg = Tseg;
-  pl->nseg = (int)nseg;
-  pl->rows = rows;
-  pl->items = rows * nseg;
+  pl->DT = best.DT;
+  pl->nDT = (int)((d.dim + best.DT - 1) / best.DT);
+  pl->S = (int)S;
+  pl->rows = best.rows;
+  pl->units = best.rows * S;
   return SSM_OK;
 }
 
@@ -298,11 +312,11 @@ ssm_status ssm_scan_get_info(const ssm_scan_plan *pl, ssm_scan_info *info) {
     info->warps_per_cta = pl->ls.warps;
     info->tile_t = pl->ls.tt;
     info->stages = pl->ls.stages;
-    info->seg_len = pl->Tseg;
+    info->stages_per_row = pl->S;
     info->chans_per_cta = pl->DT;
     info->grid = pl->ls.grid;
     info->rows = pl->rows;
-    info->items = pl->items;
+    info->units = pl->units;
     info->smem_bytes = pl->ls.smem;
   }
   info->workspace_bytes = pl->ws_state_bytes + pl->ws_flag_bytes + sizeof(ssm::Control);
@@ -311,7 +325,7 @@ ssm_status ssm_scan_get_info(const ssm_scan_plan *pl, ssm_scan_info *info) {
 
 ssm_status ssm_scan_set_config(ssm_scan_plan *pl, const ssm_scan_config *cfg) {
   if (!pl || !cfg) return SSM_ERR_INVALID_ARG;
-  if (cfg->lanes_per_chan < 0 || cfg->warps_per_cta < 0 || cfg->seg_len < 0 || cfg->grid < 0)
+  if (cfg->lanes_per_chan < 0 || cfg->warps_per_cta < 0 || cfg->grid < 0 || cfg->tile_t < 0)
     return SSM_ERR_INVALID_ARG;
   DeviceGuard guard(pl->device);
   if (!guard.ok) return SSM_ERR_CUDA;
@@ -327,10 +341,10 @@ ssm_status ssm_scan_set_config(ssm_scan_plan *pl, const ssm_scan_config *cfg) {
   return s;
 }
 
-ssm_status ssm_scan_set_debug(ssm_scan_plan *pl, uint64_t wait_timeout_ns, int64_t drop_item) {
+ssm_status ssm_scan_set_debug(ssm_scan_plan *pl, uint64_t wait_timeout_ns, int64_t drop_unit) {
   if (!pl) return SSM_ERR_INVALID_ARG;
   pl->timeout_ns = wait_timeout_ns ? wait_timeout_ns : kDefaultTimeoutNs;
-  pl->drop_item = drop_item;
+  pl->drop_unit = drop_unit;
   return SSM_OK;
 }
 
@@ -399,24 +413,22 @@ ssm_status ssm_scan_fwd(ssm_scan_plan *pl, const void *x, const void *delta,
         !encode3d(&maps.dt, d.in_dtype, delta, Dm, L, Bn, DT, TT) ||
         !encode3d(&maps.z, d.in_dtype, z ? z : x, Dm, L, Bn, DT, TT) ||
         !encode3d(&maps.B, d.in_dtype, B, N, L, Bn, (uint32_t)N, TT) ||
-        !encode3d(&maps.C, d.in_dtype, C, N, L, Bn, (uint32_t)N, TT) ||
-        !encode3d(&maps.y, d.out_dtype, y, Dm, L, Bn, DT, TT))
+        !encode3d(&maps.C, d.in_dtype, C, N, L, Bn, (uint32_t)N, TT))
       return SSM_ERR_CUDA;
     ssm::FwdParams p{};
     p.Bsz = (int)d.batch; p.L = (int)d.seqlen; p.D = (int)d.dim; p.N = (int)d.dstate;
-    p.DT = pl->DT; p.nDT = pl->nDT; p.Tseg = pl->Tseg; p.nseg = pl->nseg;
-    p.rows = (int)pl->rows; p.total_items = pl->items;
-    p.softplus = f & SSM_DELTA_SOFTPLUS;
-    p.has_z = f & SSM_HAS_Z;
-    p.has_D = f & SSM_HAS_D;
-    p.has_bias = f & SSM_HAS_DELTA_BIAS;
-    p.has_h0 = f & SSM_HAS_H0;
-    p.want_hlast = f & SSM_WANT_HLAST;
+    p.DT = pl->DT; p.nDT = pl->nDT; p.rows = (int)pl->rows; p.S = pl->S;
+    p.softplus = (f & SSM_DELTA_SOFTPLUS) != 0;
+    p.has_z = (f & SSM_HAS_Z) != 0;
+    p.has_D = (f & SSM_HAS_D) != 0;
+    p.has_bias = (f & SSM_HAS_DELTA_BIAS) != 0;
+    p.has_h0 = (f & SSM_HAS_H0) != 0;
+    p.want_hlast = (f & SSM_WANT_HLAST) != 0;
     p.A = static_cast<const float *>(A);
-    p.Dv = D; p.bias = delta_bias; p.h0 = h0; p.h_last = h_last;
+    p.Dv = D; p.bias = delta_bias; p.h0 = h0; p.h_last = h_last; p.y = y;
     p.ws_state = pl->ws_state; p.ws_flags = pl->ws_flags; p.ctl = pl->ctl;
     p.timeout_ns = pl->timeout_ns;
-    p.drop_item = pl->drop_item;
+    p.drop_unit = pl->drop_unit;
     return map_cuda(ssm::launch_fwd_tma((int)d.in_dtype, (int)d.out_dtype, pl->ls, maps, p, stream));
   }
 

@@ -32,29 +32,23 @@ def test_tiny_fp32_workload():
 
 
 @pytest.mark.parametrize("lpc", [1, 2, 4, 8])
-@pytest.mark.parametrize("warps", [2, 4, 8])
-def test_bf16_all_options_every_variant(lpc, warps):
+@pytest.mark.parametrize("warps", [2, 4])
+@pytest.mark.parametrize("grid", [0, 5, 40])
+def test_bf16_all_options_every_variant(lpc, warps, grid):
     """bf16 in/out, gate, skip, bias, h0; ragged L (not a multiple of the
-    stage) and chunks of one stage so the carry crosses many work items."""
+    stage).  grid=5 splits rows between CTAs (carried state handed over);
+    grid=40 gives CTAs less than a row each, so a row passes through a chain
+    of CTAs."""
     inp = synth.make_fwd(3, 389, 64, 16, seed=21, has_h0=True)
-    if lpc == 1 and warps == 8:   # 256 bf16 channels x 3 stages does not fit in shared memory
-        from selective_state_space_31_b200 import binding as bnd
-        plan = gu.make_plan(inp)
-        with pytest.raises(bnd.SsmError):
-            plan.set_config(lanes_per_chan=lpc, warps_per_cta=warps, seg_len=64)
-        gy, gh = gu.run_gpu(inp, plan)   # the previous shape stays in force
-        ry, rh = gu.run_oracle(inp)
-        gu.assert_parity(gy, ry, gh, rh, gu.TOL["bf16"], "after rejected config")
-        return
-    _case(inp, dict(lanes_per_chan=lpc, warps_per_cta=warps, seg_len=64), expect_path=0)
+    _case(inp, dict(lanes_per_chan=lpc, warps_per_cta=warps, grid=grid), expect_path=0)
 
 
-@pytest.mark.parametrize("seg_len,grid", [(64, 1), (128, 2), (192, 0), (0, 0), (64, 500)])
-def test_chunking_and_grid(seg_len, grid):
-    """A single CTA walking every item (grid=1), small grids that must wait
-    for predecessors, default and oversize grids."""
+@pytest.mark.parametrize("grid", [1, 2, 7, 0, 64, 5000])
+def test_schedule_grid_sizes(grid):
+    """One CTA walking every unit, small grids, the default, and grids
+    larger than the rows (clamped to what is co-resident)."""
     inp = synth.make_fwd(2, 1000, 128, 16, seed=22, has_h0=True)
-    _case(inp, dict(seg_len=seg_len, grid=grid), expect_path=0)
+    _case(inp, dict(grid=grid), expect_path=0)
 
 
 @pytest.mark.parametrize("N", [4, 8, 16])
@@ -120,7 +114,7 @@ def test_zero_length_and_empty():
 def test_deterministic():
     inp = synth.make_fwd(2, 700, 128, 16, seed=29, has_h0=True)
     plan = gu.make_plan(inp)
-    plan.set_config(seg_len=64)
+    plan.set_config(grid=7)
     dev = gu.upload(inp)
     a = gu.run_gpu(inp, plan, dev)
     b = gu.run_gpu(inp, plan, dev)
@@ -194,15 +188,16 @@ def test_decode_steps_match_full_sequence(N, dt):
 
 
 def test_timeout_is_reported_without_hanging():
-    """A work item that never hands its state on makes the next chunk's
-    bounded wait expire: the kernel records SSM_ERR_TIMEOUT and returns; the
-    plan stays usable and the next call is exact again."""
+    """A CTA that never hands its state on makes the CTA continuing that row
+    wait until the bound expires: the kernel records SSM_ERR_TIMEOUT and
+    returns; the plan stays usable and the next call is exact again."""
     inp = synth.make_fwd(1, 512, 32, 16, seed=34)
     plan = gu.make_plan(inp)
-    plan.set_config(seg_len=128)
+    plan.set_config(lanes_per_chan=4, warps_per_cta=4, grid=3)
     info = plan.info()
-    assert info["items"] >= 2
-    plan.set_debug(wait_timeout_ns=50_000_000, drop_item=0)
+    assert info["rows"] == 1 and info["stages_per_row"] == 16 and info["grid"] == 3, info
+    # CTA 0 runs units [0, 5) of the single row and hands over after unit 4
+    plan.set_debug(wait_timeout_ns=50_000_000, drop_unit=4)
     dev = gu.upload(inp)
     gu.run_gpu(inp, plan, dev)
     assert plan.status() == 5  # SSM_ERR_TIMEOUT
