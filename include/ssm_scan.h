@@ -112,11 +112,13 @@ typedef struct {
   int warps_per_cta;
   int tile_t;          /* tokens per pipeline stage (one work unit) */
   int stages;          /* pipeline depth */
-  int stages_per_row;  /* work units per row = ceil(seqlen / tile_t) */
+  int stages_per_row;  /* ceil(seqlen / tile_t) */
   int chans_per_cta;   /* channels per row tile */
-  int grid;            /* CTAs launched (each takes an equal share of the units) */
+  int grid;            /* CTAs launched (CTA c runs items c, c + grid, ...) */
   int64_t rows;        /* independent (batch, channel-tile) rows */
-  int64_t units;       /* work units = rows * stages_per_row */
+  int64_t units;       /* stages in all = rows * stages_per_row */
+  int parts_per_row;   /* work items per row (a row's parts hand their state on) */
+  int stages_per_part;
   size_t smem_bytes;
   size_t workspace_bytes;
 } ssm_scan_info;

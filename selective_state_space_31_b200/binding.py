@@ -43,6 +43,7 @@ class Info(ctypes.Structure):
                 ("warps_per_cta", ctypes.c_int), ("tile_t", ctypes.c_int), ("stages", ctypes.c_int),
                 ("stages_per_row", ctypes.c_int), ("chans_per_cta", ctypes.c_int),
                 ("grid", ctypes.c_int), ("rows", ctypes.c_int64), ("units", ctypes.c_int64),
+                ("parts_per_row", ctypes.c_int), ("stages_per_part", ctypes.c_int),
                 ("smem_bytes", ctypes.c_size_t), ("workspace_bytes", ctypes.c_size_t)]
 
     def as_dict(self):

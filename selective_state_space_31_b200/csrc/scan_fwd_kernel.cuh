@@ -16,16 +16,17 @@
 //     LPC lanes (NPL = N / LPC each); the lanes' partial readouts of a group
 //     of LPC tokens are combined by a shuffle butterfly that leaves lane q with
 //     token q, and lane q finishes that token.
-//   * Static balanced schedule: the R*S (row, stage) units, in row-major
-//     order, are cut into gridDim.x equal contiguous ranges, one per CTA.  A
-//     range is the tail of one row, some whole rows, and the head of one row.
-//     The CTA runs the head and whole rows first and the tail last; a row
-//     split between CTAs j and j+1 has its head done first by j, so the
-//     carried state j hands to j+1 (a (row, stage) flag, release/acquire) is
-//     normally ready long before j+1 reaches the tail.  This is the pages'
-//     associative carry ("Scan bien recurrence ...": (A2,b2) (x) (A1,b1) =
-//     (A2A1, A2b1+b2)): the state after the head is the exact starting state
-//     of the tail.  Every wait is bounded by a timer.
+//   * Strided item schedule.  Each row's S stages are cut into parts of PL
+//     stages; item i = part * R + row.  CTA c runs items c, c + P, c + 2P, ...
+//     in order (P = gridDim.x <= R).  The predecessor of an item (same row,
+//     previous part) has index i - R <= i - P, so it belongs to an earlier
+//     slot of some CTA: run in lock-step, no CTA waits, and every CTA gets the
+//     same number of items (to within one).  A part hands its final state to
+//     the next part through a per-(row, warp) flag carrying the stage index
+//     and a launch epoch (release/acquire) -- the pages' associative carry
+//     ("Scan bien recurrence ...": (A2,b2) (x) (A1,b1) = (A2A1, A2b1+b2)): the
+//     state after one part is the exact starting state of the next.  Every
+//     wait is bounded by a timer.
 //   * Warp specialisation.  One producer warp per CTA issues the TMA loads
 //     (cp.async.bulk.tensor, no multicast) of the [TT, DT] tiles of
 //     x / delta / z and the [TT, N] tiles of B / C into a ring of raw slots,
@@ -52,7 +53,7 @@ struct FwdCfg {
   static constexpr int NPL = NS / LPC;    // states per lane
   static constexpr int DTW = 32 / LPC;    // channels per consumer warp
   static constexpr int DT = WARPS * DTW;  // channels per row tile
-  static constexpr int PWARPS = 2;                  // producer warps
+  static constexpr int PWARPS = WARPS >= 4 ? WARPS / 2 : 1;  // producer warps
   static constexpr int THREADS = (WARPS + PWARPS) * 32;
   // ring depths: ~96 tokens of TMA prefetch and 3 fp32 stage slots, halved
   // for wide tiles (>= 128 channels) so that the CTA still fits one SM
@@ -136,50 +137,32 @@ __device__ __forceinline__ float2 load_pair<__nv_bfloat16>(const __nv_bfloat16 *
   return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(p));
 }
 
-// Walks one CTA's units in processing order (the range [ua, u1) first, then
-// [u0, ua)) with increments only; divisions happen at construction and at
-// the single jump between the two ranges.
-struct UnitCursor {
-  int k;          // position in the CTA's sequence
-  int row, st;    // current unit: row and stage within the row
-  int b, dtile;   // batch element and channel tile of `row`
-  int n1, S, nDT;
-  int r0, s0;     // start of the second range
-  __device__ __forceinline__ void set_row(int r) {
-    row = r;
-    b = r / nDT;
-    dtile = r - b * nDT;
+// Walks one CTA's items (c, c + P, c + 2P, ...) stage by stage; a division
+// happens only when a new item starts.
+struct ItemCursor {
+  int item, items, P, R, PL, S, nDT;
+  int row, part, st, st_end, b, dtile;
+  __device__ __forceinline__ void load() {
+    if (item >= items) return;
+    part = item / R;
+    row = item - part * R;
+    st = part * PL;
+    st_end = min(S, st + PL);
+    b = row / nDT;
+    dtile = row - b * nDT;
   }
-  __device__ __forceinline__ void init(long long u0, long long ua, long long u1, int S_, int nDT_) {
-    S = S_;
-    nDT = nDT_;
-    n1 = (int)(u1 - ua);
-    r0 = (int)(u0 / S);
-    s0 = (int)(u0 - (long long)r0 * S);
-    k = 0;
-    if (n1 > 0) {
-      set_row((int)(ua / S));
-      st = 0;
-    } else {
-      set_row(r0);
-      st = s0;
-    }
+  __device__ __forceinline__ void init(int c, const FwdParams &p) {
+    item = c; items = p.items; P = gridDim.x; R = p.rows; PL = p.PL; S = p.S; nDT = p.nDT;
+    row = part = st = st_end = b = dtile = 0;
+    load();
   }
   __device__ __forceinline__ void advance() {
-    ++k;
-    if (k == n1) {
-      set_row(r0);
-      st = s0;
-    } else if (++st == S) {
-      st = 0;
-      ++row;
-      if (++dtile == nDT) { dtile = 0; ++b; }
-    }
+    if (++st == st_end) { item += P; load(); }
   }
 };
 
 template <typename InT, typename OutT, int NS, int LPC, int WARPS, int TT>
-__global__ void __launch_bounds__((WARPS + 2) * 32)
+__global__ void __launch_bounds__((WARPS + (WARPS >= 4 ? WARPS / 2 : 1)) * 32)
     fwd_kernel(const __grid_constant__ TmaMaps maps, const FwdParams p) {
   using Cfg = FwdCfg<InT, OutT, NS, LPC, WARPS, TT>;
   constexpr int NPL = Cfg::NPL, DTW = Cfg::DTW, DT = Cfg::DT, RAW = Cfg::RAW,
@@ -194,14 +177,13 @@ __global__ void __launch_bounds__((WARPS + 2) * 32)
 
   const unsigned int epoch = *reinterpret_cast<volatile unsigned int *>(&p.ctl->epoch);
 
-  // ---- static schedule: units [u0, u1) in the order [ua, u1) then [u0, ua) ----
+  // ---- strided item schedule: stages this CTA runs ----
   const int S = p.S;
-  const long long U = (long long)p.rows * S;
-  const long long u0 = U * blockIdx.x / gridDim.x;
-  const long long u1 = U * (blockIdx.x + 1) / gridDim.x;
-  const int n = (int)(u1 - u0);
-  const long long ua = min(u1, (u0 + S - 1) / S * S);  // first row start in range
-  const int n1 = (int)(u1 - ua);
+  int n = 0;
+  for (int it = blockIdx.x; it < p.items; it += gridDim.x) {
+    const int part = it / p.rows;
+    n += min(S, (part + 1) * p.PL) - part * p.PL;
+  }
 
   if (tid == 0) {
 #pragma unroll
@@ -224,10 +206,11 @@ __global__ void __launch_bounds__((WARPS + 2) * 32)
     const bool issuer = ptid == 0;
     const uint32_t tx_bytes =
         (p.has_z ? 3u : 2u) * TT * DT * sizeof(InT) + 2u * TT * NS * sizeof(InT);
-    UnitCursor iss;  // next stage to load (issuer thread)
-    iss.init(u0, ua, u1, S, p.nDT);
+    ItemCursor iss;  // next stage to load (issuer thread)
+    iss.init(blockIdx.x, p);
+    int iss_k = 0;
     auto issue = [&]() {
-      const int r = iss.k % RAW;
+      const int r = iss_k % RAW;
       const int d0 = iss.dtile * DT, t0 = iss.st * TT, b = iss.b;
       unsigned char *sb = smem + r * Cfg::SLOT;
       mbar_arrive_expect_tx(&rfull[r], tx_bytes);
@@ -237,6 +220,7 @@ __global__ void __launch_bounds__((WARPS + 2) * 32)
       tma_load_3d(sb + 3 * Cfg::XTILE, &maps.B, &rfull[r], 0, t0, b);
       tma_load_3d(sb + 3 * Cfg::XTILE + Cfg::BCTILE, &maps.C, &rfull[r], 0, t0, b);
       iss.advance();
+      ++iss_k;
     };
     if (issuer)
       for (int k = 0; k < n && k < RAW; ++k) issue();
@@ -266,8 +250,8 @@ __global__ void __launch_bounds__((WARPS + 2) * 32)
     int pre_row = -1;
     float2 bias2 = make_float2(0.f, 0.f), dsk2 = make_float2(0.f, 0.f);
 
-    UnitCursor cur;
-    cur.init(u0, ua, u1, S, p.nDT);
+    ItemCursor cur;
+    cur.init(blockIdx.x, p);
     bool ok = true;
     int k = 0;
     for (; k < n; ++k, cur.advance()) {
@@ -327,7 +311,7 @@ __global__ void __launch_bounds__((WARPS + 2) * 32)
         mbar_arrive(&pfull[s]);  // this warp's half of stage k is ready
         mbar_arrive(&rdone[r]);  // and it no longer reads raw slot r
       }
-      if (issuer && iss.k < n) {  // refill raw slot r with stage k + RAW
+      if (issuer && iss_k < n) {  // refill raw slot r with stage k + RAW
         if (mbar_wait_bounded(&rdone[r], (uint32_t)((k / RAW) & 1), p.timeout_ns)) issue();
         else ok = false;
       }
@@ -345,7 +329,7 @@ __global__ void __launch_bounds__((WARPS + 2) * 32)
     if (!__all_sync(FULL_MASK, ok) && lane == 0) {
       atomicCAS(&p.ctl->status, 0, kStatusTimeout);
       if (issuer)
-        for (int kk = k; kk < iss.k; ++kk)  // let loads in flight land (bounded)
+        for (int kk = k; kk < iss_k; ++kk)  // let loads in flight land (bounded)
           (void)mbar_wait_bounded(&rfull[kk % RAW], (uint32_t)((kk / RAW) & 1), p.timeout_ns);
     }
   } else {
@@ -356,8 +340,8 @@ __global__ void __launch_bounds__((WARPS + 2) * 32)
     float h[NPL], A2[NPL];
 #pragma unroll
     for (int i = 0; i < NPL; ++i) { h[i] = 0.f; A2[i] = 0.f; }
-    UnitCursor cur;
-    cur.init(u0, ua, u1, S, p.nDT);
+    ItemCursor cur;
+    cur.init(blockIdx.x, p);
     for (int k = 0; k < n; ++k, cur.advance()) {
       const int s = k % PS;
       if (!__all_sync(FULL_MASK, mbar_wait_bounded(&pfull[s], (uint32_t)((k / PS) & 1),
@@ -368,7 +352,7 @@ __global__ void __launch_bounds__((WARPS + 2) * 32)
       const int row = cur.row, st = cur.st, b = cur.b;
       const int d = cur.dtile * DT + ch;
       const bool valid_ch = d < p.D;
-      const bool run_start = k == 0 || st == 0 || k == n1;
+      const bool run_start = st == cur.part * cur.PL;
       if (run_start) {
 #pragma unroll
         for (int i = 0; i < NPL; ++i)
@@ -442,7 +426,7 @@ __global__ void __launch_bounds__((WARPS + 2) * 32)
       __syncwarp();
       if (lane == 0) mbar_arrive(&pempty[s]);  // slot s consumed, y tile written
 
-      const bool run_end = k == n - 1 || st == S - 1 || k == n1 - 1;
+      const bool run_end = st + 1 == cur.st_end;
       if (run_end) {
         if (st == S - 1) {
           if (p.want_hlast && valid_ch) {

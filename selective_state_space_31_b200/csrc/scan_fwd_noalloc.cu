@@ -130,7 +130,7 @@ extern "C" SSM_API ssm_status ssm_scan_fwd_noalloc(
     return SSM_ERR_CUDA;
   }
   // launch shape: the same choice a plan makes by default (most busy warps
-  // per SM, capped at 12 and weighted by the cost of splitting channels)
+  // per SM, capped at 10 and weighted by the cost of splitting channels)
   struct Cand { int lpc, warps, DT, grid; int64_t rows; size_t smem; double score; };
   Cand best{};
   best.score = -1.0;
@@ -150,11 +150,17 @@ extern "C" SSM_API ssm_status ssm_scan_fwd_noalloc(
         continue;
       }
       const int64_t rows = d.batch * ((d.dim + DT - 1) / DT);
-      const int64_t grid = std::min<int64_t>(rows, (int64_t)occ * num_sms);
-      const int64_t per_sm = (grid + num_sms - 1) / num_sms;
-      const double busy = (double)grid * warps / num_sms;
-      const double balance = (double)grid / (double)(per_sm * num_sms);
-      const double score = std::min(busy, 12.0) * balance * eff + 1e-3 * warps;
+      const int64_t cap = std::min<int64_t>(rows, (int64_t)occ * num_sms);
+      const int64_t balanced = cap >= num_sms ? cap / num_sms * num_sms : cap;
+      auto score_of = [&](int64_t g) {
+        const int64_t per_sm = (g + num_sms - 1) / num_sms;
+        const double busy = (double)g * warps / num_sms;
+        const double balance = (double)g / (double)(per_sm * num_sms);
+        const double tie = busy >= 10.0 ? -1e-3 * warps : 1e-3 * warps;
+        return std::min(busy, 10.0) * balance * eff + tie;
+      };
+      const int64_t grid = score_of(balanced) >= score_of(cap) ? balanced : cap;
+      const double score = score_of(grid);
       if (score > best.score) best = Cand{lpc, warps, DT, (int)grid, rows, smem, score};
     }
   }
@@ -163,14 +169,28 @@ extern "C" SSM_API ssm_status ssm_scan_fwd_noalloc(
   const int nDT = (int)((d.dim + DT - 1) / DT);
   const int64_t rows = best.rows;
   const int64_t S = (d.seqlen + kTTna - 1) / kTTna;
-  if (rows * S > INT32_MAX) return SSM_ERR_UNSUPPORTED;
+  // parts per row: the fewest that keep every CTA within ~5% of the mean
+  int m = 1;
+  if (best.grid < rows) {
+    double best_bal = 0.0;
+    for (int mm = 1; mm <= 64 && mm <= S; ++mm) {
+      const int64_t it = rows * mm;
+      const double bal = ((double)it / best.grid) / (double)((it + best.grid - 1) / best.grid);
+      if (bal > best_bal + 1e-9) { best_bal = bal; m = mm; }
+      if (bal >= 0.95) break;
+    }
+  }
+  const int64_t PL = (S + m - 1) / m;
+  const int64_t parts = (S + PL - 1) / PL;
+  if (rows * S > INT32_MAX || rows * parts > INT32_MAX) return SSM_ERR_UNSUPPORTED;
   // scratch layout: [Control | flags rows*warps u64 | states rows*DT*N f32]
   const size_t fl_bytes = (size_t)rows * warps * sizeof(unsigned long long);
   const size_t st_off = (kCtlBytes + fl_bytes + 255) / 256 * 256;
   const size_t need = st_off + (size_t)rows * DT * ns * sizeof(float);
   if (need > kNoAllocScratchBytes) return SSM_ERR_UNSUPPORTED;  // beyond the fixed scratch
   ssm::LaunchShape ls{best.lpc, warps, kTTna, kStagesNa, ns,
-                      (int)std::max<int64_t>(1, std::min<int64_t>(best.grid, rows * S)), best.smem};
+                      (int)std::max<int64_t>(1, std::min<int64_t>(best.grid, rows * parts)),
+                      best.smem};
 
   unsigned char *base = static_cast<unsigned char *>(scratch_address(device));
   if (!base) return SSM_ERR_CUDA;
@@ -187,6 +207,7 @@ extern "C" SSM_API ssm_status ssm_scan_fwd_noalloc(
   ssm::FwdParams p{};
   p.Bsz = (int)d.batch; p.L = (int)d.seqlen; p.D = (int)d.dim; p.N = ns;
   p.DT = DT; p.nDT = nDT; p.rows = (int)rows; p.S = (int)S;
+  p.PL = (int)PL; p.items = (int)(rows * parts);
   p.softplus = (f & SSM_DELTA_SOFTPLUS) != 0;
   p.has_z = (f & SSM_HAS_Z) != 0;
   p.has_D = (f & SSM_HAS_D) != 0;

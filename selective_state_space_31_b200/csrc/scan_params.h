@@ -25,6 +25,8 @@ struct FwdParams {
   int nDT;      // row tiles per batch element
   int rows;     // Bsz * nDT
   int S;        // stages (of the kernel's stage length) per row
+  int PL;       // stages per part (work item) of a row
+  int items;    // rows * parts per row
   bool softplus, has_z, has_D, has_bias, has_h0, want_hlast;
   const float *A;      // (D, N)
   const float *Dv;     // (D) or null

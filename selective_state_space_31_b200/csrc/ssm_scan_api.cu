@@ -82,7 +82,7 @@ struct ssm_scan_plan {
   int num_sms = 0;
   int path = PATH_GENERAL;
   ssm::LaunchShape ls{};
-  int DT = 0, nDT = 0, S = 0;
+  int DT = 0, nDT = 0, S = 0, PL = 0, parts = 0;
   int64_t rows = 0, units = 0;
   ssm_scan_config cfg{};  // user overrides
   ssm::Control *ctl = nullptr;
@@ -136,13 +136,31 @@ double lpc_efficiency(int lpc) {
   }
 }
 
+// Parts per row for P CTAs over R rows of S stages: the fewest parts that
+// keep every CTA within ~5% of the mean item count (P <= R).
+int parts_per_row(int64_t R, int64_t P, int64_t S) {
+  if (P >= R) return 1;
+  int best_m = 1;
+  double best_bal = 0.0;
+  for (int m = 1; m <= 64 && m <= S; ++m) {
+    const int64_t items = R * m;
+    const double mean = (double)items / P;
+    const double bal = mean / (double)((items + P - 1) / P);
+    if (bal > best_bal + 1e-9) { best_bal = bal; best_m = m; }
+    if (bal >= 0.95) return m;
+  }
+  return best_m;
+}
+
 // Choose the launch shape of the fused kernel and size the workspace.  Rows
 // (batch x channel tiles) are the only independent chains, so at most `rows`
-// CTAs can be busy: grid = min(rows, CTAs resident on the device), which
-// keeps every CTA's range starting at a row head (no CTA waits for another at
-// its start).  Among the variants, pick the most busy consumer warps per SM
-// (capped at 12), discounted for uneven CTAs per SM and for the instruction
-// cost of splitting channels across lanes.
+// CTAs can be busy: grid P <= min(rows, CTAs resident on the device), taken
+// as a multiple of the SM count when that keeps enough warps (every SM then
+// gets the same work).  Among the variants, pick the most busy consumer warps
+// per SM (capped at 10), discounted for uneven CTAs per SM and for the
+// instruction cost of splitting channels across lanes.  Ties: once an SM holds
+// 10 consumer warps, more CTAs of fewer warps (more independent producer
+// pipelines) measured faster on B200; below that, wider CTAs did.
 ssm_status plan_tma(ssm_scan_plan *pl) {
   const ssm_scan_desc &d = pl->desc;
   const int ns = (int)d.dstate;
@@ -172,21 +190,30 @@ ssm_status plan_tma(ssm_scan_plan *pl) {
         continue;
       }
       const int64_t rows = d.batch * ((d.dim + DT - 1) / DT);
-      int64_t grid = std::min<int64_t>(rows, (int64_t)occ * sms);
+      const int64_t cap = std::min<int64_t>(rows, (int64_t)occ * sms);
+      // either all that fits, or the largest multiple of the SM count below it
+      const int64_t balanced = cap >= sms ? cap / sms * sms : cap;
+      auto score_of = [&](int64_t g) {
+        const int64_t per_sm = (g + sms - 1) / sms;  // CTAs on the busiest SM
+        const double busy = (double)g * warps / sms;
+        const double balance = (double)g / (double)(per_sm * sms);
+        const double tie = busy >= 10.0 ? -1e-3 * warps : 1e-3 * warps;
+        return std::min(busy, 10.0) * balance * lpc_efficiency(lpc) + tie - 1e-4 * tt;
+      };
+      int64_t grid = score_of(balanced) >= score_of(cap) ? balanced : cap;
       if (pl->cfg.grid > 0) grid = std::min<int64_t>(pl->cfg.grid, (int64_t)occ * sms);
-      const int64_t per_sm = (grid + sms - 1) / sms;                 // CTAs on the busiest SM
-      const double busy = (double)std::min<int64_t>(grid, rows) * warps / sms;
-      const double balance = (double)grid / (double)(per_sm * sms);
-      const double score =
-          std::min(busy, 12.0) * balance * lpc_efficiency(lpc) + 1e-3 * warps - 1e-4 * tt;
+      const double score = score_of(grid);
       if (score > best.score) best = Cand{lpc, warps, tt, DT, occ, (int)grid, rows, smem, score};
     }
   }
   if (best.score < 0) return SSM_ERR_UNSUPPORTED;  // no variant fits (or bad override)
   const int64_t S = (d.seqlen + best.tt - 1) / best.tt;
-  if (best.rows * S > INT32_MAX) return SSM_ERR_UNSUPPORTED;
+  const int m0 = parts_per_row(best.rows, best.grid, S);
+  const int64_t PL = (S + m0 - 1) / m0;
+  const int64_t m = (S + PL - 1) / PL;
+  if (best.rows * S > INT32_MAX || best.rows * m > INT32_MAX) return SSM_ERR_UNSUPPORTED;
   ssm::LaunchShape ls{best.lpc, best.warps, best.tt, kStages, ns,
-                      (int)std::max<int64_t>(1, std::min<int64_t>(best.grid, best.rows * S)),
+                      (int)std::max<int64_t>(1, std::min<int64_t>(best.grid, best.rows * m)),
                       best.smem};
   // workspace: carried state per (row, channel, n) and a flag per (row, warp)
   const size_t st_bytes = (size_t)best.rows * best.DT * ns * sizeof(float);
@@ -211,6 +238,8 @@ ssm_status plan_tma(ssm_scan_plan *pl) {
   pl->DT = best.DT;
   pl->nDT = (int)((d.dim + best.DT - 1) / best.DT);
   pl->S = (int)S;
+  pl->PL = (int)PL;
+  pl->parts = (int)m;
   pl->rows = best.rows;
   pl->units = best.rows * S;
   return SSM_OK;
@@ -317,6 +346,8 @@ ssm_status ssm_scan_get_info(const ssm_scan_plan *pl, ssm_scan_info *info) {
     info->grid = pl->ls.grid;
     info->rows = pl->rows;
     info->units = pl->units;
+    info->parts_per_row = pl->parts;
+    info->stages_per_part = pl->PL;
     info->smem_bytes = pl->ls.smem;
   }
   info->workspace_bytes = pl->ws_state_bytes + pl->ws_flag_bytes + sizeof(ssm::Control);
@@ -418,6 +449,7 @@ ssm_status ssm_scan_fwd(ssm_scan_plan *pl, const void *x, const void *delta,
     ssm::FwdParams p{};
     p.Bsz = (int)d.batch; p.L = (int)d.seqlen; p.D = (int)d.dim; p.N = (int)d.dstate;
     p.DT = pl->DT; p.nDT = pl->nDT; p.rows = (int)pl->rows; p.S = pl->S;
+    p.PL = pl->PL; p.items = (int)(pl->rows * pl->parts);
     p.softplus = (f & SSM_DELTA_SOFTPLUS) != 0;
     p.has_z = (f & SSM_HAS_Z) != 0;
     p.has_D = (f & SSM_HAS_D) != 0;

@@ -188,16 +188,18 @@ def test_decode_steps_match_full_sequence(N, dt):
 
 
 def test_timeout_is_reported_without_hanging():
-    """A CTA that never hands its state on makes the CTA continuing that row
-    wait until the bound expires: the kernel records SSM_ERR_TIMEOUT and
-    returns; the plan stays usable and the next call is exact again."""
-    inp = synth.make_fwd(1, 512, 32, 16, seed=34)
+    """A work item that never hands its state on makes the CTA running the
+    next part of that row wait until the bound expires: the kernel records
+    SSM_ERR_TIMEOUT and returns; the plan stays usable and the next call is
+    exact again."""
+    inp = synth.make_fwd(4, 512, 32, 16, seed=34)
     plan = gu.make_plan(inp)
     plan.set_config(lanes_per_chan=4, warps_per_cta=4, grid=3)
     info = plan.info()
-    assert info["rows"] == 1 and info["stages_per_row"] == 16 and info["grid"] == 3, info
-    # CTA 0 runs units [0, 5) of the single row and hands over after unit 4
-    plan.set_debug(wait_timeout_ns=50_000_000, drop_unit=4)
+    S, PL = info["stages_per_row"], info["stages_per_part"]
+    assert info["rows"] == 4 and info["grid"] == 3 and info["parts_per_row"] >= 2, info
+    # the first part of row 2 ends at stage PL - 1; the CTA running part 2 of row 2 waits for it
+    plan.set_debug(wait_timeout_ns=50_000_000, drop_unit=2 * S + PL - 1)
     dev = gu.upload(inp)
     gu.run_gpu(inp, plan, dev)
     assert plan.status() == 5  # SSM_ERR_TIMEOUT
