@@ -125,8 +125,8 @@ typedef struct {
 
 /* Optional overrides of the launch shape (0 = keep the default). */
 typedef struct {
-  int lanes_per_chan; /* 1, 2, 4, 8 (<= dstate) */
-  int warps_per_cta;  /* 2 or 4 */
+  int lanes_per_chan; /* 1, 2, 4, 8, 16 (<= dstate) */
+  int warps_per_cta;  /* scan warps: 2, 4 or 8 (plus one load warp) */
   int grid;           /* CTAs (clamped to what is co-resident on the device) */
   int tile_t;         /* tokens per pipeline stage: 16, 32 or 64 */
 } ssm_scan_config;

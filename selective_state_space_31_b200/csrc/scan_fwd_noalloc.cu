@@ -36,8 +36,6 @@ namespace {
 constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
 constexpr size_t kCtlBytes = 256;
 constexpr int kMaxDevices = 64;
-constexpr int kTTna = 16;
-constexpr int kStagesNa = 2;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
@@ -129,85 +127,39 @@ extern "C" SSM_API ssm_status ssm_scan_fwd_noalloc(
     cudaGetLastError();
     return SSM_ERR_CUDA;
   }
-  // launch shape: the same choice a plan makes by default (most busy warps
-  // per SM, capped at 10 and weighted by the cost of splitting channels)
-  struct Cand { int lpc, warps, DT, grid; int64_t rows; size_t smem; double score; };
-  Cand best{};
-  best.score = -1.0;
-  for (int lpc : {1, 2, 4, 8}) {
-    if (lpc > ns) continue;
-    const double eff = lpc == 1 ? 1.0 : lpc == 2 ? 0.95 : lpc == 4 ? 0.9 : 0.55;
-    for (int warps : {2, 4}) {
-      const int DT = warps * 32 / lpc;
-      if ((DT * (int)ei) % 16 || (DT * (int)eo) % 16) continue;
-      ssm::LaunchShape probe{lpc, warps, kTTna, kStagesNa, ns, 0, 0};
-      int occ = 0;
-      size_t smem = 0;
-      if (ssm::fwd_tma_smem_and_occupancy((int)d.in_dtype, (int)d.out_dtype, probe, &smem,
-                                          &occ) != cudaSuccess ||
-          occ < 1) {
-        cudaGetLastError();
-        continue;
-      }
-      const int64_t rows = d.batch * ((d.dim + DT - 1) / DT);
-      const int64_t cap = std::min<int64_t>(rows, (int64_t)occ * num_sms);
-      const int64_t balanced = cap >= num_sms ? cap / num_sms * num_sms : cap;
-      auto score_of = [&](int64_t g) {
-        const int64_t per_sm = (g + num_sms - 1) / num_sms;
-        const double busy = (double)g * warps / num_sms;
-        const double balance = (double)g / (double)(per_sm * num_sms);
-        const double tie = busy >= 10.0 ? -1e-3 * warps : 1e-3 * warps;
-        return std::min(busy, 10.0) * balance * eff + tie;
-      };
-      const int64_t grid = score_of(balanced) >= score_of(cap) ? balanced : cap;
-      const double score = score_of(grid);
-      if (score > best.score) best = Cand{lpc, warps, DT, (int)grid, rows, smem, score};
-    }
+  // launch shape: the same choice a plan makes by default
+  ssm::FwdShape fs;
+  if (ssm::choose_fwd_shape((int)d.in_dtype, (int)d.out_dtype, d.batch, d.seqlen, d.dim, ns,
+                            num_sms, ssm::FwdOverrides{0, 0, 0, 0}, &fs) != cudaSuccess) {
+    cudaGetLastError();
+    return SSM_ERR_UNSUPPORTED;
   }
-  if (best.score < 0) return SSM_ERR_UNSUPPORTED;
-  const int DT = best.DT, warps = best.warps;
+  const int DT = fs.DT, warps = fs.ls.warps, TT = fs.ls.tt;
   const int nDT = (int)((d.dim + DT - 1) / DT);
-  const int64_t rows = best.rows;
-  const int64_t S = (d.seqlen + kTTna - 1) / kTTna;
-  // parts per row: the fewest that keep every CTA within ~5% of the mean
-  int m = 1;
-  if (best.grid < rows) {
-    double best_bal = 0.0;
-    for (int mm = 1; mm <= 64 && mm <= S; ++mm) {
-      const int64_t it = rows * mm;
-      const double bal = ((double)it / best.grid) / (double)((it + best.grid - 1) / best.grid);
-      if (bal > best_bal + 1e-9) { best_bal = bal; m = mm; }
-      if (bal >= 0.95) break;
-    }
-  }
-  const int64_t PL = (S + m - 1) / m;
-  const int64_t parts = (S + PL - 1) / PL;
-  if (rows * S > INT32_MAX || rows * parts > INT32_MAX) return SSM_ERR_UNSUPPORTED;
+  const int64_t rows = fs.rows;
   // scratch layout: [Control | flags rows*warps u64 | states rows*DT*N f32]
   const size_t fl_bytes = (size_t)rows * warps * sizeof(unsigned long long);
   const size_t st_off = (kCtlBytes + fl_bytes + 255) / 256 * 256;
   const size_t need = st_off + (size_t)rows * DT * ns * sizeof(float);
   if (need > kNoAllocScratchBytes) return SSM_ERR_UNSUPPORTED;  // beyond the fixed scratch
-  ssm::LaunchShape ls{best.lpc, warps, kTTna, kStagesNa, ns,
-                      (int)std::max<int64_t>(1, std::min<int64_t>(best.grid, rows * parts)),
-                      best.smem};
+  const ssm::LaunchShape ls = fs.ls;
 
   unsigned char *base = static_cast<unsigned char *>(scratch_address(device));
   if (!base) return SSM_ERR_CUDA;
 
   ssm::TmaMaps maps;
   const uint64_t Bn = d.batch, L = d.seqlen, Dm = d.dim, N = d.dstate;
-  if (!encode_na(&maps.x, d.in_dtype, x, Dm, L, Bn, DT, kTTna) ||
-      !encode_na(&maps.dt, d.in_dtype, delta, Dm, L, Bn, DT, kTTna) ||
-      !encode_na(&maps.z, d.in_dtype, z ? z : x, Dm, L, Bn, DT, kTTna) ||
-      !encode_na(&maps.B, d.in_dtype, B, N, L, Bn, (uint32_t)N, kTTna) ||
-      !encode_na(&maps.C, d.in_dtype, C, N, L, Bn, (uint32_t)N, kTTna))
+  if (!encode_na(&maps.x, d.in_dtype, x, Dm, L, Bn, DT, TT) ||
+      !encode_na(&maps.dt, d.in_dtype, delta, Dm, L, Bn, DT, TT) ||
+      !encode_na(&maps.z, d.in_dtype, z ? z : x, Dm, L, Bn, DT, TT) ||
+      !encode_na(&maps.B, d.in_dtype, B, N, L, Bn, (uint32_t)N, TT) ||
+      !encode_na(&maps.C, d.in_dtype, C, N, L, Bn, (uint32_t)N, TT))
     return SSM_ERR_CUDA;
 
   ssm::FwdParams p{};
   p.Bsz = (int)d.batch; p.L = (int)d.seqlen; p.D = (int)d.dim; p.N = ns;
-  p.DT = DT; p.nDT = nDT; p.rows = (int)rows; p.S = (int)S;
-  p.PL = (int)PL; p.items = (int)(rows * parts);
+  p.DT = DT; p.nDT = nDT; p.rows = (int)rows; p.S = fs.S;
+  p.PL = fs.PL; p.items = (int)(rows * fs.parts);
   p.softplus = (f & SSM_DELTA_SOFTPLUS) != 0;
   p.has_z = (f & SSM_HAS_Z) != 0;
   p.has_D = (f & SSM_HAS_D) != 0;

@@ -58,6 +58,28 @@ cudaError_t launch_fwd_tma(int in_dtype, int out_dtype, const LaunchShape &ls,
 cudaError_t fwd_tma_smem_and_occupancy(int in_dtype, int out_dtype, const LaunchShape &ls,
                                        size_t *smem, int *blocks_per_sm);
 
+// Pipeline tag every fused-kernel LaunchShape carries (`stages`).
+constexpr int kStages = 2;
+
+// Launch-shape overrides (0 = free choice).
+struct FwdOverrides {
+  int lpc, warps, tt, grid;
+};
+// A launch shape of the fused kernel with its work split.
+struct FwdShape {
+  LaunchShape ls;  // lpc, warps, tt, stages, ns, grid, smem
+  int DT;          // channels per row tile
+  int64_t rows;    // batch * ceil(dim / DT)
+  int S;           // stages per row
+  int PL;          // stages per part
+  int parts;       // parts per row
+};
+// Choose the fused kernel's launch shape for a problem (scan_fwd_dispatch.cu).
+// Returns cudaErrorInvalidValue when no variant fits the overrides.
+cudaError_t choose_fwd_shape(int in_dtype, int out_dtype, int64_t batch, int64_t seqlen,
+                             int64_t dim, int ns, int sms, const FwdOverrides &o,
+                             FwdShape *out);
+
 struct GenericParams {
   int Bsz, L, D, N;
   bool softplus, has_z, has_D, has_bias, has_h0, want_hlast;

@@ -20,8 +20,6 @@ namespace {
 constexpr uint32_t kKnownFlags = SSM_HAS_Z | SSM_HAS_D | SSM_DELTA_SOFTPLUS | SSM_HAS_DELTA_BIAS |
                                  SSM_HAS_H0 | SSM_WANT_HLAST | SSM_A_DIRECT;
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
-constexpr int kTTDefault = 32;  // default stage length (work unit) of the fused kernel
-constexpr int kStages = 2;      // TMA slots of the fused kernel
 constexpr int kMaxDstate = 64;
 
 enum Path { PATH_TMA = 0, PATH_GENERAL = 1, PATH_DIRECT = 2 };
@@ -124,100 +122,24 @@ bool tma_eligible(const ssm_scan_desc &d) {
   return true;
 }
 
-// Measured relative efficiency of each lanes-per-channel choice (B200,
-// consumer scan loop at equal warps per SM): splitting a channel's states over
-// more lanes adds shuffles and shared loads per update.
-double lpc_efficiency(int lpc) {
-  switch (lpc) {
-    case 1: return 1.0;
-    case 2: return 0.95;
-    case 4: return 0.9;
-    default: return 0.55;
-  }
-}
-
-// Parts per row for P CTAs over R rows of S stages: the fewest parts that
-// keep every CTA within ~5% of the mean item count (P <= R).
-int parts_per_row(int64_t R, int64_t P, int64_t S) {
-  if (P >= R) return 1;
-  int best_m = 1;
-  double best_bal = 0.0;
-  for (int m = 1; m <= 64 && m <= S; ++m) {
-    const int64_t items = R * m;
-    const double mean = (double)items / P;
-    const double bal = mean / (double)((items + P - 1) / P);
-    if (bal > best_bal + 1e-9) { best_bal = bal; best_m = m; }
-    if (bal >= 0.95) return m;
-  }
-  return best_m;
-}
-
-// Choose the launch shape of the fused kernel and size the workspace.  Rows
-// (batch x channel tiles) are the only independent chains, so at most `rows`
-// CTAs can be busy: grid P <= min(rows, CTAs resident on the device), taken
-// as a multiple of the SM count when that keeps enough warps (every SM then
-// gets the same work).  Among the variants, pick the most busy consumer warps
-// per SM (capped at 10), discounted for uneven CTAs per SM and for the
-// instruction cost of splitting channels across lanes.  Ties: once an SM holds
-// 10 consumer warps, more CTAs of fewer warps (more independent producer
-// pipelines) measured faster on B200; below that, wider CTAs did.
+// Choose the launch shape of the fused kernel (shared with the
+// allocation-free entry point) and size the workspace.
 ssm_status plan_tma(ssm_scan_plan *pl) {
   const ssm_scan_desc &d = pl->desc;
   const int ns = (int)d.dstate;
-  const int sms = pl->num_sms;
-  const int ei = (int)dtype_size(d.in_dtype), eo = (int)dtype_size(d.out_dtype);
   if (pl->cfg.tile_t && pl->cfg.tile_t != 16 && pl->cfg.tile_t != 32 && pl->cfg.tile_t != 64)
     return SSM_ERR_INVALID_ARG;
-  struct Cand { int lpc, warps, tt, DT, occ, grid; int64_t rows; size_t smem; double score; };
-  Cand best{};
-  best.score = -1.0;
-  for (int lpc : {1, 2, 4, 8}) {
-    if (lpc > ns) continue;
-    if (pl->cfg.lanes_per_chan && lpc != pl->cfg.lanes_per_chan) continue;
-    for (int warps : {2, 4})
-    for (int tt : {kTTDefault, 16}) {
-      if (pl->cfg.warps_per_cta && warps != pl->cfg.warps_per_cta) continue;
-      if (pl->cfg.tile_t ? tt != pl->cfg.tile_t : false) continue;
-      const int DT = warps * 32 / lpc;
-      if ((DT * ei) % 16 || (DT * eo) % 16) continue;
-      ssm::LaunchShape ls{lpc, warps, tt, kStages, ns, 0, 0};
-      int occ = 0;
-      size_t smem = 0;
-      if (ssm::fwd_tma_smem_and_occupancy((int)d.in_dtype, (int)d.out_dtype, ls, &smem, &occ) !=
-              cudaSuccess ||
-          occ < 1) {
-        cudaGetLastError();
-        continue;
-      }
-      const int64_t rows = d.batch * ((d.dim + DT - 1) / DT);
-      const int64_t cap = std::min<int64_t>(rows, (int64_t)occ * sms);
-      // either all that fits, or the largest multiple of the SM count below it
-      const int64_t balanced = cap >= sms ? cap / sms * sms : cap;
-      auto score_of = [&](int64_t g) {
-        const int64_t per_sm = (g + sms - 1) / sms;  // CTAs on the busiest SM
-        const double busy = (double)g * warps / sms;
-        const double balance = (double)g / (double)(per_sm * sms);
-        const double tie = busy >= 10.0 ? -1e-3 * warps : 1e-3 * warps;
-        return std::min(busy, 10.0) * balance * lpc_efficiency(lpc) + tie - 1e-4 * tt;
-      };
-      int64_t grid = score_of(balanced) >= score_of(cap) ? balanced : cap;
-      if (pl->cfg.grid > 0) grid = std::min<int64_t>(pl->cfg.grid, (int64_t)occ * sms);
-      const double score = score_of(grid);
-      if (score > best.score) best = Cand{lpc, warps, tt, DT, occ, (int)grid, rows, smem, score};
-    }
+  const ssm::FwdOverrides o{pl->cfg.lanes_per_chan, pl->cfg.warps_per_cta, pl->cfg.tile_t,
+                            pl->cfg.grid};
+  ssm::FwdShape fs;
+  if (ssm::choose_fwd_shape((int)d.in_dtype, (int)d.out_dtype, d.batch, d.seqlen, d.dim, ns,
+                            pl->num_sms, o, &fs) != cudaSuccess) {
+    cudaGetLastError();
+    return SSM_ERR_UNSUPPORTED;  // no variant fits (or bad override)
   }
-  if (best.score < 0) return SSM_ERR_UNSUPPORTED;  // no variant fits (or bad override)
-  const int64_t S = (d.seqlen + best.tt - 1) / best.tt;
-  const int m0 = parts_per_row(best.rows, best.grid, S);
-  const int64_t PL = (S + m0 - 1) / m0;
-  const int64_t m = (S + PL - 1) / PL;
-  if (best.rows * S > INT32_MAX || best.rows * m > INT32_MAX) return SSM_ERR_UNSUPPORTED;
-  ssm::LaunchShape ls{best.lpc, best.warps, best.tt, kStages, ns,
-                      (int)std::max<int64_t>(1, std::min<int64_t>(best.grid, best.rows * m)),
-                      best.smem};
   // workspace: carried state per (row, channel, n) and a flag per (row, warp)
-  const size_t st_bytes = (size_t)best.rows * best.DT * ns * sizeof(float);
-  const size_t fl_bytes = (size_t)best.rows * best.warps * sizeof(unsigned long long);
+  const size_t st_bytes = (size_t)fs.rows * fs.DT * ns * sizeof(float);
+  const size_t fl_bytes = (size_t)fs.rows * fs.ls.warps * sizeof(unsigned long long);
   if (st_bytes > pl->ws_state_bytes) {
     if (pl->ws_state) cudaFree(pl->ws_state);
     pl->ws_state = nullptr;
@@ -234,14 +156,14 @@ ssm_status plan_tma(ssm_scan_plan *pl) {
   }
   // flags start below every epoch tag (epochs start at 1)
   if (cudaMemset(pl->ws_flags, 0, pl->ws_flag_bytes) != cudaSuccess) return SSM_ERR_CUDA;
-  pl->ls = ls;
-  pl->DT = best.DT;
-  pl->nDT = (int)((d.dim + best.DT - 1) / best.DT);
-  pl->S = (int)S;
-  pl->PL = (int)PL;
-  pl->parts = (int)m;
-  pl->rows = best.rows;
-  pl->units = best.rows * S;
+  pl->ls = fs.ls;
+  pl->DT = fs.DT;
+  pl->nDT = (int)((d.dim + fs.DT - 1) / fs.DT);
+  pl->S = fs.S;
+  pl->PL = fs.PL;
+  pl->parts = fs.parts;
+  pl->rows = fs.rows;
+  pl->units = fs.rows * fs.S;
   return SSM_OK;
 }
 
