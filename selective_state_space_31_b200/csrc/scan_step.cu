@@ -20,43 +20,77 @@ __device__ __forceinline__ float ld1(const void *base, size_t i) {
   return to_f32(reinterpret_cast<const T *>(base)[i]);
 }
 
+// NPT consecutive B or C values of one batch row (16-byte aligned) as fp32.
+template <int NPT>
+__device__ __forceinline__ void ldg_vec(const float *src, float (&v)[NPT]) {
+#pragma unroll
+  for (int i = 0; i < NPT; i += 4) {
+    const float4 w = __ldg(reinterpret_cast<const float4 *>(src + i));
+    v[i] = w.x; v[i + 1] = w.y; v[i + 2] = w.z; v[i + 3] = w.w;
+  }
+}
+template <int NPT>
+__device__ __forceinline__ void ldg_vec(const __nv_bfloat16 *src, float (&v)[NPT]) {
+  if constexpr (NPT % 8 == 0) {
+#pragma unroll
+    for (int i = 0; i < NPT; i += 8) {
+      const uint4 w = __ldg(reinterpret_cast<const uint4 *>(src + i));
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {  // a bf16 is the upper half of the equal fp32
+        v[i + 2 * k] = __uint_as_float(ws[k] << 16);
+        v[i + 2 * k + 1] = __uint_as_float(ws[k] & 0xffff0000u);
+      }
+    }
+  } else {
+    const uint2 w = __ldg(reinterpret_cast<const uint2 *>(src));
+    v[0] = __uint_as_float(w.x << 16);
+    v[1] = __uint_as_float(w.x & 0xffff0000u);
+    v[2] = __uint_as_float(w.y << 16);
+    v[3] = __uint_as_float(w.y & 0xffff0000u);
+  }
+}
+
 template <typename InT, typename OutT, int NPT, int TPC>
 __global__ void __launch_bounds__(256) step_kernel(const StepParams p) {
   const long long gt = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const long long chn = gt / TPC;
   const int q = (int)(gt % TPC);
   const bool active = chn < (long long)p.Bsz * p.D;
-  const int N = NPT * TPC;
+  constexpr int N = NPT * TPC;
   float acc = 0.f, xv = 0.f, zv = 0.f, Dd = 0.f;
-  int b = 0, d = 0;
-  float h[NPT];
-  float *sp = nullptr;
   if (active) {
-    b = (int)(chn / p.D);
-    d = (int)(chn % p.D);
+    // the state first: its HBM reads are the long pole, everything else is
+    // cache-resident (A, bias, D) or small (per-token vectors)
+    float4 *sp = reinterpret_cast<float4 *>(p.state + (size_t)chn * N + q * NPT);
+    float4 s4[NPT / 4];
+#pragma unroll
+    for (int i = 0; i < NPT / 4; ++i) s4[i] = __ldcs(sp + i);
+    const int b = (int)(chn / p.D), d = (int)(chn % p.D);
+    float Av[NPT], Bv[NPT], Cv[NPT];
+    ldg_vec<NPT>(p.A + (size_t)d * N + q * NPT, Av);
+    ldg_vec<NPT>(reinterpret_cast<const InT *>(p.B) + (size_t)b * N + q * NPT, Bv);
+    ldg_vec<NPT>(reinterpret_cast<const InT *>(p.C) + (size_t)b * N + q * NPT, Cv);
     xv = ld1<InT>(p.x, (size_t)chn);
     const float v = ld1<InT>(p.dt, (size_t)chn) + (p.has_bias ? __ldg(p.bias + d) : 0.f);
-    const float dlt = p.softplus ? softplus_f(v) : v;
-    const float dtx = dlt * xv;
     if (p.has_z) zv = ld1<InT>(p.z, (size_t)chn);
     if (p.has_D) Dd = __ldg(p.Dv + d);
-    sp = p.state + (size_t)chn * N + q * NPT;
+    const float dlt = p.softplus ? softplus_f(v) : v;
+    const float dtx = dlt * xv;
+    float h[NPT];
 #pragma unroll
-    for (int i = 0; i < NPT; i += 4) {
-      const float4 s4 = __ldcs(reinterpret_cast<const float4 *>(sp + i));
-      h[i] = s4.x; h[i + 1] = s4.y; h[i + 2] = s4.z; h[i + 3] = s4.w;
+    for (int i = 0; i < NPT / 4; ++i) {
+      h[4 * i] = s4[i].x; h[4 * i + 1] = s4[i].y; h[4 * i + 2] = s4[i].z; h[4 * i + 3] = s4[i].w;
     }
-    const float *Ar = p.A + (size_t)d * N + q * NPT;
-    const size_t bc = (size_t)b * N + q * NPT;
 #pragma unroll
     for (int n = 0; n < NPT; ++n) {
-      const float a = ex2_approx(dlt * (__ldg(Ar + n) * kLog2e));
-      h[n] = fmaf(a, h[n], dtx * ld1<InT>(p.B, bc + n));
-      acc = fmaf(ld1<InT>(p.C, bc + n), h[n], acc);
+      const float a = ex2_approx(dlt * (Av[n] * kLog2e));
+      h[n] = fmaf(a, h[n], dtx * Bv[n]);
+      acc = fmaf(Cv[n], h[n], acc);
     }
 #pragma unroll
-    for (int i = 0; i < NPT; i += 4)
-      __stcs(reinterpret_cast<float4 *>(sp + i), make_float4(h[i], h[i + 1], h[i + 2], h[i + 3]));
+    for (int i = 0; i < NPT / 4; ++i)
+      __stcs(sp + i, make_float4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]));
   }
 #pragma unroll
   for (int m = TPC / 2; m >= 1; m >>= 1) acc += __shfl_xor_sync(FULL_MASK, acc, m);
@@ -110,7 +144,8 @@ static cudaError_t step_typed(const StepParams &p, bool vec_ok, cudaStream_t str
 }
 
 cudaError_t launch_step(const StepParams &p, cudaStream_t stream) {
-  const bool vec_ok = (reinterpret_cast<uintptr_t>(p.state) % 16) == 0;
+  auto al16 = [](const void *q) { return (reinterpret_cast<uintptr_t>(q) % 16) == 0; };
+  const bool vec_ok = al16(p.state) && al16(p.A) && al16(p.B) && al16(p.C);
   if (!p.in_bf16 && !p.out_bf16) return step_typed<float, float>(p, vec_ok, stream);
   if (p.in_bf16 && p.out_bf16) return step_typed<__nv_bfloat16, __nv_bfloat16>(p, vec_ok, stream);
   if (p.in_bf16) return step_typed<__nv_bfloat16, float>(p, vec_ok, stream);
