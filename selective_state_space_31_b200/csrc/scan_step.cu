@@ -13,6 +13,10 @@
 #include "device_common.cuh"
 #include "scan_params.h"
 
+#ifndef SSM_STEP_ITEMS
+#define SSM_STEP_ITEMS 1
+#endif
+
 namespace ssm {
 
 template <typename T>
@@ -51,53 +55,67 @@ __device__ __forceinline__ void ldg_vec(const __nv_bfloat16 *src, float (&v)[NPT
   }
 }
 
-template <typename InT, typename OutT, int NPT, int TPC>
+template <typename InT, typename OutT, int NPT, int TPC, int ITEMS>
 __global__ void __launch_bounds__(256) step_kernel(const StepParams p) {
-  const long long gt = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  const long long chn = gt / TPC;
-  const int q = (int)(gt % TPC);
-  const bool active = chn < (long long)p.Bsz * p.D;
+  // ITEMS work items per thread, a grid apart: every item's state reads are
+  // issued before any of them is used, so each thread keeps ITEMS x NPT x 4
+  // bytes of HBM reads in flight
+  const long long total = (long long)gridDim.x * blockDim.x;
+  const long long g0 = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long nch = (long long)p.Bsz * p.D;
   constexpr int N = NPT * TPC;
-  float acc = 0.f, xv = 0.f, zv = 0.f, Dd = 0.f;
-  if (active) {
-    // the state first: its HBM reads are the long pole, everything else is
-    // cache-resident (A, bias, D) or small (per-token vectors)
-    float4 *sp = reinterpret_cast<float4 *>(p.state + (size_t)chn * N + q * NPT);
-    float4 s4[NPT / 4];
+  const int q = (int)(g0 % TPC);  // the same for every item (total is a multiple of TPC)
+  float4 s4[ITEMS][NPT / 4];
 #pragma unroll
-    for (int i = 0; i < NPT / 4; ++i) s4[i] = __ldcs(sp + i);
-    const int b = (int)(chn / p.D), d = (int)(chn % p.D);
-    float Av[NPT], Bv[NPT], Cv[NPT];
-    ldg_vec<NPT>(p.A + (size_t)d * N + q * NPT, Av);
-    ldg_vec<NPT>(reinterpret_cast<const InT *>(p.B) + (size_t)b * N + q * NPT, Bv);
-    ldg_vec<NPT>(reinterpret_cast<const InT *>(p.C) + (size_t)b * N + q * NPT, Cv);
-    xv = ld1<InT>(p.x, (size_t)chn);
-    const float v = ld1<InT>(p.dt, (size_t)chn) + (p.has_bias ? __ldg(p.bias + d) : 0.f);
-    if (p.has_z) zv = ld1<InT>(p.z, (size_t)chn);
-    if (p.has_D) Dd = __ldg(p.Dv + d);
-    const float dlt = p.softplus ? softplus_f(v) : v;
-    const float dtx = dlt * xv;
-    float h[NPT];
+  for (int it = 0; it < ITEMS; ++it) {
+    const long long chn = (g0 + it * total) / TPC;
+    if (chn < nch) {
+      const float4 *sp = reinterpret_cast<const float4 *>(p.state + (size_t)chn * N + q * NPT);
 #pragma unroll
-    for (int i = 0; i < NPT / 4; ++i) {
-      h[4 * i] = s4[i].x; h[4 * i + 1] = s4[i].y; h[4 * i + 2] = s4[i].z; h[4 * i + 3] = s4[i].w;
+      for (int i = 0; i < NPT / 4; ++i) s4[it][i] = __ldcs(sp + i);
     }
-#pragma unroll
-    for (int n = 0; n < NPT; ++n) {
-      const float a = ex2_approx(dlt * (Av[n] * kLog2e));
-      h[n] = fmaf(a, h[n], dtx * Bv[n]);
-      acc = fmaf(Cv[n], h[n], acc);
-    }
-#pragma unroll
-    for (int i = 0; i < NPT / 4; ++i)
-      __stcs(sp + i, make_float4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]));
   }
 #pragma unroll
-  for (int m = TPC / 2; m >= 1; m >>= 1) acc += __shfl_xor_sync(FULL_MASK, acc, m);
-  if (active && q == 0) {
-    float yv = fmaf(Dd, xv, acc);
-    if (p.has_z) yv *= silu_f(zv);
-    reinterpret_cast<OutT *>(p.y)[chn] = from_f32<OutT>(yv);
+  for (int it = 0; it < ITEMS; ++it) {
+    const long long chn = (g0 + it * total) / TPC;
+    const bool active = chn < nch;
+    float acc = 0.f, xv = 0.f, zv = 0.f, Dd = 0.f;
+    if (active) {
+      const int b = (int)(chn / p.D), d = (int)(chn % p.D);
+      float Av[NPT], Bv[NPT], Cv[NPT];
+      ldg_vec<NPT>(p.A + (size_t)d * N + q * NPT, Av);
+      ldg_vec<NPT>(reinterpret_cast<const InT *>(p.B) + (size_t)b * N + q * NPT, Bv);
+      ldg_vec<NPT>(reinterpret_cast<const InT *>(p.C) + (size_t)b * N + q * NPT, Cv);
+      xv = ld1<InT>(p.x, (size_t)chn);
+      const float v = ld1<InT>(p.dt, (size_t)chn) + (p.has_bias ? __ldg(p.bias + d) : 0.f);
+      if (p.has_z) zv = ld1<InT>(p.z, (size_t)chn);
+      if (p.has_D) Dd = __ldg(p.Dv + d);
+      const float dlt = p.softplus ? softplus_f(v) : v;
+      const float dtx = dlt * xv;
+      float h[NPT];
+#pragma unroll
+      for (int i = 0; i < NPT / 4; ++i) {
+        h[4 * i] = s4[it][i].x; h[4 * i + 1] = s4[it][i].y;
+        h[4 * i + 2] = s4[it][i].z; h[4 * i + 3] = s4[it][i].w;
+      }
+#pragma unroll
+      for (int n = 0; n < NPT; ++n) {
+        const float a = ex2_approx(dlt * (Av[n] * kLog2e));
+        h[n] = fmaf(a, h[n], dtx * Bv[n]);
+        acc = fmaf(Cv[n], h[n], acc);
+      }
+      float4 *sp = reinterpret_cast<float4 *>(p.state + (size_t)chn * N + q * NPT);
+#pragma unroll
+      for (int i = 0; i < NPT / 4; ++i)
+        __stcs(sp + i, make_float4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]));
+    }
+#pragma unroll
+    for (int m = TPC / 2; m >= 1; m >>= 1) acc += __shfl_xor_sync(FULL_MASK, acc, m);
+    if (active && q == 0) {
+      float yv = fmaf(Dd, xv, acc);
+      if (p.has_z) yv *= silu_f(zv);
+      reinterpret_cast<OutT *>(p.y)[chn] = from_f32<OutT>(yv);
+    }
   }
 }
 
@@ -128,14 +146,15 @@ template <typename InT, typename OutT>
 static cudaError_t step_typed(const StepParams &p, bool vec_ok, cudaStream_t stream) {
   const long long chans = (long long)p.Bsz * p.D;
   if (chans == 0) return cudaSuccess;
-  auto grid_for = [&](int tpc) { return (unsigned)((chans * tpc + 255) / 256); };
+  constexpr int IT = SSM_STEP_ITEMS;
+  auto grid_for = [&](int tpc) { return (unsigned)((chans * tpc + 256 * IT - 1) / (256 * IT)); };
   if (vec_ok) {
     switch (p.N) {
-      case 4: step_kernel<InT, OutT, 4, 1><<<grid_for(1), 256, 0, stream>>>(p); return cudaGetLastError();
-      case 8: step_kernel<InT, OutT, 8, 1><<<grid_for(1), 256, 0, stream>>>(p); return cudaGetLastError();
-      case 16: step_kernel<InT, OutT, 8, 2><<<grid_for(2), 256, 0, stream>>>(p); return cudaGetLastError();
-      case 32: step_kernel<InT, OutT, 8, 4><<<grid_for(4), 256, 0, stream>>>(p); return cudaGetLastError();
-      case 64: step_kernel<InT, OutT, 8, 8><<<grid_for(8), 256, 0, stream>>>(p); return cudaGetLastError();
+      case 4: step_kernel<InT, OutT, 4, 1, IT><<<grid_for(1), 256, 0, stream>>>(p); return cudaGetLastError();
+      case 8: step_kernel<InT, OutT, 8, 1, IT><<<grid_for(1), 256, 0, stream>>>(p); return cudaGetLastError();
+      case 16: step_kernel<InT, OutT, 8, 2, IT><<<grid_for(2), 256, 0, stream>>>(p); return cudaGetLastError();
+      case 32: step_kernel<InT, OutT, 8, 4, IT><<<grid_for(4), 256, 0, stream>>>(p); return cudaGetLastError();
+      case 64: step_kernel<InT, OutT, 8, 8, IT><<<grid_for(8), 256, 0, stream>>>(p); return cudaGetLastError();
       default: break;
     }
   }

@@ -187,6 +187,28 @@ def test_decode_steps_match_full_sequence(N, dt):
     gu.assert_parity(y, ry, state.cpu().numpy(), rh, gu.TOL[dt], f"decode N={N}")
 
 
+def test_decode_streaming_many_tiles_per_cta():
+    """Enough channels that the streaming step kernel's CTAs each run several
+    state tiles through their ring, with a ragged last tile (16 x 4004
+    channels = 1001 tiles of 64): three steps against the oracle on every
+    channel."""
+    import oracle
+    from selective_state_space_31_b200 import binding as bnd
+    inp = synth.make_fwd(16, 3, 4004, 16, in_dtype="bf16", seed=35, has_h0=True)
+    dev = gu.upload(inp)
+    state = dev["h0"].clone()
+    ys = []
+    for t in range(inp.L):
+        ys.append(bnd.step(state, dev["x"][:, t].contiguous(), dev["delta"][:, t].contiguous(),
+                           dev["A"], dev["B"][:, t].contiguous(), dev["C"][:, t].contiguous(),
+                           D=dev["D"], z=dev["z"][:, t].contiguous(),
+                           delta_bias=dev["delta_bias"]))
+    y = torch.stack(ys, dim=1).float().cpu().numpy()
+    ry, rh = oracle.get().fwd(inp.x, inp.delta, inp.A, inp.B, inp.C, D=inp.Dskip, z=inp.z,
+                              delta_bias=inp.delta_bias, h0=inp.h0)
+    gu.assert_parity(y, ry, state.cpu().numpy(), rh, gu.TOL["bf16"], "decode, many tiles")
+
+
 def test_timeout_is_reported_without_hanging():
     """A work item that never hands its state on makes the CTA running the
     next part of that row wait until the bound expires: the kernel records
