@@ -13,6 +13,9 @@
 #include "device_common.cuh"
 #include "scan_params.h"
 
+#ifndef SSM_STEP_MINB
+#define SSM_STEP_MINB 1
+#endif
 #ifndef SSM_STEP_ITEMS
 #define SSM_STEP_ITEMS 1
 #endif
@@ -24,55 +27,40 @@ __device__ __forceinline__ float ld1(const void *base, size_t i) {
   return to_f32(reinterpret_cast<const T *>(base)[i]);
 }
 
-// NPT consecutive B or C values of one batch row (16-byte aligned) as fp32.
-template <int NPT>
-__device__ __forceinline__ void ldg_vec(const float *src, float (&v)[NPT]) {
-#pragma unroll
-  for (int i = 0; i < NPT; i += 4) {
-    const float4 w = __ldg(reinterpret_cast<const float4 *>(src + i));
-    v[i] = w.x; v[i + 1] = w.y; v[i + 2] = w.z; v[i + 3] = w.w;
-  }
+// Four consecutive values (a 16-byte-aligned group of states) as fp32.
+__device__ __forceinline__ void ldg4(const float *src, float *v) {
+  const float4 w = __ldg(reinterpret_cast<const float4 *>(src));
+  v[0] = w.x; v[1] = w.y; v[2] = w.z; v[3] = w.w;
 }
-template <int NPT>
-__device__ __forceinline__ void ldg_vec(const __nv_bfloat16 *src, float (&v)[NPT]) {
-  if constexpr (NPT % 8 == 0) {
-#pragma unroll
-    for (int i = 0; i < NPT; i += 8) {
-      const uint4 w = __ldg(reinterpret_cast<const uint4 *>(src + i));
-      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {  // a bf16 is the upper half of the equal fp32
-        v[i + 2 * k] = __uint_as_float(ws[k] << 16);
-        v[i + 2 * k + 1] = __uint_as_float(ws[k] & 0xffff0000u);
-      }
-    }
-  } else {
-    const uint2 w = __ldg(reinterpret_cast<const uint2 *>(src));
-    v[0] = __uint_as_float(w.x << 16);
-    v[1] = __uint_as_float(w.x & 0xffff0000u);
-    v[2] = __uint_as_float(w.y << 16);
-    v[3] = __uint_as_float(w.y & 0xffff0000u);
-  }
+__device__ __forceinline__ void ldg4(const __nv_bfloat16 *src, float *v) {
+  const uint2 w = __ldg(reinterpret_cast<const uint2 *>(src));
+  v[0] = __uint_as_float(w.x << 16);  // a bf16 is the upper half of the equal fp32
+  v[1] = __uint_as_float(w.x & 0xffff0000u);
+  v[2] = __uint_as_float(w.y << 16);
+  v[3] = __uint_as_float(w.y & 0xffff0000u);
 }
 
+// TPC threads share a channel; thread q owns the 4-state groups q, q + TPC,
+// q + 2 TPC, ... (NPT states), so each of its 16-byte state accesses, taken
+// over the warp, covers whole 32-byte sectors.
 template <typename InT, typename OutT, int NPT, int TPC, int ITEMS>
-__global__ void __launch_bounds__(256) step_kernel(const StepParams p) {
+__global__ void __launch_bounds__(256, SSM_STEP_MINB) step_kernel(const StepParams p) {
   // ITEMS work items per thread, a grid apart: every item's state reads are
-  // issued before any of them is used, so each thread keeps ITEMS x NPT x 4
-  // bytes of HBM reads in flight
+  // issued before any of them is used
+  constexpr int G = NPT / 4;  // state groups per thread
   const long long total = (long long)gridDim.x * blockDim.x;
   const long long g0 = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const long long nch = (long long)p.Bsz * p.D;
   constexpr int N = NPT * TPC;
   const int q = (int)(g0 % TPC);  // the same for every item (total is a multiple of TPC)
-  float4 s4[ITEMS][NPT / 4];
+  float4 s4[ITEMS][G];
 #pragma unroll
   for (int it = 0; it < ITEMS; ++it) {
     const long long chn = (g0 + it * total) / TPC;
     if (chn < nch) {
-      const float4 *sp = reinterpret_cast<const float4 *>(p.state + (size_t)chn * N + q * NPT);
+      const float4 *sp = reinterpret_cast<const float4 *>(p.state + (size_t)chn * N);
 #pragma unroll
-      for (int i = 0; i < NPT / 4; ++i) s4[it][i] = __ldcs(sp + i);
+      for (int i = 0; i < G; ++i) s4[it][i] = __ldcs(sp + i * TPC + q);
     }
   }
 #pragma unroll
@@ -83,9 +71,13 @@ __global__ void __launch_bounds__(256) step_kernel(const StepParams p) {
     if (active) {
       const int b = (int)(chn / p.D), d = (int)(chn % p.D);
       float Av[NPT], Bv[NPT], Cv[NPT];
-      ldg_vec<NPT>(p.A + (size_t)d * N + q * NPT, Av);
-      ldg_vec<NPT>(reinterpret_cast<const InT *>(p.B) + (size_t)b * N + q * NPT, Bv);
-      ldg_vec<NPT>(reinterpret_cast<const InT *>(p.C) + (size_t)b * N + q * NPT, Cv);
+#pragma unroll
+      for (int i = 0; i < G; ++i) {
+        const int n0 = 4 * (i * TPC + q);
+        ldg4(p.A + (size_t)d * N + n0, Av + 4 * i);
+        ldg4(reinterpret_cast<const InT *>(p.B) + (size_t)b * N + n0, Bv + 4 * i);
+        ldg4(reinterpret_cast<const InT *>(p.C) + (size_t)b * N + n0, Cv + 4 * i);
+      }
       xv = ld1<InT>(p.x, (size_t)chn);
       const float v = ld1<InT>(p.dt, (size_t)chn) + (p.has_bias ? __ldg(p.bias + d) : 0.f);
       if (p.has_z) zv = ld1<InT>(p.z, (size_t)chn);
@@ -94,7 +86,7 @@ __global__ void __launch_bounds__(256) step_kernel(const StepParams p) {
       const float dtx = dlt * xv;
       float h[NPT];
 #pragma unroll
-      for (int i = 0; i < NPT / 4; ++i) {
+      for (int i = 0; i < G; ++i) {
         h[4 * i] = s4[it][i].x; h[4 * i + 1] = s4[it][i].y;
         h[4 * i + 2] = s4[it][i].z; h[4 * i + 3] = s4[it][i].w;
       }
@@ -104,10 +96,10 @@ __global__ void __launch_bounds__(256) step_kernel(const StepParams p) {
         h[n] = fmaf(a, h[n], dtx * Bv[n]);
         acc = fmaf(Cv[n], h[n], acc);
       }
-      float4 *sp = reinterpret_cast<float4 *>(p.state + (size_t)chn * N + q * NPT);
+      float4 *sp = reinterpret_cast<float4 *>(p.state + (size_t)chn * N);
 #pragma unroll
-      for (int i = 0; i < NPT / 4; ++i)
-        __stcs(sp + i, make_float4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]));
+      for (int i = 0; i < G; ++i)
+        __stcs(sp + i * TPC + q, make_float4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]));
     }
 #pragma unroll
     for (int m = TPC / 2; m >= 1; m >>= 1) acc += __shfl_xor_sync(FULL_MASK, acc, m);
