@@ -85,18 +85,22 @@ FWD_KERNEL_SOURCES = ("device_common.cuh", "scan_params.h", "scan_fwd_kernel.cuh
                       "scan_fwd_dispatch.cu")
 
 
-def source_hash():
+STEP_KERNEL_SOURCES = ("device_common.cuh", "scan_params.h", "scan_step.cu")
+
+
+def source_hash(sources=FWD_KERNEL_SOURCES):
     h = hashlib.sha256()
-    for name in FWD_KERNEL_SOURCES:
+    for name in sources:
         with open(os.path.join(ROOT, "selective_state_space_31_b200", "csrc", name), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload):
-    """dram bytes per launch of the forward kernel from the committed ncu
-    summary, or None when it was taken on other source code."""
-    path = os.path.join(ROOT, "profiles", f"fwd_kernel_{workload}.md")
+def profiled_traffic(workload, kernel="fwd_kernel", sources=FWD_KERNEL_SOURCES):
+    """dram bytes per launch of a kernel from its committed ncu summary
+    (profiles/<kernel>_<workload>.md), or None when the summary was taken on
+    other source code."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
     if not os.path.exists(path):
         return None
     kv = {}
@@ -104,7 +108,7 @@ def profiled_traffic(workload):
         if ":" in line and line.strip().startswith("- "):
             k, v = line.strip()[2:].split(":", 1)
             kv[k.strip()] = v.strip().strip("`")
-    if kv.get("source_sha256") != source_hash():
+    if kv.get("source_sha256") != source_hash(sources):
         return None
     try:
         return int(float(kv["dram_bytes_per_launch"]))
@@ -531,7 +535,9 @@ def run_decode(args, rank, world, device):
                    "l2": "3 independent 84 MB states take turns (252 MB > 126 MB L2)",
                    "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": gbs / hbm_peak, "traffic": None, "algorithmic_bytes": byt},
+                     "frac": gbs / hbm_peak,
+                     "traffic": profiled_traffic("decode", "step_kernel", STEP_KERNEL_SOURCES),
+                     "algorithmic_bytes": byt},
         "gpu_launches": steps,
         "clocks": sampler.summary(),
         "e2e": {"value": replica_throughput(upd, world, e_ms), "unit": "state-updates/s",
