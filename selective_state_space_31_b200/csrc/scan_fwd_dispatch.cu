@@ -69,8 +69,8 @@ int parts_per_row(int64_t R, int64_t P, int64_t S) {
 // `rows` CTAs can be busy: grid P <= min(rows, CTAs resident on the device),
 // taken as a multiple of the SM count when that scores better (every SM then
 // gets the same work).  Score = busy scan warps per SM (saturating at 12) x
-// balance of CTAs over SMs x the measured weights above.  Ties: once an SM
-// holds 10 scan warps, fewer warps per CTA; below that, more.
+// balance of CTAs over SMs x the measured weights above.  Ties go to fewer
+// warps per CTA (more, smaller CTAs measured faster at equal warps per SM).
 cudaError_t choose_fwd_shape(int in_dtype, int out_dtype, int64_t batch, int64_t seqlen,
                              int64_t dim, int ns, int sms, const FwdOverrides &o,
                              FwdShape *out) {
@@ -102,8 +102,7 @@ cudaError_t choose_fwd_shape(int in_dtype, int out_dtype, int64_t batch, int64_t
           const int64_t per_sm = (g + sms - 1) / sms;  // CTAs on the busiest SM
           const double busy = (double)g * warps / sms;
           const double balance = (double)g / (double)(per_sm * sms);
-          const double tie = busy >= 10.0 ? -1e-3 * warps : 1e-3 * warps;
-          return std::min(busy, 12.0) / 12.0 * balance * w + tie;
+          return std::min(busy, 12.0) / 12.0 * balance * w - 1e-3 * warps;
         };
         int64_t grid = score_of(balanced) >= score_of(cap) ? balanced : cap;
         if (o.grid > 0) grid = std::min<int64_t>(o.grid, (int64_t)occ * sms);

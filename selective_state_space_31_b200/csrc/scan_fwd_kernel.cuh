@@ -62,7 +62,11 @@ struct FwdCfg {
   static constexpr int SLOT = 3 * XTILE + 2 * BCTILE;
   // ring depth: ~128 tokens of prefetch, within ~64 KB, at least 3 slots
   static constexpr int RAW = clamp_int(65536 / SLOT, 3, 128 / TT > 3 ? 128 / TT : 3);
-  static constexpr int PLANE = align_up(TT * DTW * 8, 128);  // (Delta, Delta*x) per warp
+  // (Delta, Delta*x) per warp, channel-major: row c holds tokens 0..TT-1 of
+  // channel c, rows TTP float2 apart (TTP - TT spreads the rows over the
+  // shared-memory banks; TTP even keeps token pairs 16-byte aligned)
+  static constexpr int TTP = TT + (LPC > 2 ? LPC : 2);
+  static constexpr int PLANE = align_up(TTP * DTW * 8, 128);
   static constexpr int OFF_PLANE = RAW * SLOT;
   static constexpr int OFF_BAR = OFF_PLANE + WARPS * PLANE;
   static constexpr int SMEM = OFF_BAR + 2 * RAW * 8;
@@ -299,8 +303,8 @@ __global__ void __launch_bounds__((WARPS + 1) * 32)
           if (ta >= nvalid) v.x = 0.f;  // past the end: identity update
           if (tb >= nvalid) v.y = 0.f;
           const float2 dx = fmul2(v, xv);
-          plane[ta * DTW + c_loc] = make_float2(v.x, dx.x);
-          plane[tb * DTW + c_loc] = make_float2(v.y, dx.y);
+          plane[c_loc * Cfg::TTP + ta] = make_float2(v.x, dx.x);
+          plane[c_loc * Cfg::TTP + tb] = make_float2(v.y, dx.y);
           float2 g = make_float2(1.f, 1.f);
           if (p.has_z) g = silu_f2(make_float2(to_f32(zs[ta * DT + ch]), to_f32(zs[tb * DT + ch])));
           const float2 gd = fmul2(fmul2(make_float2(dsk, dsk), xv), g);
@@ -315,7 +319,7 @@ __global__ void __launch_bounds__((WARPS + 1) * 32)
           float v = to_f32(ds[ta * DT + ch]) + bias;
           if (p.softplus) v = softplus_f(v);
           if (ta >= nvalid) v = 0.f;
-          plane[ta * DTW + c_loc] = make_float2(v, v * xv);
+          plane[c_loc * Cfg::TTP + ta] = make_float2(v, v * xv);
           const float g = p.has_z ? silu_f(to_f32(zs[ta * DT + ch])) : 1.f;
           g1[j] = g;
           g2[j] = dsk * xv * g;
@@ -325,12 +329,16 @@ __global__ void __launch_bounds__((WARPS + 1) * 32)
 
       // -- the scan over TT tokens of this lane's channel --
       OutT *yrow = ybase + ((size_t)b * p.L + t0) * p.D + d;
+      const float2 *prow = plane + c_loc * Cfg::TTP;
+      float4 dpair;  // (Delta, Delta*x) of an even token and the next, one 16-byte load
 #pragma unroll
       for (int tt = 0; tt < TT; tt += LPC) {
         float yp[LPC];
 #pragma unroll
         for (int j = 0; j < LPC; ++j) {
-          const float2 dd = plane[(tt + j) * DTW + c_loc];
+          const int t = tt + j;
+          if ((t & 1) == 0) dpair = *reinterpret_cast<const float4 *>(prow + t);
+          const float2 dd = (t & 1) ? make_float2(dpair.z, dpair.w) : make_float2(dpair.x, dpair.y);
           float bv[NPL], cv[NPL];
           load_bc<NPL>(Bs + (tt + j) * NS + q * NPL, bv);
           load_bc<NPL>(Cs + (tt + j) * NS + q * NPL, cv);
