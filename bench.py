@@ -54,6 +54,8 @@ def parse_args():
     ap.add_argument("--warps", type=int, default=0)
     ap.add_argument("--grid", type=int, default=0)
     ap.add_argument("--tile-t", type=int, default=0)
+    ap.add_argument("--zoh", action="store_true",
+                    help="zero-order-hold input matrix (exp(Delta A) - 1)/A * B instead of Delta * B")
     return ap.parse_args()
 
 
@@ -229,7 +231,7 @@ def oracle_sample_rate(inp, budget_cpu_s, threads=None):
     t0 = time.perf_counter()
     oracle.fwd_rows(inp.x, inp.delta, inp.A, inp.B, inp.C, [(0, 0)], D=inp.Dskip, z=inp.z,
                     delta_bias=inp.delta_bias, h0=inp.h0, delta_softplus=inp.delta_softplus,
-                    oracle=orc)
+                    oracle=orc, zoh=inp.zoh)
     per_row = max(time.perf_counter() - t0, 1e-6)
     n_rows = int(min(inp.Bsz * inp.D, max(threads, budget_cpu_s / per_row)))
     rows = [(r // inp.D, r % inp.D) for r in range(n_rows)]
@@ -239,7 +241,7 @@ def oracle_sample_rate(inp, budget_cpu_s, threads=None):
         if ch:
             oracle.fwd_rows(inp.x, inp.delta, inp.A, inp.B, inp.C, ch, D=inp.Dskip, z=inp.z,
                             delta_bias=inp.delta_bias, h0=inp.h0,
-                            delta_softplus=inp.delta_softplus, oracle=orc)
+                            delta_softplus=inp.delta_softplus, oracle=orc, zoh=inp.zoh)
 
     t0 = time.perf_counter()
     with cf.ThreadPoolExecutor(max_workers=threads) as ex:
@@ -267,6 +269,7 @@ def run_ours(args, rank, world, device):
     inp = make()
     inp_b = make(seed={"tiny_fp32": 0, "mamba130m_layer": 1, "mamba1p4b_layer": 2,
                        "long_seq": 3}[args.workload] + 1000 + rank)
+    inp.zoh = inp_b.zoh = bool(args.zoh)
     tdt = {"f32": torch.float32, "bf16": torch.bfloat16}
 
     def up(a, dt):
@@ -281,7 +284,7 @@ def run_ours(args, rank, world, device):
 
     sets = [upload(inp), upload(inp_b)]
     flags = bnd.flags_for(z=inp.z, D=inp.Dskip, delta_bias=inp.delta_bias, h0=inp.h0,
-                          delta_softplus=inp.delta_softplus, want_h_last=True)
+                          delta_softplus=inp.delta_softplus, want_h_last=True, zoh=inp.zoh)
     plan = bnd.Plan(inp.Bsz, inp.L, inp.D, inp.N, tdt[inp.in_dtype], tdt[inp.out_dtype], flags,
                     device)
     if args.lpc or args.warps or args.grid or args.tile_t:
@@ -405,6 +408,7 @@ def run_ours(args, rank, world, device):
         "config": {"workload": inp.name, "batch": inp.Bsz, "seqlen": inp.L, "dim": inp.D,
                    "dstate": inp.N, "in_dtype": inp.in_dtype, "out_dtype": inp.out_dtype,
                    "state_dtype": "f32", "gate": inp.z is not None, "h0": inp.h0 is not None,
+                   "discretisation": "zoh" if inp.zoh else "delta_B",
                    "l2": "two input sets alternate between steps (2x inputs > 126 MB L2)",
                    "parallelism": f"replicas x{world}",
                    "launch": {k: info[k] for k in ("lanes_per_chan", "warps_per_cta",
@@ -605,6 +609,7 @@ def run_reference(args):
                 "e2e": {"value": value, "unit": "state-updates/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
     inp = synth.FWD_WORKLOADS[args.workload]()
+    inp.zoh = bool(args.zoh)
     threads = os.cpu_count() or 1
     total_budget = args.cpu_budget_s * threads   # CPU-seconds for warmup + timed steps
     per_step = total_budget / max(1, args.steps + args.warmup)

@@ -24,6 +24,7 @@
  * Computed per channel (b, d), for t = 0 .. L-1, per state n < N:
  *   Delta   = softplus(delta[b,t,d] + delta_bias[d])   (softplus if flagged)
  *   h[n]    = exp(Delta * A[d,n]) * h[n] + (Delta * B[b,t,n]) * x[b,t,d]
+ *             (SSM_ZOH: (exp(Delta*A[d,n]) - 1) / A[d,n] * B[b,t,n] * x[b,t,d])
  *   y[b,t,d]= (sum_n C[b,t,n] * h[n] + D[d] * x[b,t,d]) * silu(z[b,t,d])
  * with h starting at h0 (or 0) and h_last = h after the last token.  The
  * skip and gate terms are present only when flagged; silu(z) = z*sigmoid(z).
@@ -93,7 +94,10 @@ enum {
   SSM_HAS_DELTA_BIAS = 8,   /* add delta_bias[d] before softplus */
   SSM_HAS_H0 = 16,          /* start from h0 (else from 0) */
   SSM_WANT_HLAST = 32,      /* write h_last */
-  SSM_A_DIRECT = 64         /* elementwise variant: N = 1, A/B/C per (b,t,d), no delta/D/z */
+  SSM_A_DIRECT = 64,        /* elementwise variant: N = 1, A/B/C per (b,t,d), no delta/D/z */
+  SSM_ZOH = 128             /* zero-order-hold input matrix: Bbar = (exp(Delta*A) - 1) / A * B
+                               ("Vi du Python" of the first page) instead of Delta * B;
+                               Bbar -> Delta * B where A = 0.  Not with SSM_A_DIRECT. */
 };
 
 typedef struct {

@@ -169,7 +169,7 @@ def get() -> Oracle:
 
 
 def fwd_rows(x, delta, A, B, C, rows, D=None, z=None, delta_bias=None, h0=None,
-             delta_softplus=True, oracle: Oracle | None = None):
+             delta_softplus=True, oracle: Oracle | None = None, zoh=False):
     """Run the oracle on selected channels only.  ``rows`` is a list of (b, d)
     pairs; every array keeps its full layout and only the needed slices are
     copied.  Returns (y[len(rows), L], h_last[len(rows), N])."""
@@ -182,7 +182,7 @@ def fwd_rows(x, delta, A, B, C, rows, D=None, z=None, delta_bias=None, h0=None,
                          None if D is None else np.asarray(D)[d:d + 1], sl(z),
                          None if delta_bias is None else np.asarray(delta_bias)[d:d + 1],
                          None if h0 is None else np.asarray(h0)[b:b + 1, d:d + 1],
-                         delta_softplus=delta_softplus)
+                         delta_softplus=delta_softplus, zoh=zoh)
         ys.append(yb[0, :, 0])
         hs.append(hb[0, 0])
     return np.stack(ys), np.stack(hs)

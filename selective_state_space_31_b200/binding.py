@@ -22,6 +22,7 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_MISALIGNED, ERR_CUDA, ERR_TIMEOUT, ERR
 F32, BF16 = 0, 1
 # flags
 HAS_Z, HAS_D, DELTA_SOFTPLUS, HAS_DELTA_BIAS, HAS_H0, WANT_HLAST, A_DIRECT = 1, 2, 4, 8, 16, 32, 64
+ZOH = 128  # zero-order-hold input matrix: Bbar = (exp(Delta A) - 1) / A * B
 
 _TORCH_TO_SSM = {torch.float32: F32, torch.bfloat16: BF16}
 
@@ -230,11 +231,12 @@ class Plan:
 
 
 def flags_for(*, z=None, D=None, delta_bias=None, h0=None, delta_softplus=True,
-              want_h_last=True) -> int:
+              want_h_last=True, zoh=False) -> int:
     return ((HAS_Z if z is not None else 0) | (HAS_D if D is not None else 0)
             | (DELTA_SOFTPLUS if delta_softplus else 0)
             | (HAS_DELTA_BIAS if delta_bias is not None else 0)
-            | (HAS_H0 if h0 is not None else 0) | (WANT_HLAST if want_h_last else 0))
+            | (HAS_H0 if h0 is not None else 0) | (WANT_HLAST if want_h_last else 0)
+            | (ZOH if zoh else 0))
 
 
 _plans: dict = {}
@@ -251,14 +253,15 @@ def _plan_for(key, make):
 
 
 def fwd(x, delta, A, B, C, D=None, z=None, delta_bias=None, h0=None, delta_softplus=True,
-        want_h_last=True, out_dtype=None):
+        want_h_last=True, out_dtype=None, zoh=False):
     """Selective-scan forward.  x, delta, z: (B, L, D); B, C: (B, L, N);
     A: (D, N) fp32; D, delta_bias: (D,) fp32; h0: (B, D, N) fp32.
+    zoh selects the zero-order-hold input matrix (exp(Delta A) - 1) / A * B.
     Returns (y, h_last) (h_last is None when not requested)."""
     Bz, L, Dm = x.shape
     N = A.shape[1]
     flags = flags_for(z=z, D=D, delta_bias=delta_bias, h0=h0, delta_softplus=delta_softplus,
-                      want_h_last=want_h_last)
+                      want_h_last=want_h_last, zoh=zoh)
     out_dtype = out_dtype or x.dtype
     key = ("fwd", Bz, L, Dm, N, x.dtype, out_dtype, flags, x.device)
     plan = _plan_for(key, lambda: Plan(Bz, L, Dm, N, x.dtype, out_dtype, flags, x.device))
@@ -266,11 +269,11 @@ def fwd(x, delta, A, B, C, D=None, z=None, delta_bias=None, h0=None, delta_softp
 
 
 def step(state, x, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True,
-         out_dtype=None):
+         out_dtype=None, zoh=False):
     """One decode step: updates ``state`` (B, D, N) fp32 in place, returns y (B, D)."""
     Bz, Dm, N = state.shape
     flags = flags_for(z=z, D=D, delta_bias=delta_bias, delta_softplus=delta_softplus,
-                      want_h_last=False)
+                      want_h_last=False, zoh=zoh)
     out_dtype = out_dtype or x.dtype
     key = ("step", Bz, Dm, N, x.dtype, out_dtype, flags, x.device)
     plan = _plan_for(key, lambda: Plan(Bz, 1, Dm, N, x.dtype, out_dtype, flags, x.device))

@@ -105,6 +105,38 @@ __device__ __forceinline__ float2 silu_f2(float2 z) {
   return fmul2(z, make_float2(rcp_approx(den.x), rcp_approx(den.y)));
 }
 
+// Zero-order hold ("Vi du Python" of the first page): Bbar / B = (e^u - 1) / A
+// with u = Delta * A, given e = e^u from ex2.approx.  For |u| < 1/4 it is
+// Delta * (expm1(u) / u), the Taylor series 1 + u/2 + u^2/6 + ... + u^6/5040
+// (the next term is below 2e-9 relative), so a small or zero A needs neither
+// a division nor the cancellation of e - 1; elsewhere (e - 1) * (1/A), where
+// |e - 1| > 0.22 keeps ex2.approx's 2^-22 relative error below 1.2e-6.
+__device__ __forceinline__ float zoh_coef(float u, float e, float dlt, float invA) {
+  float p = 1.f / 5040.f;
+  p = fmaf(p, u, 1.f / 720.f);
+  p = fmaf(p, u, 1.f / 120.f);
+  p = fmaf(p, u, 1.f / 24.f);
+  p = fmaf(p, u, 1.f / 6.f);
+  p = fmaf(p, u, 0.5f);
+  p = fmaf(p, u, 1.f);
+  return fabsf(u) < 0.25f ? dlt * p : (e - 1.f) * invA;
+}
+// The same for two states at once (packed polynomial).
+__device__ __forceinline__ float2 zoh_coef2(float2 u, float2 e, float2 dlt, float2 invA) {
+  float2 p = make_float2(1.f / 5040.f, 1.f / 5040.f);
+  p = ffma2(p, u, make_float2(1.f / 720.f, 1.f / 720.f));
+  p = ffma2(p, u, make_float2(1.f / 120.f, 1.f / 120.f));
+  p = ffma2(p, u, make_float2(1.f / 24.f, 1.f / 24.f));
+  p = ffma2(p, u, make_float2(1.f / 6.f, 1.f / 6.f));
+  p = ffma2(p, u, make_float2(0.5f, 0.5f));
+  p = ffma2(p, u, make_float2(1.f, 1.f));
+  const float2 small = fmul2(dlt, p);
+  const float2 large = fmul2(fadd2(e, make_float2(-1.f, -1.f)), invA);
+  return make_float2(fabsf(u.x) < 0.25f ? small.x : large.x,
+                     fabsf(u.y) < 0.25f ? small.y : large.y);
+}
+constexpr float kLn2 = 0.6931471805599453f;
+
 template <typename T> __device__ __forceinline__ float to_f32(T v);
 template <> __device__ __forceinline__ float to_f32<float>(float v) { return v; }
 template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) {

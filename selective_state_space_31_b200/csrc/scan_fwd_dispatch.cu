@@ -72,7 +72,7 @@ int parts_per_row(int64_t R, int64_t P, int64_t S) {
 // balance of CTAs over SMs x the measured weights above.  Ties go to fewer
 // warps per CTA (more, smaller CTAs measured faster at equal warps per SM).
 cudaError_t choose_fwd_shape(int in_dtype, int out_dtype, int64_t batch, int64_t seqlen,
-                             int64_t dim, int ns, int sms, const FwdOverrides &o,
+                             int64_t dim, int ns, bool zoh, int sms, const FwdOverrides &o,
                              FwdShape *out) {
   const int ei = in_dtype == 1 ? 2 : 4, eo = out_dtype == 1 ? 2 : 4;
   bool found = false;
@@ -83,10 +83,10 @@ cudaError_t choose_fwd_shape(int in_dtype, int out_dtype, int64_t batch, int64_t
     for (int warps : {2, 4, 8}) {
       if (o.warps && warps != o.warps) continue;
       for (int tt : {32, 64, 16}) {
-        if (o.tt && tt != o.tt) continue;
+        if ((o.tt && tt != o.tt) || (zoh && tt == 16)) continue;
         const int DT = warps * 32 / lpc;
         if ((DT * ei) % 16 || (DT * eo) % 16) continue;
-        LaunchShape ls{lpc, warps, tt, kStages, ns, 0, 0};
+        LaunchShape ls{lpc, warps, tt, kStages, ns, 0, 0, zoh};
         int occ = 0;
         size_t smem = 0;
         if (fwd_tma_smem_and_occupancy(in_dtype, out_dtype, ls, &smem, &occ) != cudaSuccess ||

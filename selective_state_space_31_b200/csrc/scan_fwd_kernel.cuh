@@ -163,7 +163,7 @@ struct ItemCursor {
   }
 };
 
-template <typename InT, typename OutT, int NS, int LPC, int WARPS, int TT>
+template <typename InT, typename OutT, int NS, int LPC, int WARPS, int TT, bool ZOH>
 __global__ void __launch_bounds__((WARPS + 1) * 32)
     fwd_kernel(const __grid_constant__ TmaMaps maps, const FwdParams p) {
   using Cfg = FwdCfg<InT, OutT, NS, LPC, WARPS, TT>;
@@ -232,9 +232,9 @@ __global__ void __launch_bounds__((WARPS + 1) * 32)
     const int q = lane % LPC;           // state group of this lane
     const int ch = warp * DTW + c_loc;  // channel within the row tile
     float2 *plane = reinterpret_cast<float2 *>(smem + Cfg::OFF_PLANE + warp * Cfg::PLANE);
-    float h[NPL], A2[NPL];
+    float h[NPL], A2[NPL], invA[NPL];  // invA: 1/A (0 where A = 0), zero-order hold only
 #pragma unroll
-    for (int i = 0; i < NPL; ++i) { h[i] = 0.f; A2[i] = 0.f; }
+    for (int i = 0; i < NPL; ++i) { h[i] = 0.f; A2[i] = 0.f; invA[i] = 0.f; }
     float bias = 0.f, dsk = 0.f;
     OutT *const ybase = reinterpret_cast<OutT *>(p.y);
     ItemCursor cur;
@@ -247,8 +247,11 @@ __global__ void __launch_bounds__((WARPS + 1) * 32)
       const bool run_start = st == cur.part * cur.PL;
       if (run_start) {  // per-item parameters and starting state of this lane
 #pragma unroll
-        for (int i = 0; i < NPL; ++i)
-          A2[i] = valid_ch ? __ldg(p.A + (size_t)d * NS + q * NPL + i) * kLog2e : 0.f;
+        for (int i = 0; i < NPL; ++i) {
+          const float a = valid_ch ? __ldg(p.A + (size_t)d * NS + q * NPL + i) : 0.f;
+          A2[i] = a * kLog2e;
+          if constexpr (ZOH) invA[i] = a != 0.f ? 1.f / a : 0.f;
+        }
         bias = (p.has_bias && valid_ch) ? __ldg(p.bias + d) : 0.f;
         dsk = (p.has_D && valid_ch) ? __ldg(p.Dv + d) : 0.f;
         if (st == 0) {
@@ -303,8 +306,9 @@ __global__ void __launch_bounds__((WARPS + 1) * 32)
           if (ta >= nvalid) v.x = 0.f;  // past the end: identity update
           if (tb >= nvalid) v.y = 0.f;
           const float2 dx = fmul2(v, xv);
-          plane[c_loc * Cfg::TTP + ta] = make_float2(v.x, dx.x);
-          plane[c_loc * Cfg::TTP + tb] = make_float2(v.y, dx.y);
+          // zero-order hold keeps x itself: its input term is not a multiple of Delta
+          plane[c_loc * Cfg::TTP + ta] = make_float2(v.x, ZOH ? xv.x : dx.x);
+          plane[c_loc * Cfg::TTP + tb] = make_float2(v.y, ZOH ? xv.y : dx.y);
           float2 g = make_float2(1.f, 1.f);
           if (p.has_z) g = silu_f2(make_float2(to_f32(zs[ta * DT + ch]), to_f32(zs[tb * DT + ch])));
           const float2 gd = fmul2(fmul2(make_float2(dsk, dsk), xv), g);
@@ -319,7 +323,7 @@ __global__ void __launch_bounds__((WARPS + 1) * 32)
           float v = to_f32(ds[ta * DT + ch]) + bias;
           if (p.softplus) v = softplus_f(v);
           if (ta >= nvalid) v = 0.f;
-          plane[c_loc * Cfg::TTP + ta] = make_float2(v, v * xv);
+          plane[c_loc * Cfg::TTP + ta] = make_float2(v, ZOH ? xv : v * xv);
           const float g = p.has_z ? silu_f(to_f32(zs[ta * DT + ch])) : 1.f;
           g1[j] = g;
           g2[j] = dsk * xv * g;
@@ -349,7 +353,11 @@ __global__ void __launch_bounds__((WARPS + 1) * 32)
             for (int i = 0; i < NPL; i += 2) {
               const float2 arg = fmul2(dA, make_float2(A2[i], A2[i + 1]));
               const float2 a = make_float2(ex2_approx(arg.x), ex2_approx(arg.y));
-              const float2 bx = fmul2(dX, make_float2(bv[i], bv[i + 1]));
+              float2 bx = fmul2(dX, make_float2(bv[i], bv[i + 1]));
+              if constexpr (ZOH)  // dX holds x: Bbar x = ((e^u - 1) / A) * (B x)
+                bx = fmul2(zoh_coef2(fmul2(arg, make_float2(kLn2, kLn2)), a, dA,
+                                     make_float2(invA[i], invA[i + 1])),
+                           bx);
               const float2 hn = ffma2(a, make_float2(h[i], h[i + 1]), bx);
               h[i] = hn.x;
               h[i + 1] = hn.y;
@@ -357,8 +365,11 @@ __global__ void __launch_bounds__((WARPS + 1) * 32)
             }
             yp[j] = acc.x + acc.y;
           } else {
-            const float a = ex2_approx(dd.x * A2[0]);
-            h[0] = fmaf(a, h[0], dd.y * bv[0]);
+            const float arg = dd.x * A2[0];
+            const float a = ex2_approx(arg);
+            float bx = dd.y * bv[0];
+            if constexpr (ZOH) bx *= zoh_coef(arg * kLn2, a, dd.x, invA[0]);
+            h[0] = fmaf(a, h[0], bx);
             yp[j] = cv[0] * h[0];
           }
         }
@@ -408,11 +419,11 @@ __global__ void __launch_bounds__((WARPS + 1) * 32)
 // host-side variant table (one translation unit per dtype pair)
 // ---------------------------------------------------------------------------
 
-template <typename InT, typename OutT, int NS, int LPC, int WARPS, int TT>
+template <typename InT, typename OutT, int NS, int LPC, int WARPS, int TT, bool ZOH>
 static cudaError_t run_variant(const LaunchShape *ls, const TmaMaps *maps, const FwdParams *p,
                                cudaStream_t stream, size_t *smem_out, int *occ_out) {
   using Cfg = FwdCfg<InT, OutT, NS, LPC, WARPS, TT>;
-  auto kern = fwd_kernel<InT, OutT, NS, LPC, WARPS, TT>;
+  auto kern = fwd_kernel<InT, OutT, NS, LPC, WARPS, TT, ZOH>;
   if (Cfg::SMEM > 227 * 1024) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
   if (e != cudaSuccess) {
@@ -429,7 +440,7 @@ static cudaError_t run_variant(const LaunchShape *ls, const TmaMaps *maps, const
   return cudaGetLastError();
 }
 
-template <typename InT, typename OutT, int NS, int LPC, int WARPS>
+template <typename InT, typename OutT, int NS, int LPC, int WARPS, bool ZOH>
 static cudaError_t by_tt(const LaunchShape *ls, const TmaMaps *maps, const FwdParams *p,
                          cudaStream_t st, size_t *sm, int *oc) {
   // a row tile's x / delta / z rows must be whole 16-byte TMA units
@@ -437,38 +448,53 @@ static cudaError_t by_tt(const LaunchShape *ls, const TmaMaps *maps, const FwdPa
     return cudaErrorInvalidValue;
   } else {
     switch (ls->tt) {
-      case 16: return run_variant<InT, OutT, NS, LPC, WARPS, 16>(ls, maps, p, st, sm, oc);
-      case 32: return run_variant<InT, OutT, NS, LPC, WARPS, 32>(ls, maps, p, st, sm, oc);
-      case 64: return run_variant<InT, OutT, NS, LPC, WARPS, 64>(ls, maps, p, st, sm, oc);
+      case 16:
+        if constexpr (!ZOH) return run_variant<InT, OutT, NS, LPC, WARPS, 16, ZOH>(ls, maps, p, st, sm, oc);
+        return cudaErrorInvalidValue;
+      case 32: return run_variant<InT, OutT, NS, LPC, WARPS, 32, ZOH>(ls, maps, p, st, sm, oc);
+      case 64: return run_variant<InT, OutT, NS, LPC, WARPS, 64, ZOH>(ls, maps, p, st, sm, oc);
       default: return cudaErrorInvalidValue;
     }
   }
 }
 
-template <typename InT, typename OutT, int NS, int LPC>
+template <typename InT, typename OutT, int NS, int LPC, bool ZOH>
 static cudaError_t by_warps(const LaunchShape *ls, const TmaMaps *maps, const FwdParams *p,
                             cudaStream_t st, size_t *sm, int *oc) {
   switch (ls->warps) {
-    case 2: return by_tt<InT, OutT, NS, LPC, 2>(ls, maps, p, st, sm, oc);
-    case 4: return by_tt<InT, OutT, NS, LPC, 4>(ls, maps, p, st, sm, oc);
-    case 8: return by_tt<InT, OutT, NS, LPC, 8>(ls, maps, p, st, sm, oc);
+    case 2: return by_tt<InT, OutT, NS, LPC, 2, ZOH>(ls, maps, p, st, sm, oc);
+    case 4: return by_tt<InT, OutT, NS, LPC, 4, ZOH>(ls, maps, p, st, sm, oc);
+    case 8: return by_tt<InT, OutT, NS, LPC, 8, ZOH>(ls, maps, p, st, sm, oc);
     default: return cudaErrorInvalidValue;
   }
 }
 
-template <typename InT, typename OutT, int NS>
+template <typename InT, typename OutT, int NS, bool ZOH>
 static cudaError_t by_lpc(const LaunchShape *ls, const TmaMaps *maps, const FwdParams *p,
                           cudaStream_t st, size_t *sm, int *oc) {
   switch (ls->lpc) {
-    case 1: return by_warps<InT, OutT, NS, 1>(ls, maps, p, st, sm, oc);
-    case 2: return by_warps<InT, OutT, NS, 2>(ls, maps, p, st, sm, oc);
-    case 4: return by_warps<InT, OutT, NS, 4>(ls, maps, p, st, sm, oc);
+    case 1: return by_warps<InT, OutT, NS, 1, ZOH>(ls, maps, p, st, sm, oc);
+    case 2: return by_warps<InT, OutT, NS, 2, ZOH>(ls, maps, p, st, sm, oc);
+    case 4: return by_warps<InT, OutT, NS, 4, ZOH>(ls, maps, p, st, sm, oc);
     case 8:
-      if constexpr (NS >= 8) return by_warps<InT, OutT, NS, 8>(ls, maps, p, st, sm, oc);
+      if constexpr (NS >= 8) return by_warps<InT, OutT, NS, 8, ZOH>(ls, maps, p, st, sm, oc);
       return cudaErrorInvalidValue;
     case 16:
-      if constexpr (NS >= 16) return by_warps<InT, OutT, NS, 16>(ls, maps, p, st, sm, oc);
+      if constexpr (NS >= 16) return by_warps<InT, OutT, NS, 16, ZOH>(ls, maps, p, st, sm, oc);
       return cudaErrorInvalidValue;
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <typename InT, typename OutT, bool ZOH>
+static cudaError_t by_ns_zoh(const LaunchShape *ls, const TmaMaps *maps, const FwdParams *p,
+                             cudaStream_t st, size_t *sm, int *oc) {
+  switch (ls->ns) {
+    case 4:
+      if constexpr (sizeof(InT) == 4) return by_lpc<InT, OutT, 4, ZOH>(ls, maps, p, st, sm, oc);
+      return cudaErrorInvalidValue;
+    case 8: return by_lpc<InT, OutT, 8, ZOH>(ls, maps, p, st, sm, oc);
+    case 16: return by_lpc<InT, OutT, 16, ZOH>(ls, maps, p, st, sm, oc);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -477,14 +503,9 @@ template <typename InT, typename OutT>
 static cudaError_t by_ns(const LaunchShape *ls, const TmaMaps *maps, const FwdParams *p,
                          cudaStream_t st, size_t *sm, int *oc) {
   if (ls->stages != kStages) return cudaErrorInvalidValue;
-  switch (ls->ns) {
-    case 4:
-      if constexpr (sizeof(InT) == 4) return by_lpc<InT, OutT, 4>(ls, maps, p, st, sm, oc);
-      return cudaErrorInvalidValue;
-    case 8: return by_lpc<InT, OutT, 8>(ls, maps, p, st, sm, oc);
-    case 16: return by_lpc<InT, OutT, 16>(ls, maps, p, st, sm, oc);
-    default: return cudaErrorInvalidValue;
-  }
+  if (p && p->zoh != ls->zoh) return cudaErrorInvalidValue;
+  return ls->zoh ? by_ns_zoh<InT, OutT, true>(ls, maps, p, st, sm, oc)
+                 : by_ns_zoh<InT, OutT, false>(ls, maps, p, st, sm, oc);
 }
 
 // per-dtype entry points (defined in scan_fwd_<dtypes>.cu)

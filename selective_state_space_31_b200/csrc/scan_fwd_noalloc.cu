@@ -103,7 +103,7 @@ extern "C" SSM_API ssm_status ssm_scan_fwd_noalloc(
       (d.out_dtype != SSM_F32 && d.out_dtype != SSM_BF16))
     return SSM_ERR_INVALID_ARG;
   constexpr uint32_t known = SSM_HAS_Z | SSM_HAS_D | SSM_DELTA_SOFTPLUS | SSM_HAS_DELTA_BIAS |
-                             SSM_HAS_H0 | SSM_WANT_HLAST;
+                             SSM_HAS_H0 | SSM_WANT_HLAST | SSM_ZOH;
   if (f & ~known) return SSM_ERR_INVALID_ARG;
   // the fast-path shape rules of the chunked kernel
   const int ns = (int)d.dstate;
@@ -130,7 +130,8 @@ extern "C" SSM_API ssm_status ssm_scan_fwd_noalloc(
   // launch shape: the same choice a plan makes by default
   ssm::FwdShape fs;
   if (ssm::choose_fwd_shape((int)d.in_dtype, (int)d.out_dtype, d.batch, d.seqlen, d.dim, ns,
-                            num_sms, ssm::FwdOverrides{0, 0, 0, 0}, &fs) != cudaSuccess) {
+                            (f & SSM_ZOH) != 0, num_sms, ssm::FwdOverrides{0, 0, 0, 0},
+                            &fs) != cudaSuccess) {
     cudaGetLastError();
     return SSM_ERR_UNSUPPORTED;
   }
@@ -166,6 +167,7 @@ extern "C" SSM_API ssm_status ssm_scan_fwd_noalloc(
   p.has_bias = (f & SSM_HAS_DELTA_BIAS) != 0;
   p.has_h0 = (f & SSM_HAS_H0) != 0;
   p.want_hlast = (f & SSM_WANT_HLAST) != 0;
+  p.zoh = (f & SSM_ZOH) != 0;
   p.A = A; p.Dv = D; p.bias = delta_bias; p.h0 = h0; p.h_last = h_last; p.y = y;
   p.ctl = reinterpret_cast<ssm::Control *>(base);
   p.ws_flags = reinterpret_cast<unsigned long long *>(base + kCtlBytes);

@@ -27,12 +27,14 @@ __global__ void __launch_bounds__(128) fwd_general_kernel(const GenericParams p)
   if (chn >= (long long)p.Bsz * p.D) return;
   const int b = (int)(chn / p.D), d = (int)(chn % p.D);
   const int N = p.N;
-  float h[NMAX], A2[NMAX];
+  float h[NMAX], A2[NMAX], invA[NMAX];
 #pragma unroll
   for (int n = 0; n < NMAX; ++n) {
     const bool on = n < N;
     h[n] = (on && p.has_h0) ? p.h0[((size_t)b * p.D + d) * N + n] : 0.f;
-    A2[n] = on ? p.A[(size_t)d * N + n] * kLog2e : 0.f;
+    const float a = on ? p.A[(size_t)d * N + n] : 0.f;
+    A2[n] = a * kLog2e;
+    invA[n] = a != 0.f ? 1.f / a : 0.f;
   }
   const float Dd = p.has_D ? p.Dv[d] : 0.f;
   const float bias = p.has_bias ? p.bias[d] : 0.f;
@@ -47,8 +49,12 @@ __global__ void __launch_bounds__(128) fwd_general_kernel(const GenericParams p)
 #pragma unroll
     for (int n = 0; n < NMAX; ++n) {
       if (n < N) {
-        const float a = ex2_approx(dlt * A2[n]);
-        h[n] = fmaf(a, h[n], dtx * ldf<InT>(p.B, j + n));
+        const float arg = dlt * A2[n];
+        const float a = ex2_approx(arg);
+        // Bbar x: Delta B x, or (e^{Delta A} - 1) / A * B x under zero-order hold
+        const float bx = p.zoh ? zoh_coef(arg * kLn2, a, dlt, invA[n]) * xv * ldf<InT>(p.B, j + n)
+                               : dtx * ldf<InT>(p.B, j + n);
+        h[n] = fmaf(a, h[n], bx);
         acc = fmaf(ldf<InT>(p.C, j + n), h[n], acc);
       }
     }

@@ -28,6 +28,7 @@ struct FwdParams {
   int PL;       // stages per part (work item) of a row
   int items;    // rows * parts per row
   bool softplus, has_z, has_D, has_bias, has_h0, want_hlast;
+  bool zoh;            // zero-order-hold Bbar (selects the kernel template too)
   const float *A;      // (D, N)
   const float *Dv;     // (D) or null
   const float *bias;   // (D) or null
@@ -49,6 +50,7 @@ struct LaunchShape {
   int lpc, warps, tt, stages, ns;
   int grid;
   size_t smem;
+  bool zoh;  // zero-order-hold variant of the kernel
 };
 
 // Fused forward kernel (scan_fwd_kernel.cuh, instantiated per dtype pair).
@@ -65,6 +67,7 @@ constexpr int kStages = 2;
 struct FwdOverrides {
   int lpc, warps, tt, grid;
 };
+// (the zero-order-hold variants exist for 32- and 64-token stages only)
 // A launch shape of the fused kernel with its work split.
 struct FwdShape {
   LaunchShape ls;  // lpc, warps, tt, stages, ns, grid, smem
@@ -77,12 +80,12 @@ struct FwdShape {
 // Choose the fused kernel's launch shape for a problem (scan_fwd_dispatch.cu).
 // Returns cudaErrorInvalidValue when no variant fits the overrides.
 cudaError_t choose_fwd_shape(int in_dtype, int out_dtype, int64_t batch, int64_t seqlen,
-                             int64_t dim, int ns, int sms, const FwdOverrides &o,
+                             int64_t dim, int ns, bool zoh, int sms, const FwdOverrides &o,
                              FwdShape *out);
 
 struct GenericParams {
   int Bsz, L, D, N;
-  bool softplus, has_z, has_D, has_bias, has_h0, want_hlast;
+  bool softplus, has_z, has_D, has_bias, has_h0, want_hlast, zoh;
   int in_bf16, out_bf16;
   const void *x, *dt, *z, *B, *C;
   const float *A, *Dv, *bias, *h0;
@@ -105,7 +108,7 @@ cudaError_t launch_direct(const DirectParams &p, cudaStream_t stream);
 
 struct StepParams {
   int Bsz, D, N;
-  bool softplus, has_z, has_D, has_bias;
+  bool softplus, has_z, has_D, has_bias, zoh;
   int in_bf16, out_bf16;
   const void *x, *dt, *z, *B, *C;
   const float *A, *Dv, *bias;

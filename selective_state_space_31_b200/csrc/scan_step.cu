@@ -92,8 +92,13 @@ __global__ void __launch_bounds__(256, SSM_STEP_MINB) step_kernel(const StepPara
       }
 #pragma unroll
       for (int n = 0; n < NPT; ++n) {
-        const float a = ex2_approx(dlt * (Av[n] * kLog2e));
-        h[n] = fmaf(a, h[n], dtx * Bv[n]);
+        const float arg = dlt * (Av[n] * kLog2e);
+        const float a = ex2_approx(arg);
+        // Bbar x: Delta B x, or (e^{Delta A} - 1) / A * B x under zero-order hold
+        const float bx = p.zoh ? zoh_coef(arg * kLn2, a, dlt, Av[n] != 0.f ? 1.f / Av[n] : 0.f) *
+                                     xv * Bv[n]
+                               : dtx * Bv[n];
+        h[n] = fmaf(a, h[n], bx);
         acc = fmaf(Cv[n], h[n], acc);
       }
       float4 *sp = reinterpret_cast<float4 *>(p.state + (size_t)chn * N);
@@ -124,8 +129,13 @@ __global__ void __launch_bounds__(128) step_general_kernel(const StepParams p) {
   float acc = 0.f;
   for (int n = 0; n < N; ++n) {
     float *sp = p.state + (size_t)chn * N + n;
-    const float a = ex2_approx(dlt * (p.A[(size_t)d * N + n] * kLog2e));
-    const float hn = fmaf(a, *sp, dtx * ld1<InT>(p.B, (size_t)b * N + n));
+    const float An = p.A[(size_t)d * N + n];
+    const float arg = dlt * (An * kLog2e);
+    const float a = ex2_approx(arg);
+    const float Bn = ld1<InT>(p.B, (size_t)b * N + n);
+    const float bx = p.zoh ? zoh_coef(arg * kLn2, a, dlt, An != 0.f ? 1.f / An : 0.f) * xv * Bn
+                           : dtx * Bn;
+    const float hn = fmaf(a, *sp, bx);
     *sp = hn;
     acc = fmaf(ld1<InT>(p.C, (size_t)b * N + n), hn, acc);
   }

@@ -18,7 +18,7 @@
 namespace {
 
 constexpr uint32_t kKnownFlags = SSM_HAS_Z | SSM_HAS_D | SSM_DELTA_SOFTPLUS | SSM_HAS_DELTA_BIAS |
-                                 SSM_HAS_H0 | SSM_WANT_HLAST | SSM_A_DIRECT;
+                                 SSM_HAS_H0 | SSM_WANT_HLAST | SSM_A_DIRECT | SSM_ZOH;
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
 constexpr int kMaxDstate = 64;
 
@@ -103,7 +103,7 @@ ssm_status validate_desc(const ssm_scan_desc *d) {
   if (d->flags & ~kKnownFlags) return SSM_ERR_INVALID_ARG;
   if (d->flags & SSM_A_DIRECT) {
     if (d->dstate != 1) return SSM_ERR_INVALID_ARG;
-    if (d->flags & (SSM_HAS_Z | SSM_HAS_D | SSM_DELTA_SOFTPLUS | SSM_HAS_DELTA_BIAS))
+    if (d->flags & (SSM_HAS_Z | SSM_HAS_D | SSM_DELTA_SOFTPLUS | SSM_HAS_DELTA_BIAS | SSM_ZOH))
       return SSM_ERR_INVALID_ARG;
   }
   if (d->dstate > kMaxDstate) return SSM_ERR_UNSUPPORTED;
@@ -133,7 +133,7 @@ ssm_status plan_tma(ssm_scan_plan *pl) {
                             pl->cfg.grid};
   ssm::FwdShape fs;
   if (ssm::choose_fwd_shape((int)d.in_dtype, (int)d.out_dtype, d.batch, d.seqlen, d.dim, ns,
-                            pl->num_sms, o, &fs) != cudaSuccess) {
+                            (d.flags & SSM_ZOH) != 0, pl->num_sms, o, &fs) != cudaSuccess) {
     cudaGetLastError();
     return SSM_ERR_UNSUPPORTED;  // no variant fits (or bad override)
   }
@@ -378,6 +378,7 @@ ssm_status ssm_scan_fwd(ssm_scan_plan *pl, const void *x, const void *delta,
     p.has_bias = (f & SSM_HAS_DELTA_BIAS) != 0;
     p.has_h0 = (f & SSM_HAS_H0) != 0;
     p.want_hlast = (f & SSM_WANT_HLAST) != 0;
+    p.zoh = (f & SSM_ZOH) != 0;
     p.A = static_cast<const float *>(A);
     p.Dv = D; p.bias = delta_bias; p.h0 = h0; p.h_last = h_last; p.y = y;
     p.ws_state = pl->ws_state; p.ws_flags = pl->ws_flags; p.ctl = pl->ctl;
@@ -394,6 +395,7 @@ ssm_status ssm_scan_fwd(ssm_scan_plan *pl, const void *x, const void *delta,
   p.has_bias = f & SSM_HAS_DELTA_BIAS;
   p.has_h0 = f & SSM_HAS_H0;
   p.want_hlast = f & SSM_WANT_HLAST;
+  p.zoh = f & SSM_ZOH;
   p.in_bf16 = d.in_dtype == SSM_BF16;
   p.out_bf16 = d.out_dtype == SSM_BF16;
   p.x = x; p.dt = delta; p.z = z; p.B = B; p.C = C;
@@ -424,6 +426,7 @@ ssm_status ssm_scan_step(ssm_scan_plan *pl, const void *x, const void *delta,
   p.has_z = f & SSM_HAS_Z;
   p.has_D = f & SSM_HAS_D;
   p.has_bias = f & SSM_HAS_DELTA_BIAS;
+  p.zoh = f & SSM_ZOH;
   p.in_bf16 = d.in_dtype == SSM_BF16;
   p.out_bf16 = d.out_dtype == SSM_BF16;
   p.x = x; p.dt = delta; p.z = z; p.B = B; p.C = C;

@@ -96,6 +96,7 @@ class ScanInputs:
     h0: np.ndarray | None = None
     delta_softplus: bool = True
     want_h_last: bool = True
+    zoh: bool = False          # zero-order-hold input matrix instead of Delta * B
     meta: dict = field(default_factory=dict)
 
     @property
@@ -105,7 +106,7 @@ class ScanInputs:
 
 def make_fwd(Bsz, L, D, N, *, in_dtype="bf16", out_dtype=None, seed=0, has_z=True,
              has_D=True, has_bias=True, has_h0=False, delta_softplus=True,
-             delta_shift=0.0, A=None, name="custom") -> ScanInputs:
+             delta_shift=0.0, A=None, name="custom", zoh=False) -> ScanInputs:
     """Generic seeded forward workload with the standard distributions."""
     out_dtype = out_dtype or in_dtype
     x = _normal(seed, _F_X, (Bsz, L, D), in_dtype)
@@ -119,7 +120,7 @@ def make_fwd(Bsz, L, D, N, *, in_dtype="bf16", out_dtype=None, seed=0, has_z=Tru
           if has_h0 else None)
     A = s4d_real_A(D, N) if A is None else np.ascontiguousarray(A, dtype=np.float32)
     return ScanInputs(name, Bsz, L, D, N, in_dtype, out_dtype, x, delta, A, Bm, Cm, Dv, z,
-                      bias, h0, delta_softplus, True)
+                      bias, h0, delta_softplus, True, zoh)
 
 
 def tiny_fp32(seed=0):

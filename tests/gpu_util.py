@@ -40,7 +40,8 @@ def upload(inp, device="cuda"):
 def make_plan(inp, device="cuda"):
     from selective_state_space_31_b200 import binding as bnd
     flags = bnd.flags_for(z=inp.z, D=inp.Dskip, delta_bias=inp.delta_bias, h0=inp.h0,
-                          delta_softplus=inp.delta_softplus, want_h_last=inp.want_h_last)
+                          delta_softplus=inp.delta_softplus, want_h_last=inp.want_h_last,
+                          zoh=inp.zoh)
     return bnd.Plan(inp.Bsz, inp.L, inp.D, inp.N, TDT[inp.in_dtype], TDT[inp.out_dtype], flags,
                     device)
 
@@ -58,7 +59,7 @@ def run_oracle(inp):
     import oracle
     return oracle.get().fwd(inp.x, inp.delta, inp.A, inp.B, inp.C, D=inp.Dskip, z=inp.z,
                             delta_bias=inp.delta_bias, h0=inp.h0,
-                            delta_softplus=inp.delta_softplus)
+                            delta_softplus=inp.delta_softplus, zoh=inp.zoh)
 
 
 def normwise(got, ref):

@@ -232,6 +232,65 @@ def test_decode_streaming_many_tiles_per_cta():
     gu.assert_parity(y, ry, state.cpu().numpy(), rh, gu.TOL["bf16"], "decode, many tiles")
 
 
+@pytest.mark.parametrize("cfg", [None, dict(lanes_per_chan=4, warps_per_cta=4, tile_t=32),
+                                 dict(lanes_per_chan=8, warps_per_cta=4, tile_t=64, grid=2),
+                                 dict(lanes_per_chan=16, warps_per_cta=4, tile_t=64),
+                                 dict(lanes_per_chan=1, warps_per_cta=2, tile_t=32),
+                                 dict(lanes_per_chan=2, warps_per_cta=8, tile_t=64)])
+@pytest.mark.parametrize("shift", [0.0, 3.0])
+def test_zoh_fused(cfg, shift):
+    """Zero-order hold ([P1] "Vi du Python": Bbar = (exp(Delta A) - 1)/A * B)
+    on the fused kernel: bf16, gate, skip, bias, h0, ragged L.  shift=3 moves
+    Delta up so most |Delta A| take the e - 1 branch; shift=0 keeps most in
+    the Taylor branch."""
+    inp = synth.make_fwd(3, 389, 64, 16, seed=41, has_h0=True, delta_shift=shift, zoh=True)
+    _case(inp, cfg, expect_path=0)
+
+
+@pytest.mark.parametrize("N", [4, 16])
+def test_zoh_fp32_and_zero_A(N):
+    """fp32 zero-order hold at the fp32 tolerance, with some A entries 0 (the
+    limit Bbar = Delta * B) and some tiny."""
+    A = -np.tile(np.arange(1, N + 1, dtype=np.float32), (32, 1))
+    A[::3, 0] = 0.0
+    A[1::3, 1] = -1e-6
+    inp = synth.make_fwd(2, 200, 32, N, in_dtype="f32", seed=42, has_h0=True, A=A, zoh=True)
+    _case(inp, expect_path=0)
+
+
+def test_zoh_general_path():
+    """Zero-order hold on the general kernel (odd dim and dstate)."""
+    inp = synth.make_fwd(2, 77, 37, 12, in_dtype="f32", seed=43, has_h0=True, zoh=True)
+    _case(inp, expect_path=1)
+
+
+@pytest.mark.parametrize("N,dt", [(16, "bf16"), (4, "f32"), (12, "f32")])
+def test_zoh_decode_steps(N, dt):
+    """Zero-order-hold decode steps reproduce the oracle's full sequence."""
+    import oracle
+    from selective_state_space_31_b200 import binding as bnd
+    inp = synth.make_fwd(4, 24, 96, N, in_dtype=dt, seed=44, has_h0=True, delta_shift=1.0,
+                         zoh=True)
+    dev = gu.upload(inp)
+    state = dev["h0"].clone()
+    ys = []
+    for t in range(inp.L):
+        ys.append(bnd.step(state, dev["x"][:, t].contiguous(), dev["delta"][:, t].contiguous(),
+                           dev["A"], dev["B"][:, t].contiguous(), dev["C"][:, t].contiguous(),
+                           D=dev["D"], z=dev["z"][:, t].contiguous(),
+                           delta_bias=dev["delta_bias"], zoh=True))
+    y = torch.stack(ys, dim=1).float().cpu().numpy()
+    ry, rh = gu.run_oracle(inp)
+    gu.assert_parity(y, ry, state.cpu().numpy(), rh, gu.TOL[dt], f"zoh decode N={N}")
+
+
+def test_zoh_refused_with_elementwise_variant():
+    from selective_state_space_31_b200 import binding as bnd
+    with pytest.raises(bnd.SsmError):
+        bnd.Plan(1, 4, 8, 1, torch.float32, torch.float32, bnd.A_DIRECT | bnd.ZOH,
+                 torch.device("cuda", 0))
+
+
 def test_timeout_is_reported_without_hanging():
     """A work item that never hands its state on makes the CTA running the
     next part of that row wait until the bound expires: the kernel records
