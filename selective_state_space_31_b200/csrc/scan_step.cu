@@ -43,7 +43,7 @@ __device__ __forceinline__ void ldg4(const __nv_bfloat16 *src, float *v) {
 // TPC threads share a channel; thread q owns the 4-state groups q, q + TPC,
 // q + 2 TPC, ... (NPT states), so each of its 16-byte state accesses, taken
 // over the warp, covers whole 32-byte sectors.
-template <typename InT, typename OutT, int NPT, int TPC, int ITEMS>
+template <typename InT, typename OutT, int NPT, int TPC, int ITEMS, bool ZOH>
 __global__ void __launch_bounds__(256, SSM_STEP_MINB) step_kernel(const StepParams p) {
   // ITEMS work items per thread, a grid apart: every item's state reads are
   // issued before any of them is used
@@ -95,9 +95,9 @@ __global__ void __launch_bounds__(256, SSM_STEP_MINB) step_kernel(const StepPara
         const float arg = dlt * (Av[n] * kLog2e);
         const float a = ex2_approx(arg);
         // Bbar x: Delta B x, or (e^{Delta A} - 1) / A * B x under zero-order hold
-        const float bx = p.zoh ? zoh_coef(arg * kLn2, a, dlt, Av[n] != 0.f ? 1.f / Av[n] : 0.f) *
-                                     xv * Bv[n]
-                               : dtx * Bv[n];
+        float bx = dtx * Bv[n];
+        if constexpr (ZOH)
+          bx = zoh_coef(arg * kLn2, a, dlt, Av[n] != 0.f ? 1.f / Av[n] : 0.f) * xv * Bv[n];
         h[n] = fmaf(a, h[n], bx);
         acc = fmaf(Cv[n], h[n], acc);
       }
@@ -151,13 +151,24 @@ static cudaError_t step_typed(const StepParams &p, bool vec_ok, cudaStream_t str
   constexpr int IT = SSM_STEP_ITEMS;
   auto grid_for = [&](int tpc) { return (unsigned)((chans * tpc + 256 * IT - 1) / (256 * IT)); };
   if (vec_ok) {
-    switch (p.N) {
-      case 4: step_kernel<InT, OutT, 4, 1, IT><<<grid_for(1), 256, 0, stream>>>(p); return cudaGetLastError();
-      case 8: step_kernel<InT, OutT, 8, 1, IT><<<grid_for(1), 256, 0, stream>>>(p); return cudaGetLastError();
-      case 16: step_kernel<InT, OutT, 8, 2, IT><<<grid_for(2), 256, 0, stream>>>(p); return cudaGetLastError();
-      case 32: step_kernel<InT, OutT, 8, 4, IT><<<grid_for(4), 256, 0, stream>>>(p); return cudaGetLastError();
-      case 64: step_kernel<InT, OutT, 8, 8, IT><<<grid_for(8), 256, 0, stream>>>(p); return cudaGetLastError();
-      default: break;
+    if (p.zoh) {
+      switch (p.N) {
+        case 4: step_kernel<InT, OutT, 4, 1, IT, true><<<grid_for(1), 256, 0, stream>>>(p); return cudaGetLastError();
+        case 8: step_kernel<InT, OutT, 8, 1, IT, true><<<grid_for(1), 256, 0, stream>>>(p); return cudaGetLastError();
+        case 16: step_kernel<InT, OutT, 8, 2, IT, true><<<grid_for(2), 256, 0, stream>>>(p); return cudaGetLastError();
+        case 32: step_kernel<InT, OutT, 8, 4, IT, true><<<grid_for(4), 256, 0, stream>>>(p); return cudaGetLastError();
+        case 64: step_kernel<InT, OutT, 8, 8, IT, true><<<grid_for(8), 256, 0, stream>>>(p); return cudaGetLastError();
+        default: break;
+      }
+    } else {
+      switch (p.N) {
+        case 4: step_kernel<InT, OutT, 4, 1, IT, false><<<grid_for(1), 256, 0, stream>>>(p); return cudaGetLastError();
+        case 8: step_kernel<InT, OutT, 8, 1, IT, false><<<grid_for(1), 256, 0, stream>>>(p); return cudaGetLastError();
+        case 16: step_kernel<InT, OutT, 8, 2, IT, false><<<grid_for(2), 256, 0, stream>>>(p); return cudaGetLastError();
+        case 32: step_kernel<InT, OutT, 8, 4, IT, false><<<grid_for(4), 256, 0, stream>>>(p); return cudaGetLastError();
+        case 64: step_kernel<InT, OutT, 8, 8, IT, false><<<grid_for(8), 256, 0, stream>>>(p); return cudaGetLastError();
+        default: break;
+      }
     }
   }
   step_general_kernel<InT, OutT><<<(unsigned)((chans + 127) / 128), 128, 0, stream>>>(p);
