@@ -313,6 +313,47 @@ def test_degenerate_A(case, dim, path):
         assert gu.normwise(gy, ref) <= gu.TOL["f32"]
 
 
+def test_fwd_replayed_from_a_cuda_graph():
+    """Two forward calls captured in one CUDA graph and replayed four times:
+    the launch epoch and finished-CTA counter live on the device (no memset,
+    no host round trip), so every replay hands carried states between CTAs
+    correctly and reproduces the eager result bit for bit."""
+    inp = synth.make_fwd(3, 389, 64, 16, seed=46, has_h0=True)
+    plan = gu.make_plan(inp)
+    plan.set_config(lanes_per_chan=4, warps_per_cta=4, grid=4, tile_t=32)  # 6 rows on 4 CTAs
+    assert plan.info()["parts_per_row"] >= 2
+    dev = gu.upload(inp)
+    y = torch.empty((inp.Bsz, inp.L, inp.D), dtype=torch.bfloat16, device="cuda")
+    hl = torch.empty((inp.Bsz, inp.D, inp.N), dtype=torch.float32, device="cuda")
+
+    def call():
+        plan.fwd(dev["x"], dev["delta"], dev["A"], dev["B"], dev["C"], D=dev["D"], z=dev["z"],
+                 delta_bias=dev["delta_bias"], h0=dev["h0"], y=y, h_last=hl)
+
+    call()
+    torch.cuda.synchronize()
+    y_ref, hl_ref = y.clone(), hl.clone()
+    ry, rh = gu.run_oracle(inp)
+    gu.assert_parity(y_ref.float().cpu().numpy(), ry, hl_ref.cpu().numpy(), rh, gu.TOL["bf16"],
+                     "eager")
+    side = torch.cuda.Stream()
+    with torch.cuda.stream(side):
+        call()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        call()
+        call()
+    for _ in range(4):
+        y.zero_()
+        hl.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(y, y_ref) and torch.equal(hl, hl_ref)
+    assert plan.status() == 0
+    del graph
+
+
 def test_timeout_is_reported_without_hanging():
     """A work item that never hands its state on makes the CTA running the
     next part of that row wait until the bound expires: the kernel records
