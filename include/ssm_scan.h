@@ -115,7 +115,7 @@ typedef struct {
   int lanes_per_chan;  /* lanes sharing one channel's dstate states */
   int warps_per_cta;
   int tile_t;          /* tokens per pipeline stage (one work unit) */
-  int stages;          /* pipeline depth */
+  int stages;          /* stage slots in the TMA ring (fused kernel) */
   int stages_per_row;  /* ceil(seqlen / tile_t) */
   int chans_per_cta;   /* channels per row tile */
   int grid;            /* CTAs launched (CTA c runs items c, c + grid, ...) */

@@ -6,8 +6,8 @@
 namespace ssm {
 
 cudaError_t fwd_dispatch_bf16_f32(const LaunchShape *ls, const TmaMaps *maps, const FwdParams *p,
-                            cudaStream_t st, size_t *sm, int *oc) {
-  return by_ns<__nv_bfloat16, float>(ls, maps, p, st, sm, oc);
+                            cudaStream_t st, VariantInfo *vi) {
+  return by_ns<__nv_bfloat16, float>(ls, maps, p, st, vi);
 }
 
 }  // namespace ssm

@@ -8,21 +8,21 @@ namespace ssm {
 
 static cudaError_t dispatch(int in_dtype, int out_dtype, const LaunchShape *ls,
                             const TmaMaps *maps, const FwdParams *p, cudaStream_t st,
-                            size_t *sm, int *oc) {
-  if (in_dtype == 0 && out_dtype == 0) return fwd_dispatch_f32(ls, maps, p, st, sm, oc);
-  if (in_dtype == 1 && out_dtype == 1) return fwd_dispatch_bf16(ls, maps, p, st, sm, oc);
-  if (in_dtype == 1 && out_dtype == 0) return fwd_dispatch_bf16_f32(ls, maps, p, st, sm, oc);
+                            VariantInfo *vi) {
+  if (in_dtype == 0 && out_dtype == 0) return fwd_dispatch_f32(ls, maps, p, st, vi);
+  if (in_dtype == 1 && out_dtype == 1) return fwd_dispatch_bf16(ls, maps, p, st, vi);
+  if (in_dtype == 1 && out_dtype == 0) return fwd_dispatch_bf16_f32(ls, maps, p, st, vi);
   return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_fwd_tma(int in_dtype, int out_dtype, const LaunchShape &ls,
                            const TmaMaps &maps, const FwdParams &p, cudaStream_t stream) {
-  return dispatch(in_dtype, out_dtype, &ls, &maps, &p, stream, nullptr, nullptr);
+  return dispatch(in_dtype, out_dtype, &ls, &maps, &p, stream, nullptr);
 }
 
-cudaError_t fwd_tma_smem_and_occupancy(int in_dtype, int out_dtype, const LaunchShape &ls,
-                                       size_t *smem, int *blocks_per_sm) {
-  return dispatch(in_dtype, out_dtype, &ls, nullptr, nullptr, nullptr, smem, blocks_per_sm);
+cudaError_t fwd_variant_info(int in_dtype, int out_dtype, const LaunchShape &ls,
+                             VariantInfo *vi) {
+  return dispatch(in_dtype, out_dtype, &ls, nullptr, nullptr, nullptr, vi);
 }
 
 namespace {
@@ -87,15 +87,13 @@ cudaError_t choose_fwd_shape(int in_dtype, int out_dtype, int64_t batch, int64_t
         const int DT = warps * 32 / lpc;
         if ((DT * ei) % 16 || (DT * eo) % 16) continue;
         LaunchShape ls{lpc, warps, tt, kStages, ns, 0, 0, zoh};
-        int occ = 0;
-        size_t smem = 0;
-        if (fwd_tma_smem_and_occupancy(in_dtype, out_dtype, ls, &smem, &occ) != cudaSuccess ||
-            occ < 1) {
+        VariantInfo vi{};
+        if (fwd_variant_info(in_dtype, out_dtype, ls, &vi) != cudaSuccess || vi.occ < 1) {
           cudaGetLastError();
           continue;
         }
         const int64_t rows = batch * ((dim + DT - 1) / DT);
-        const int64_t cap = std::min<int64_t>(rows, (int64_t)occ * sms);
+        const int64_t cap = std::min<int64_t>(rows, (int64_t)vi.occ * sms);
         const int64_t balanced = cap >= sms ? cap / sms * sms : cap;
         const double w = shape_weight(lpc, tt) * warps_weight(warps);
         auto score_of = [&](int64_t g) {
@@ -105,14 +103,15 @@ cudaError_t choose_fwd_shape(int in_dtype, int out_dtype, int64_t batch, int64_t
           return std::min(busy, 12.0) / 12.0 * balance * w - 1e-3 * warps;
         };
         int64_t grid = score_of(balanced) >= score_of(cap) ? balanced : cap;
-        if (o.grid > 0) grid = std::min<int64_t>(o.grid, (int64_t)occ * sms);
+        if (o.grid > 0) grid = std::min<int64_t>(o.grid, (int64_t)vi.occ * sms);
         const double score = score_of(grid);
         if (!found || score > best_score) {
           found = true;
           best_score = score;
-          best = FwdShape{ls, DT, rows, 0, 0, 0};
+          best = FwdShape{ls, DT, rows, 0, 0, 0, 0};
           best.ls.grid = (int)grid;
-          best.ls.smem = smem;
+          best.ls.smem = vi.smem;
+          best.ring = vi.ring;
         }
       }
     }

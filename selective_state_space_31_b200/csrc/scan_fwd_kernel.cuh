@@ -421,7 +421,7 @@ __global__ void __launch_bounds__((WARPS + 1) * 32)
 
 template <typename InT, typename OutT, int NS, int LPC, int WARPS, int TT, bool ZOH>
 static cudaError_t run_variant(const LaunchShape *ls, const TmaMaps *maps, const FwdParams *p,
-                               cudaStream_t stream, size_t *smem_out, int *occ_out) {
+                               cudaStream_t stream, VariantInfo *vi) {
   using Cfg = FwdCfg<InT, OutT, NS, LPC, WARPS, TT>;
   auto kern = fwd_kernel<InT, OutT, NS, LPC, WARPS, TT, ZOH>;
   if (Cfg::SMEM > 227 * 1024) return cudaErrorInvalidValue;
@@ -430,9 +430,10 @@ static cudaError_t run_variant(const LaunchShape *ls, const TmaMaps *maps, const
     cudaGetLastError();
     return e;
   }
-  if (smem_out) *smem_out = Cfg::SMEM;
-  if (occ_out) {
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(occ_out, kern, Cfg::THREADS, Cfg::SMEM);
+  if (vi) {
+    vi->smem = Cfg::SMEM;
+    vi->ring = Cfg::RAW;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&vi->occ, kern, Cfg::THREADS, Cfg::SMEM);
     if (e != cudaSuccess) return e;
   }
   if (!maps) return cudaSuccess;
@@ -442,17 +443,17 @@ static cudaError_t run_variant(const LaunchShape *ls, const TmaMaps *maps, const
 
 template <typename InT, typename OutT, int NS, int LPC, int WARPS, bool ZOH>
 static cudaError_t by_tt(const LaunchShape *ls, const TmaMaps *maps, const FwdParams *p,
-                         cudaStream_t st, size_t *sm, int *oc) {
+                         cudaStream_t st, VariantInfo *vi) {
   // a row tile's x / delta / z rows must be whole 16-byte TMA units
   if constexpr ((WARPS * (32 / LPC) * (int)sizeof(InT)) % 16 != 0) {
     return cudaErrorInvalidValue;
   } else {
     switch (ls->tt) {
       case 16:
-        if constexpr (!ZOH) return run_variant<InT, OutT, NS, LPC, WARPS, 16, ZOH>(ls, maps, p, st, sm, oc);
+        if constexpr (!ZOH) return run_variant<InT, OutT, NS, LPC, WARPS, 16, ZOH>(ls, maps, p, st, vi);
         return cudaErrorInvalidValue;
-      case 32: return run_variant<InT, OutT, NS, LPC, WARPS, 32, ZOH>(ls, maps, p, st, sm, oc);
-      case 64: return run_variant<InT, OutT, NS, LPC, WARPS, 64, ZOH>(ls, maps, p, st, sm, oc);
+      case 32: return run_variant<InT, OutT, NS, LPC, WARPS, 32, ZOH>(ls, maps, p, st, vi);
+      case 64: return run_variant<InT, OutT, NS, LPC, WARPS, 64, ZOH>(ls, maps, p, st, vi);
       default: return cudaErrorInvalidValue;
     }
   }
@@ -460,27 +461,27 @@ static cudaError_t by_tt(const LaunchShape *ls, const TmaMaps *maps, const FwdPa
 
 template <typename InT, typename OutT, int NS, int LPC, bool ZOH>
 static cudaError_t by_warps(const LaunchShape *ls, const TmaMaps *maps, const FwdParams *p,
-                            cudaStream_t st, size_t *sm, int *oc) {
+                            cudaStream_t st, VariantInfo *vi) {
   switch (ls->warps) {
-    case 2: return by_tt<InT, OutT, NS, LPC, 2, ZOH>(ls, maps, p, st, sm, oc);
-    case 4: return by_tt<InT, OutT, NS, LPC, 4, ZOH>(ls, maps, p, st, sm, oc);
-    case 8: return by_tt<InT, OutT, NS, LPC, 8, ZOH>(ls, maps, p, st, sm, oc);
+    case 2: return by_tt<InT, OutT, NS, LPC, 2, ZOH>(ls, maps, p, st, vi);
+    case 4: return by_tt<InT, OutT, NS, LPC, 4, ZOH>(ls, maps, p, st, vi);
+    case 8: return by_tt<InT, OutT, NS, LPC, 8, ZOH>(ls, maps, p, st, vi);
     default: return cudaErrorInvalidValue;
   }
 }
 
 template <typename InT, typename OutT, int NS, bool ZOH>
 static cudaError_t by_lpc(const LaunchShape *ls, const TmaMaps *maps, const FwdParams *p,
-                          cudaStream_t st, size_t *sm, int *oc) {
+                          cudaStream_t st, VariantInfo *vi) {
   switch (ls->lpc) {
-    case 1: return by_warps<InT, OutT, NS, 1, ZOH>(ls, maps, p, st, sm, oc);
-    case 2: return by_warps<InT, OutT, NS, 2, ZOH>(ls, maps, p, st, sm, oc);
-    case 4: return by_warps<InT, OutT, NS, 4, ZOH>(ls, maps, p, st, sm, oc);
+    case 1: return by_warps<InT, OutT, NS, 1, ZOH>(ls, maps, p, st, vi);
+    case 2: return by_warps<InT, OutT, NS, 2, ZOH>(ls, maps, p, st, vi);
+    case 4: return by_warps<InT, OutT, NS, 4, ZOH>(ls, maps, p, st, vi);
     case 8:
-      if constexpr (NS >= 8) return by_warps<InT, OutT, NS, 8, ZOH>(ls, maps, p, st, sm, oc);
+      if constexpr (NS >= 8) return by_warps<InT, OutT, NS, 8, ZOH>(ls, maps, p, st, vi);
       return cudaErrorInvalidValue;
     case 16:
-      if constexpr (NS >= 16) return by_warps<InT, OutT, NS, 16, ZOH>(ls, maps, p, st, sm, oc);
+      if constexpr (NS >= 16) return by_warps<InT, OutT, NS, 16, ZOH>(ls, maps, p, st, vi);
       return cudaErrorInvalidValue;
     default: return cudaErrorInvalidValue;
   }
@@ -488,32 +489,32 @@ static cudaError_t by_lpc(const LaunchShape *ls, const TmaMaps *maps, const FwdP
 
 template <typename InT, typename OutT, bool ZOH>
 static cudaError_t by_ns_zoh(const LaunchShape *ls, const TmaMaps *maps, const FwdParams *p,
-                             cudaStream_t st, size_t *sm, int *oc) {
+                             cudaStream_t st, VariantInfo *vi) {
   switch (ls->ns) {
     case 4:
-      if constexpr (sizeof(InT) == 4) return by_lpc<InT, OutT, 4, ZOH>(ls, maps, p, st, sm, oc);
+      if constexpr (sizeof(InT) == 4) return by_lpc<InT, OutT, 4, ZOH>(ls, maps, p, st, vi);
       return cudaErrorInvalidValue;
-    case 8: return by_lpc<InT, OutT, 8, ZOH>(ls, maps, p, st, sm, oc);
-    case 16: return by_lpc<InT, OutT, 16, ZOH>(ls, maps, p, st, sm, oc);
+    case 8: return by_lpc<InT, OutT, 8, ZOH>(ls, maps, p, st, vi);
+    case 16: return by_lpc<InT, OutT, 16, ZOH>(ls, maps, p, st, vi);
     default: return cudaErrorInvalidValue;
   }
 }
 
 template <typename InT, typename OutT>
 static cudaError_t by_ns(const LaunchShape *ls, const TmaMaps *maps, const FwdParams *p,
-                         cudaStream_t st, size_t *sm, int *oc) {
+                         cudaStream_t st, VariantInfo *vi) {
   if (ls->stages != kStages) return cudaErrorInvalidValue;
   if (p && p->zoh != ls->zoh) return cudaErrorInvalidValue;
-  return ls->zoh ? by_ns_zoh<InT, OutT, true>(ls, maps, p, st, sm, oc)
-                 : by_ns_zoh<InT, OutT, false>(ls, maps, p, st, sm, oc);
+  return ls->zoh ? by_ns_zoh<InT, OutT, true>(ls, maps, p, st, vi)
+                 : by_ns_zoh<InT, OutT, false>(ls, maps, p, st, vi);
 }
 
 // per-dtype entry points (defined in scan_fwd_<dtypes>.cu)
 cudaError_t fwd_dispatch_f32(const LaunchShape *, const TmaMaps *, const FwdParams *, cudaStream_t,
-                             size_t *, int *);
+                             VariantInfo *);
 cudaError_t fwd_dispatch_bf16(const LaunchShape *, const TmaMaps *, const FwdParams *,
-                              cudaStream_t, size_t *, int *);
+                              cudaStream_t, VariantInfo *);
 cudaError_t fwd_dispatch_bf16_f32(const LaunchShape *, const TmaMaps *, const FwdParams *,
-                                  cudaStream_t, size_t *, int *);
+                                  cudaStream_t, VariantInfo *);
 
 }  // namespace ssm

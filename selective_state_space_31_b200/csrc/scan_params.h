@@ -56,9 +56,14 @@ struct LaunchShape {
 // Fused forward kernel (scan_fwd_kernel.cuh, instantiated per dtype pair).
 cudaError_t launch_fwd_tma(int in_dtype, int out_dtype, const LaunchShape &ls,
                            const TmaMaps &maps, const FwdParams &p, cudaStream_t stream);
-// Dynamic shared memory and per-SM residency of one chunked-kernel variant.
-cudaError_t fwd_tma_smem_and_occupancy(int in_dtype, int out_dtype, const LaunchShape &ls,
-                                       size_t *smem, int *blocks_per_sm);
+// What one fused-kernel variant needs and gets on the device.
+struct VariantInfo {
+  size_t smem;  // dynamic shared memory per CTA
+  int occ;      // CTAs resident per SM
+  int ring;     // stage slots in the TMA ring
+};
+cudaError_t fwd_variant_info(int in_dtype, int out_dtype, const LaunchShape &ls,
+                             VariantInfo *vi);
 
 // Pipeline tag every fused-kernel LaunchShape carries (`stages`).
 constexpr int kStages = 2;
@@ -76,6 +81,7 @@ struct FwdShape {
   int S;           // stages per row
   int PL;          // stages per part
   int parts;       // parts per row
+  int ring;        // stage slots in the TMA ring
 };
 // Choose the fused kernel's launch shape for a problem (scan_fwd_dispatch.cu).
 // Returns cudaErrorInvalidValue when no variant fits the overrides.

@@ -84,6 +84,7 @@ struct ssm_scan_plan {
   int64_t rows = 0, units = 0;
   ssm_scan_config cfg{};  // user overrides
   ssm::Control *ctl = nullptr;
+  int ring = 0;  // stage slots of the fused kernel's TMA ring
   float *ws_state = nullptr;
   unsigned long long *ws_flags = nullptr;
   size_t ws_state_bytes = 0, ws_flag_bytes = 0;
@@ -162,6 +163,7 @@ ssm_status plan_tma(ssm_scan_plan *pl) {
   pl->S = fs.S;
   pl->PL = fs.PL;
   pl->parts = fs.parts;
+  pl->ring = fs.ring;
   pl->rows = fs.rows;
   pl->units = fs.rows * fs.S;
   return SSM_OK;
@@ -262,7 +264,7 @@ ssm_status ssm_scan_get_info(const ssm_scan_plan *pl, ssm_scan_info *info) {
     info->lanes_per_chan = pl->ls.lpc;
     info->warps_per_cta = pl->ls.warps;
     info->tile_t = pl->ls.tt;
-    info->stages = pl->ls.stages;
+    info->stages = pl->ring;
     info->stages_per_row = pl->S;
     info->chans_per_cta = pl->DT;
     info->grid = pl->ls.grid;
