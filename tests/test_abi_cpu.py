@@ -36,6 +36,20 @@ def test_every_declared_symbol_is_exported(lib):
     assert not missing, missing
 
 
+def test_flag_and_status_values_match_the_header():
+    """The binding's flag, dtype and status constants are the values the C
+    header defines."""
+    src = open(os.path.join(ROOT, "include", "ssm_scan.h")).read()
+    defined = {name: int(val) for name, val in re.findall(r"\b(SSM_[A-Z0-9_]+)\s*=\s*(\d+)", src)}
+    expect = {"SSM_HAS_Z": bnd.HAS_Z, "SSM_HAS_D": bnd.HAS_D,
+              "SSM_DELTA_SOFTPLUS": bnd.DELTA_SOFTPLUS, "SSM_HAS_DELTA_BIAS": bnd.HAS_DELTA_BIAS,
+              "SSM_HAS_H0": bnd.HAS_H0, "SSM_WANT_HLAST": bnd.WANT_HLAST,
+              "SSM_A_DIRECT": bnd.A_DIRECT, "SSM_ZOH": bnd.ZOH, "SSM_F32": bnd.F32,
+              "SSM_BF16": bnd.BF16, "SSM_OK": bnd.OK, "SSM_ERR_INVALID_ARG": bnd.ERR_INVALID_ARG}
+    for name, val in expect.items():
+        assert defined.get(name) == val, (name, defined.get(name), val)
+
+
 def test_status_strings(lib):
     for s in range(7):
         assert bnd.status_string(s)

@@ -31,10 +31,12 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-@pytest.mark.parametrize("shape,dt", [((4, 1000, 256, 16), "bf16"), ((2, 333, 64, 8), "f32")])
-def test_noalloc_matches_plan_entry_point(shape, dt):
+@pytest.mark.parametrize("shape,dt,zoh", [((4, 1000, 256, 16), "bf16", False),
+                                          ((2, 333, 64, 8), "f32", False),
+                                          ((2, 333, 64, 16), "bf16", True)])
+def test_noalloc_matches_plan_entry_point(shape, dt, zoh):
     Bz, L, D, N = shape
-    inp = synth.make_fwd(Bz, L, D, N, in_dtype=dt, seed=41, has_h0=True)
+    inp = synth.make_fwd(Bz, L, D, N, in_dtype=dt, seed=41, has_h0=True, zoh=zoh)
     dev = gu.upload(inp)
     plan = gu.make_plan(inp)
     y_ref, h_ref = gu.run_gpu(inp, plan, dev)
