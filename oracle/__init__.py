@@ -75,6 +75,8 @@ class Oracle:
         self._lib.ssm_oracle_step.restype = ctypes.c_int
         self._lib.ssm_oracle_direct.argtypes = [i64, i64, i64] + [_dp] * 7
         self._lib.ssm_oracle_direct.restype = ctypes.c_int
+        self._lib.ssm_oracle_bwd.argtypes = [i64, i64, i64, i64, u32] + [_dp] * 20
+        self._lib.ssm_oracle_bwd.restype = ctypes.c_int
         self._lib.ssm_oracle_softplus.argtypes = [ctypes.c_double]
         self._lib.ssm_oracle_softplus.restype = ctypes.c_double
         self._lib.ssm_oracle_silu.argtypes = [ctypes.c_double]
@@ -113,6 +115,46 @@ class Oracle:
         if rc != 0:
             raise ValueError("oracle fwd rejected its arguments")
         return y, hl
+
+    def bwd(self, x, delta, A, B, C, dy, D=None, z=None, delta_bias=None, h0=None,
+            dh_last=None, delta_softplus=True):
+        """Gradients of the Mamba-form scan (Delta*B coefficient) for
+        dL/dy = dy (Bsz, L, Dm) and dL/dh_last = dh_last (Bsz, Dm, N) or None.
+        Returns a dict with x, delta, A, B, C and, where given, D, z,
+        delta_bias, h0 (float64 arrays shaped like the inputs)."""
+        x = _arr(x)
+        Bsz, L, Dm = x.shape
+        A = _arr(A)
+        N = A.shape[1]
+        delta = _arr(delta, x.shape)
+        Bm = _arr(B, (Bsz, L, N))
+        Cm = _arr(C, (Bsz, L, N))
+        z = _arr(z, x.shape)
+        Dv = _arr(D, (Dm,))
+        bias = _arr(delta_bias, (Dm,))
+        h0 = _arr(h0, (Bsz, Dm, N))
+        dy = _arr(dy, x.shape)
+        dhl = _arr(dh_last, (Bsz, Dm, N))
+        flags = ((HAS_Z if z is not None else 0) | (HAS_D if Dv is not None else 0)
+                 | (SOFTPLUS if delta_softplus else 0) | (HAS_BIAS if bias is not None else 0)
+                 | (HAS_H0 if h0 is not None else 0))
+        out = {"x": np.empty_like(x), "delta": np.empty_like(x), "A": np.empty_like(A),
+               "B": np.empty_like(Bm), "C": np.empty_like(Cm)}
+        if Dv is not None:
+            out["D"] = np.empty_like(Dv)
+        if z is not None:
+            out["z"] = np.empty_like(z)
+        if bias is not None:
+            out["delta_bias"] = np.empty_like(bias)
+        out["h0"] = np.empty((Bsz, Dm, N), np.float64)
+        g = lambda k: _ptr(out.get(k))
+        rc = self._lib.ssm_oracle_bwd(Bsz, L, Dm, N, flags, _ptr(x), _ptr(delta), _ptr(bias),
+                                      _ptr(A), _ptr(Bm), _ptr(Cm), _ptr(Dv), _ptr(z), _ptr(h0),
+                                      _ptr(dy), _ptr(dhl), g("x"), g("delta"), g("delta_bias"),
+                                      g("A"), g("B"), g("C"), g("D"), g("z"), g("h0"))
+        if rc != 0:
+            raise ValueError("oracle bwd rejected its arguments")
+        return out
 
     def step(self, state, x, delta, A, B, C, D=None, z=None, delta_bias=None,
              delta_softplus=True):

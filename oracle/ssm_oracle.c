@@ -31,6 +31,10 @@
  * In the elementwise variant x, A, B, C, y are (B, L, D) and h0, h_last are
  * (B, D).
  *
+ * ssm_oracle_bwd is the reverse-mode gradient of the forward pass (the
+ * chain rule applied to the same steps), pinned by central finite
+ * differences of ssm_oracle_fwd.
+ *
  * ORACLE_MUTANT (compile-time, tests only) plants one deliberate mistake so a
  * test can show that the pins catch it.  The default build has none.
  */
@@ -217,5 +221,114 @@ int ssm_oracle_direct(int64_t Bsz, int64_t L, int64_t D, const double *x,
       if (h_last) h_last[b * D + d] = h;
     }
   }
+  return 0;
+}
+
+/* Reverse-mode gradient of ssm_oracle_fwd (Delta*B input coefficient; the
+ * zero-order-hold option is not covered and returns -1) for a loss whose
+ * derivatives are dy = dL/dy (B, L, D) and dh_last = dL/dh_last (B, D, N,
+ * NULL for 0).  For each channel the states h_0 .. h_L are recomputed and
+ * kept, then t runs L-1 .. 0 applying the chain rule to the forward steps of
+ * [P1] "Selection pha vo convolution kernel co dinh" / "Vi du Python":
+ *   v = delta + bias, Delta = softplus(v), abar_n = exp(Delta A_n),
+ *   h_t = abar h_{t-1} + Delta B_t x_t,  s_t = C_t . h_t + D x_t,
+ *   y_t = s_t silu(z_t),
+ * with g = dL/dh_t carried backwards (g <- g * abar after each token).
+ * dx, ddelta, dz: (B, L, D); dB, dC: (B, L, N); dA: (D, N); dD, dbias: (D);
+ * dh0: (B, D, N).  Outputs for absent inputs may be NULL.  Returns 0, or -1
+ * on a bad argument / allocation failure. */
+int ssm_oracle_bwd(int64_t Bsz, int64_t L, int64_t D, int64_t N, uint32_t flags,
+                   const double *x, const double *delta, const double *bias,
+                   const double *A, const double *Bm, const double *Cm,
+                   const double *Dv, const double *z, const double *h0,
+                   const double *dy, const double *dh_last, double *dx, double *ddelta,
+                   double *dbias, double *dA, double *dB, double *dC, double *dD,
+                   double *dz, double *dh0) {
+  if (Bsz < 0 || L < 0 || D < 0 || N < 1) return -1;
+  if (flags & ORC_ZOH) return -1;
+  if (!x || !delta || !A || !Bm || !Cm || !dy || !dx || !ddelta || !dA || !dB || !dC)
+    return -1;
+  if ((flags & ORC_HAS_Z) && (!z || !dz)) return -1;
+  if ((flags & ORC_HAS_D) && (!Dv || !dD)) return -1;
+  if ((flags & ORC_HAS_BIAS) && (!bias || !dbias)) return -1;
+  if ((flags & ORC_HAS_H0) && !h0) return -1;
+  for (int64_t k = 0; k < D * N; ++k) dA[k] = 0.0;
+  for (int64_t k = 0; k < Bsz * L * N; ++k) dB[k] = dC[k] = 0.0;
+  for (int64_t k = 0; k < D; ++k) {
+    if (dD) dD[k] = 0.0;
+    if (dbias) dbias[k] = 0.0;
+  }
+  double *hs = (double *)malloc((size_t)(L + 1) * (size_t)N * sizeof(double));
+  double *g = (double *)malloc((size_t)N * sizeof(double));
+  if (!hs || !g) {
+    free(hs);
+    free(g);
+    return -1;
+  }
+  for (int64_t b = 0; b < Bsz; ++b) {
+    for (int64_t d = 0; d < D; ++d) {
+      const double *Arow = A + d * N;
+      const double bv = (flags & ORC_HAS_BIAS) ? bias[d] : 0.0;
+      const double Dd = (flags & ORC_HAS_D) ? Dv[d] : 0.0;
+      /* forward, keeping every state: hs[t*N ..] = h_t (h_0 = h0) */
+      for (int64_t n = 0; n < N; ++n)
+        hs[n] = (flags & ORC_HAS_H0) ? h0[(b * D + d) * N + n] : 0.0;
+      for (int64_t t = 0; t < L; ++t) {
+        size_t i = (size_t)((b * L + t) * D + d), j = (size_t)((b * L + t) * N);
+        double v = delta[i] + bv;
+        double dt = (flags & ORC_SOFTPLUS) ? ssm_oracle_softplus(v) : v;
+        for (int64_t n = 0; n < N; ++n)
+          hs[(t + 1) * N + n] = exp(dt * Arow[n]) * hs[t * N + n] + dt * Bm[j + n] * x[i];
+      }
+      /* backward */
+      for (int64_t n = 0; n < N; ++n) g[n] = dh_last ? dh_last[(b * D + d) * N + n] : 0.0;
+      for (int64_t t = L - 1; t >= 0; --t) {
+        size_t i = (size_t)((b * L + t) * D + d), j = (size_t)((b * L + t) * N);
+        const double xv = x[i];
+        const double v = delta[i] + bv;
+        const double dt = (flags & ORC_SOFTPLUS) ? ssm_oracle_softplus(v) : v;
+        const double *ht = hs + (t + 1) * N, *hp = hs + t * N;
+        double s = Dd * xv;
+        for (int64_t n = 0; n < N; ++n) s += Cm[j + n] * ht[n];
+        double ds = dy[i];
+        if (flags & ORC_HAS_Z) {
+          const double zv = z[i], sig = 1.0 / (1.0 + exp(-zv));
+          ds = dy[i] * zv * sig;                          /* dy * silu(z) */
+          dz[i] = dy[i] * s * sig * (1.0 + zv * (1.0 - sig)); /* silu'(z) */
+#if ORACLE_MUTANT == 15
+          dz[i] = dy[i] * s * sig; /* sigmoid in place of silu' */
+#endif
+        }
+        double dxi = ds * Dd;
+        if (flags & ORC_HAS_D) dD[d] += ds * xv;
+        double ddt = 0.0;
+        for (int64_t n = 0; n < N; ++n) {
+          const double abar = exp(dt * Arow[n]);
+          dC[j + n] += ds * ht[n];
+          g[n] += ds * Cm[j + n];
+          const double dabar = g[n] * hp[n];
+          ddt += dabar * abar * Arow[n] + g[n] * Bm[j + n] * xv;
+#if ORACLE_MUTANT == 14
+          ddt -= g[n] * Bm[j + n] * xv; /* Delta's input term dropped */
+#endif
+          dA[d * N + n] += dabar * abar * dt;
+          dB[j + n] += g[n] * dt * xv;
+          dxi += g[n] * dt * Bm[j + n];
+          g[n] *= abar;
+#if ORACLE_MUTANT == 13
+          g[n] /= abar; /* state gradient not carried through Abar */
+#endif
+        }
+        dx[i] = dxi;
+        const double dv = (flags & ORC_SOFTPLUS) ? ddt / (1.0 + exp(-v)) : ddt;
+        ddelta[i] = dv;
+        if (flags & ORC_HAS_BIAS) dbias[d] += dv;
+      }
+      if (dh0)
+        for (int64_t n = 0; n < N; ++n) dh0[(b * D + d) * N + n] = g[n];
+    }
+  }
+  free(hs);
+  free(g);
   return 0;
 }

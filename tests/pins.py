@@ -416,6 +416,56 @@ def pin_p3_shape_example(orc):
     _close(y, want, 1e-12, 1e-14, "P3 example values")
 
 
+def _fd_case(orc, rng, options):
+    """Analytic gradients of L = sum(w*y) + sum(u*h_last) from orc.bwd against
+    central finite differences of orc.fwd, element by element."""
+    bsz, sl, d, n = 2, 5, 3, 4
+    inp = {"x": rng.standard_normal((bsz, sl, d)), "delta": rng.standard_normal((bsz, sl, d)),
+           "A": -np.exp(rng.standard_normal((d, n)) * 0.5),
+           "B": rng.standard_normal((bsz, sl, n)), "C": rng.standard_normal((bsz, sl, n))}
+    if options:
+        inp.update(z=rng.standard_normal((bsz, sl, d)), D=rng.standard_normal(d),
+                   delta_bias=rng.standard_normal(d) * 0.3,
+                   h0=rng.standard_normal((bsz, d, n)) * 0.5)
+    else:
+        inp["delta"] = np.abs(inp["delta"]) * 0.3 + 0.05   # Delta itself, softplus off
+    w = rng.standard_normal((bsz, sl, d))
+    u = rng.standard_normal((bsz, d, n))
+
+    def loss(vals):
+        y, hl = orc.fwd(vals["x"], vals["delta"], vals["A"], vals["B"], vals["C"],
+                        D=vals.get("D"), z=vals.get("z"), delta_bias=vals.get("delta_bias"),
+                        h0=vals.get("h0"), delta_softplus=options)
+        return float(np.sum(w * y) + np.sum(u * hl))
+
+    grads = orc.bwd(inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], w, D=inp.get("D"),
+                    z=inp.get("z"), delta_bias=inp.get("delta_bias"), h0=inp.get("h0"),
+                    dh_last=u, delta_softplus=options)
+    for name, arr in inp.items():
+        fd = np.zeros_like(arr)
+        for k in np.ndindex(arr.shape):
+            eps = 1e-6 * max(1.0, abs(arr[k]))
+            plus = {kk: vv.copy() for kk, vv in inp.items()}
+            minus = {kk: vv.copy() for kk, vv in inp.items()}
+            plus[name][k] += eps
+            minus[name][k] -= eps
+            fd[k] = (loss(plus) - loss(minus)) / (2 * eps)
+        _close(grads[name], fd, 1e-6, 1e-7 * max(1.0, float(np.max(np.abs(fd)))),
+               f"d loss / d {name} ({'all options' if options else 'plain'})")
+
+
+def pin_backward_finite_differences(orc, seed=18):
+    """The backward oracle (reverse-mode chain rule through softplus, the
+    exp(Delta A) transition, the Delta B x input, the C readout, the D skip
+    and the silu gate) against central finite differences of the forward
+    oracle, for every element of every input, with all options on and with
+    none."""
+    rng = np.random.default_rng(seed)
+    _fd_case(orc, rng, True)
+    _fd_case(orc, rng, False)
+
+
 ALL_PINS = [pin_hand_direct, pin_hand_mamba, pin_softplus_values, pin_lti_convolution,
             pin_brute_force, pin_tree_scan, pin_degenerate, pin_skip_and_gate, pin_h0_split,
-            pin_decode, pin_p1_numpy_example, pin_p3_shape_example]
+            pin_decode, pin_p1_numpy_example, pin_p3_shape_example,
+            pin_backward_finite_differences]

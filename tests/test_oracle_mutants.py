@@ -19,6 +19,9 @@ MUTANTS = {
     10: "h0 ignored",
     11: "B, C taken from the previous token",
     12: "elementwise A from the previous token",
+    13: "backward: state gradient not carried through Abar",
+    14: "backward: Delta's input-term gradient dropped",
+    15: "backward: sigmoid in place of the silu derivative",
 }
 
 
