@@ -54,6 +54,8 @@ def parse_args():
     ap.add_argument("--warps", type=int, default=0)
     ap.add_argument("--grid", type=int, default=0)
     ap.add_argument("--tile-t", type=int, default=0)
+    ap.add_argument("--bwd", action="store_true",
+                    help="time the backward pass (ssm_scan_bwd) instead of the forward")
     ap.add_argument("--zoh", action="store_true",
                     help="zero-order-hold input matrix (exp(Delta A) - 1)/A * B instead of Delta * B")
     return ap.parse_args()
@@ -295,10 +297,19 @@ def run_ours(args, rank, world, device):
 
     def step(i):
         s, (y, hl) = sets[i & 1], outs[i & 1]
+        if args.bwd:   # y doubles as dL/dy (any values of the output dtype)
+            plan.bwd(s["x"], s["delta"], s["A"], s["B"], s["C"], y, D=s["D"], z=s["z"],
+                     delta_bias=s["delta_bias"], h0=s["h0"], dh_last=hl)
+            return
         plan.fwd(s["x"], s["delta"], s["A"], s["B"], s["C"], D=s["D"], z=s["z"],
                  delta_bias=s["delta_bias"], h0=s["h0"], y=y, h_last=hl)
 
     stream = torch.cuda.current_stream(device)
+    if args.bwd:   # real outputs as dL/dy
+        for i in range(2):
+            s, (y, hl) = sets[i], outs[i]
+            plan.fwd(s["x"], s["delta"], s["A"], s["B"], s["C"], D=s["D"], z=s["z"],
+                     delta_bias=s["delta_bias"], h0=s["h0"], y=y, h_last=hl)
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize(device)
@@ -332,11 +343,15 @@ def run_ours(args, rank, world, device):
     ms_per_step = total_ms / K
 
     counts = algorithmic_counts(inp)
+    if args.bwd:
+        # the backward evaluates every exp three times: checkpoint pass, chunk
+        # recomputation and the reverse walk
+        counts["mufu"] *= 3
     value = replica_throughput(counts["updates"], world, ms_per_step)
 
     # e2e through the public API: pinned host inputs copied in, y/h_last copied out
     e2e = None
-    if args.e2e_steps > 0:
+    if args.e2e_steps > 0 and not args.bwd:
         def pinned(a, dt):
             return None if a is None else torch.from_numpy(np.ascontiguousarray(a)).to(dt).pin_memory()
         host = dict(x=pinned(inp.x, tdt[inp.in_dtype]), delta=pinned(inp.delta, tdt[inp.in_dtype]),
@@ -409,6 +424,7 @@ def run_ours(args, rank, world, device):
                    "dstate": inp.N, "in_dtype": inp.in_dtype, "out_dtype": inp.out_dtype,
                    "state_dtype": "f32", "gate": inp.z is not None, "h0": inp.h0 is not None,
                    "discretisation": "zoh" if inp.zoh else "delta_B",
+                   "pass": "backward" if args.bwd else "forward",
                    "l2": "two input sets alternate between steps (2x inputs > 126 MB L2)",
                    "parallelism": f"replicas x{world}",
                    "launch": {k: info[k] for k in ("lanes_per_chan", "warps_per_cta",
@@ -429,7 +445,7 @@ def run_ours(args, rank, world, device):
         result["roofline"]["frac_at_sampled_clock"] = achieved_mufu / (
             MUFU_PER_CLK_PER_SM * NOMINAL_SMS * clocks["sm_mhz"] * 1e6)
 
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.bwd:
         rate, cores, desc, _ = oracle_sample_rate(inp, args.cpu_budget_s)
         result["cpu_baseline"] = {"value": rate, "unit": "state-updates/s", "cores": cores,
                                   "kind": "oracle", "sample": desc}

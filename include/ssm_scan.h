@@ -155,6 +155,28 @@ SSM_API ssm_status ssm_scan_fwd(ssm_scan_plan *plan, const void *x, const void *
                         const void *C, const float *D, const void *z,
                         const float *h0, void *y, float *h_last, ssm_stream_t stream);
 
+/* Backward pass of ssm_scan_fwd (Delta*B input coefficient; plans with
+ * SSM_ZOH or SSM_A_DIRECT get SSM_ERR_UNSUPPORTED): gradients of a loss
+ * with dL/dy = dy ((batch, seqlen, dim), out_dtype) and dL/dh_last = dh_last
+ * ((batch, dim, dstate) fp32, NULL for 0).  The inputs are the forward
+ * call's (same pointers, same flags).  Every gradient is fp32 with its
+ * input's shape: dx, ddelta, dz (batch, seqlen, dim); dB, dC
+ * (batch, seqlen, dstate); dA (dim, dstate); dD, ddelta_bias (dim); dh0
+ * (batch, dim, dstate).  dz, dD, ddelta_bias must be non-NULL exactly when
+ * SSM_HAS_Z, SSM_HAS_D, SSM_HAS_DELTA_BIAS are set; dh0 may be NULL.  The
+ * accumulated gradients (dB, dC, dA, dD, ddelta_bias) are overwritten, not
+ * added to.  States are recomputed from per-chunk checkpoints rather than
+ * stored ("Tai sao chi parallel scan van chua du nhanh?"); the first call on
+ * a plan allocates the checkpoint workspace (batch*dim*ceil(seqlen/16)*dstate
+ * floats) and may return SSM_ERR_OOM.  Summation order of dB, dC, dA, dD and
+ * ddelta_bias follows atomics, so those are reproducible to rounding only. */
+SSM_API ssm_status ssm_scan_bwd(ssm_scan_plan *plan, const void *x, const void *delta,
+                        const float *delta_bias, const float *A, const void *B,
+                        const void *C, const float *D, const void *z, const float *h0,
+                        const void *dy, const float *dh_last, float *dx, float *ddelta,
+                        float *ddelta_bias, float *dA, float *dB, float *dC, float *dD,
+                        float *dz, float *dh0, ssm_stream_t stream);
+
 /* One decode step per the pages' inference section: reads `state`
  * (batch, dim, dstate), applies one token, writes it back and writes y
  * (batch, dim).  desc.seqlen is ignored; SSM_HAS_H0 / SSM_WANT_HLAST /

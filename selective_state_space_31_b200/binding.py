@@ -81,6 +81,8 @@ def load_library(path: str | None = None):
         lib.ssm_scan_fwd.restype = st
         lib.ssm_scan_step.argtypes = [_vp] * 12
         lib.ssm_scan_step.restype = st
+        lib.ssm_scan_bwd.argtypes = [_vp] * 22
+        lib.ssm_scan_bwd.restype = st
         lib.ssm_scan_get_status.argtypes = [_vp]
         lib.ssm_scan_get_status.restype = st
         lib.ssm_scan_get_info.argtypes = [_vp, ctypes.POINTER(Info)]
@@ -208,6 +210,45 @@ class Plan:
                                     _ptr(h_last), _stream(dev))
         _check(rc, "ssm_scan_fwd")
         return y, h_last
+
+    def bwd(self, x, delta, A, B, C, dy, D=None, z=None, delta_bias=None, h0=None,
+            dh_last=None, want_dh0=True):
+        """Gradients of the forward pass for dL/dy = dy (out dtype) and
+        dL/dh_last = dh_last (fp32, or None for 0).  Returns a dict of fp32
+        tensors keyed like the inputs (x, delta, A, B, C, and D, z,
+        delta_bias, h0 where present)."""
+        d, f, dev = self.desc, self.flags, self.device
+        Bz, L, Dm, N = d.batch, d.seqlen, d.dim, d.dstate
+        for name, t in (("x", x), ("delta", delta), ("z", z)):
+            _need(t, name, (Bz, L, Dm), self.in_dtype, dev)
+        _need(B, "B", (Bz, L, N), self.in_dtype, dev)
+        _need(C, "C", (Bz, L, N), self.in_dtype, dev)
+        _need(A, "A", (Dm, N), torch.float32, dev)
+        _need(D, "D", (Dm,), torch.float32, dev)
+        _need(delta_bias, "delta_bias", (Dm,), torch.float32, dev)
+        _need(h0, "h0", (Bz, Dm, N), torch.float32, dev)
+        _need(dy, "dy", (Bz, L, Dm), self.out_dtype, dev)
+        _need(dh_last, "dh_last", (Bz, Dm, N), torch.float32, dev)
+        f32 = dict(dtype=torch.float32, device=dev)
+        g = {"x": torch.empty((Bz, L, Dm), **f32), "delta": torch.empty((Bz, L, Dm), **f32),
+             "A": torch.empty((Dm, N), **f32), "B": torch.empty((Bz, L, N), **f32),
+             "C": torch.empty((Bz, L, N), **f32)}
+        if D is not None:
+            g["D"] = torch.empty((Dm,), **f32)
+        if z is not None:
+            g["z"] = torch.empty((Bz, L, Dm), **f32)
+        if delta_bias is not None:
+            g["delta_bias"] = torch.empty((Dm,), **f32)
+        if want_dh0:
+            g["h0"] = torch.empty((Bz, Dm, N), **f32)
+        rc = self._lib.ssm_scan_bwd(self._h, _ptr(x), _ptr(delta), _ptr(delta_bias), _ptr(A),
+                                    _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(h0), _ptr(dy),
+                                    _ptr(dh_last), _ptr(g["x"]), _ptr(g["delta"]),
+                                    _ptr(g.get("delta_bias")), _ptr(g["A"]), _ptr(g["B"]),
+                                    _ptr(g["C"]), _ptr(g.get("D")), _ptr(g.get("z")),
+                                    _ptr(g.get("h0")), _stream(dev))
+        _check(rc, "ssm_scan_bwd")
+        return g
 
     def step(self, state, x, delta, A, B, C, D=None, z=None, delta_bias=None, y=None):
         d, dev = self.desc, self.device

@@ -85,6 +85,8 @@ struct ssm_scan_plan {
   ssm_scan_config cfg{};  // user overrides
   ssm::Control *ctl = nullptr;
   int ring = 0;  // stage slots of the fused kernel's TMA ring
+  float *ws_ck = nullptr;  // backward checkpoints (allocated by the first ssm_scan_bwd)
+  size_t ws_ck_bytes = 0;
   float *ws_state = nullptr;
   unsigned long long *ws_flags = nullptr;
   size_t ws_state_bytes = 0, ws_flag_bytes = 0;
@@ -249,6 +251,7 @@ ssm_status ssm_scan_destroy(ssm_scan_plan *pl) {
     DeviceGuard guard(pl->device);
     cudaDeviceSynchronize();
     if (pl->ctl) cudaFree(pl->ctl);
+    if (pl->ws_ck) cudaFree(pl->ws_ck);
     if (pl->ws_state) cudaFree(pl->ws_state);
     if (pl->ws_flags) cudaFree(pl->ws_flags);
   }
@@ -404,6 +407,61 @@ ssm_status ssm_scan_fwd(ssm_scan_plan *pl, const void *x, const void *delta,
   p.A = static_cast<const float *>(A);
   p.Dv = D; p.bias = delta_bias; p.h0 = h0; p.y = y; p.h_last = h_last;
   return map_cuda(ssm::launch_fwd_general(p, stream));
+}
+
+ssm_status ssm_scan_bwd(ssm_scan_plan *pl, const void *x, const void *delta,
+                        const float *delta_bias, const float *A, const void *B, const void *C,
+                        const float *D, const void *z, const float *h0, const void *dy,
+                        const float *dh_last, float *dx, float *ddelta, float *ddelta_bias,
+                        float *dA, float *dB, float *dC, float *dD, float *dz, float *dh0,
+                        ssm_stream_t stream_) {
+  if (!pl) return SSM_ERR_INVALID_ARG;
+  const ssm_scan_desc &d = pl->desc;
+  const uint32_t f = d.flags;
+  if (f & (SSM_ZOH | SSM_A_DIRECT)) return SSM_ERR_UNSUPPORTED;
+  const bool has_tokens = d.batch * d.seqlen * d.dim != 0;
+  const bool has_chans = d.batch * d.dim != 0;
+  if (has_tokens && (!x || !delta || !B || !C || !dy || !dx || !ddelta || !dB || !dC))
+    return SSM_ERR_INVALID_ARG;
+  if (d.dim != 0 && (!A || !dA)) return SSM_ERR_INVALID_ARG;
+  if (has_tokens && (((f & SSM_HAS_Z) != 0) != (z != nullptr) ||
+                     ((f & SSM_HAS_Z) != 0) != (dz != nullptr)))
+    return SSM_ERR_INVALID_ARG;
+  if (d.dim != 0 && (((f & SSM_HAS_D) != 0) != (D != nullptr) ||
+                     ((f & SSM_HAS_D) != 0) != (dD != nullptr) ||
+                     ((f & SSM_HAS_DELTA_BIAS) != 0) != (delta_bias != nullptr) ||
+                     ((f & SSM_HAS_DELTA_BIAS) != 0) != (ddelta_bias != nullptr)))
+    return SSM_ERR_INVALID_ARG;
+  if (has_chans && ((f & SSM_HAS_H0) != 0) != (h0 != nullptr)) return SSM_ERR_INVALID_ARG;
+  if (d.dim == 0) return SSM_OK;
+  DeviceGuard guard(pl->device);
+  if (!guard.ok) return SSM_ERR_CUDA;
+  const int64_t nck = (d.seqlen + ssm::kBwdChunk - 1) / ssm::kBwdChunk;
+  const size_t need = (size_t)(d.batch * d.dim * nck * d.dstate) * sizeof(float);
+  if (need > pl->ws_ck_bytes) {
+    if (pl->ws_ck) cudaFree(pl->ws_ck);
+    pl->ws_ck = nullptr;
+    pl->ws_ck_bytes = 0;
+    if (cudaMalloc(&pl->ws_ck, need) != cudaSuccess) {
+      cudaGetLastError();
+      return SSM_ERR_OOM;
+    }
+    pl->ws_ck_bytes = need;
+  }
+  ssm::BwdParams p{};
+  p.Bsz = (int)d.batch; p.L = (int)d.seqlen; p.D = (int)d.dim; p.N = (int)d.dstate;
+  p.softplus = f & SSM_DELTA_SOFTPLUS;
+  p.has_z = f & SSM_HAS_Z;
+  p.has_D = f & SSM_HAS_D;
+  p.has_bias = f & SSM_HAS_DELTA_BIAS;
+  p.has_h0 = f & SSM_HAS_H0;
+  p.in_bf16 = d.in_dtype == SSM_BF16;
+  p.out_bf16 = d.out_dtype == SSM_BF16;
+  p.x = x; p.dt = delta; p.z = z; p.B = B; p.C = C; p.dy = dy;
+  p.A = A; p.Dv = D; p.bias = delta_bias; p.h0 = h0; p.dh_last = dh_last;
+  p.dx = dx; p.ddelta = ddelta; p.dz = dz; p.dB = dB; p.dC = dC; p.dA = dA; p.dD = dD;
+  p.dbias = ddelta_bias; p.dh0 = dh0; p.ws_ck = pl->ws_ck;
+  return map_cuda(ssm::launch_bwd(p, reinterpret_cast<cudaStream_t>(stream_)));
 }
 
 ssm_status ssm_scan_step(ssm_scan_plan *pl, const void *x, const void *delta,
