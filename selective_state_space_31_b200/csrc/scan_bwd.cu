@@ -16,7 +16,7 @@
 // of the backward: it costs three exps per state update (forward pass,
 // recomputation, reverse) and keeps the chunk's states in local memory.
 #include "device_common.cuh"
-#include "scan_params.h"
+#include "scan_bwd.h"
 
 namespace ssm {
 

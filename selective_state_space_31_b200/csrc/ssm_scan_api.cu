@@ -14,6 +14,7 @@
 
 #include "ssm_scan.h"
 #include "scan_params.h"
+#include "scan_bwd.h"
 
 namespace {
 
