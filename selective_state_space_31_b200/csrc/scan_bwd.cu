@@ -26,7 +26,7 @@ __device__ __forceinline__ float ldb(const void *base, size_t i) {
 }
 
 template <typename InT, typename GradT, int NMAX, int K>
-__global__ void __launch_bounds__(128) bwd_kernel(const BwdParams p) {
+__global__ void __launch_bounds__(32) bwd_kernel(const BwdParams p) {
   const long long chn = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (chn >= (long long)p.Bsz * p.D) return;
   const int b = (int)(chn / p.D), d = (int)(chn % p.D);
@@ -139,13 +139,17 @@ __global__ void __launch_bounds__(128) bwd_kernel(const BwdParams p) {
   if (p.has_bias) atomicAdd(p.dbias + d, dbias_acc);
 }
 
+// One warp per CTA: a layer has only B*D channels (12288 for the 130M
+// layer), so small CTAs spread them over every SM.
+constexpr int kBwdThreads = 32;
+
 template <typename InT, typename GradT>
 static cudaError_t bwd_by_n(const BwdParams &p, cudaStream_t stream) {
   const long long chans = (long long)p.Bsz * p.D;
-  const unsigned grid = (unsigned)((chans + 127) / 128);
-  if (p.N <= 4) bwd_kernel<InT, GradT, 4, kBwdChunk><<<grid, 128, 0, stream>>>(p);
-  else if (p.N <= 16) bwd_kernel<InT, GradT, 16, kBwdChunk><<<grid, 128, 0, stream>>>(p);
-  else bwd_kernel<InT, GradT, 64, kBwdChunk><<<grid, 128, 0, stream>>>(p);
+  const unsigned grid = (unsigned)((chans + kBwdThreads - 1) / kBwdThreads);
+  if (p.N <= 4) bwd_kernel<InT, GradT, 4, kBwdChunk><<<grid, kBwdThreads, 0, stream>>>(p);
+  else if (p.N <= 16) bwd_kernel<InT, GradT, 16, kBwdChunk><<<grid, kBwdThreads, 0, stream>>>(p);
+  else bwd_kernel<InT, GradT, 64, kBwdChunk><<<grid, kBwdThreads, 0, stream>>>(p);
   return cudaGetLastError();
 }
 
