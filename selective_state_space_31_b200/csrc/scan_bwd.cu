@@ -4,7 +4,7 @@
 // the pages' third pillar, recomputation instead of storing the (B, L, D, N)
 // states, "Tai sao chi parallel scan van chua du nhanh?").
 //
-// One thread owns one channel (b, d) and all of its N states.  Pass 1 runs
+// Four lanes share one channel (b, d) and split its N states.  Pass 1 runs
 // the recurrence forward and checkpoints the state at the start of every
 // chunk of K tokens (the only state written to HBM: B*D*ceil(L/K)*N floats).
 // Pass 2 walks the chunks backwards: it recomputes the chunk's K + 1 states
@@ -25,131 +25,159 @@ __device__ __forceinline__ float ldb(const void *base, size_t i) {
   return to_f32(reinterpret_cast<const T *>(base)[i]);
 }
 
-template <typename InT, typename GradT, int NMAX, int K>
-__global__ void __launch_bounds__(32) bwd_kernel(const BwdParams p) {
-  const long long chn = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (chn >= (long long)p.Bsz * p.D) return;
-  const int b = (int)(chn / p.D), d = (int)(chn % p.D);
+// Sum over the TPC lanes that share a channel (xor butterfly; every lane of
+// the group ends with the total).
+template <int TPC>
+__device__ __forceinline__ float group_sum(float v) {
+#pragma unroll
+  for (int m = TPC / 2; m >= 1; m >>= 1) v += __shfl_xor_sync(FULL_MASK, v, m);
+  return v;
+}
+
+template <typename InT, typename GradT, int NPL, int TPC, int K>
+__global__ void __launch_bounds__(128) bwd_kernel(const BwdParams p) {
+  // TPC lanes per channel, lane q owns states q*NPL .. q*NPL + NPL-1; lanes
+  // past the last channel run along (they take part in the shuffles) but
+  // touch no memory
+  const long long gt = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long chn = gt / TPC;
+  const int q = (int)(gt % TPC);
+  const bool active = chn < (long long)p.Bsz * p.D;
+  const int b = active ? (int)(chn / p.D) : 0, d = active ? (int)(chn % p.D) : 0;
   const int N = p.N, L = p.L;
   const int nck = (L + K - 1) / K;
-  float A2[NMAX], An[NMAX], h[NMAX];
+  float A2[NPL], An[NPL], h[NPL];
+  bool on[NPL];
 #pragma unroll
-  for (int n = 0; n < NMAX; ++n) {
-    const bool on = n < N;
-    An[n] = on ? p.A[(size_t)d * N + n] : 0.f;
-    A2[n] = An[n] * kLog2e;
-    h[n] = (on && p.has_h0) ? p.h0[((size_t)b * p.D + d) * N + n] : 0.f;
+  for (int i = 0; i < NPL; ++i) {
+    const int n = q * NPL + i;
+    on[i] = active && n < N;
+    An[i] = on[i] ? p.A[(size_t)d * N + n] : 0.f;
+    A2[i] = An[i] * kLog2e;
+    h[i] = (on[i] && p.has_h0) ? p.h0[((size_t)b * p.D + d) * N + n] : 0.f;
   }
-  const float Dd = p.has_D ? p.Dv[d] : 0.f;
-  const float bias = p.has_bias ? p.bias[d] : 0.f;
-  float *ck = p.ws_ck + (size_t)chn * nck * N;
+  const float Dd = (active && p.has_D) ? p.Dv[d] : 0.f;
+  const float bias = (active && p.has_bias) ? p.bias[d] : 0.f;
+  float *ck = p.ws_ck + (size_t)(active ? chn : 0) * nck * N + q * NPL;
   auto delta_of = [&](float v) { return p.softplus ? softplus_f(v) : v; };
+  auto idx = [&](int t) { return ((size_t)b * L + t) * p.D + d; };
+  auto tok = [&](int t) { return ((size_t)b * L + t) * N + q * NPL; };
 
   // pass 1: forward with a checkpoint at the start of every chunk
   for (int c = 0; c < nck; ++c) {
 #pragma unroll
-    for (int n = 0; n < NMAX; ++n)
-      if (n < N) ck[(size_t)c * N + n] = h[n];
+    for (int i = 0; i < NPL; ++i)
+      if (on[i]) ck[(size_t)c * N + i] = h[i];
     const int t1 = min(L, (c + 1) * K);
-    for (int t = c * K; t < t1; ++t) {
-      const size_t i = ((size_t)b * L + t) * p.D + d, j = ((size_t)b * L + t) * N;
-      const float xv = ldb<InT>(p.x, i);
-      const float dt = delta_of(ldb<InT>(p.dt, i) + bias);
+    if (active) {
+      for (int t = c * K; t < t1; ++t) {
+        const float xv = ldb<InT>(p.x, idx(t));
+        const float dt = delta_of(ldb<InT>(p.dt, idx(t)) + bias);
 #pragma unroll
-      for (int n = 0; n < NMAX; ++n)
-        if (n < N) h[n] = fmaf(ex2_approx(dt * A2[n]), h[n], dt * ldb<InT>(p.B, j + n) * xv);
+        for (int i = 0; i < NPL; ++i)
+          if (on[i]) h[i] = fmaf(ex2_approx(dt * A2[i]), h[i], dt * ldb<InT>(p.B, tok(t) + i) * xv);
+      }
     }
   }
 
   // pass 2: chunks from the last, tokens from the chunk's end
-  float g[NMAX], dA_acc[NMAX];
+  float g[NPL], dA_acc[NPL];
 #pragma unroll
-  for (int n = 0; n < NMAX; ++n) {
-    g[n] = (n < N && p.dh_last) ? p.dh_last[((size_t)b * p.D + d) * N + n] : 0.f;
-    dA_acc[n] = 0.f;
+  for (int i = 0; i < NPL; ++i) {
+    g[i] = (on[i] && p.dh_last) ? p.dh_last[((size_t)b * p.D + d) * N + q * NPL + i] : 0.f;
+    dA_acc[i] = 0.f;
   }
   float dD_acc = 0.f, dbias_acc = 0.f;
-  float hs[K + 1][NMAX];  // states h_{t0} .. h_{t1} of the chunk
+  float hs[K + 1][NPL];  // this lane's states h_{t0} .. h_{t1} of the chunk
   for (int c = nck - 1; c >= 0; --c) {
     const int t0 = c * K, t1 = min(L, t0 + K);
 #pragma unroll
-    for (int n = 0; n < NMAX; ++n) hs[0][n] = n < N ? ck[(size_t)c * N + n] : 0.f;
+    for (int i = 0; i < NPL; ++i) hs[0][i] = on[i] ? ck[(size_t)c * N + i] : 0.f;
     for (int t = t0; t < t1; ++t) {
-      const size_t i = ((size_t)b * L + t) * p.D + d, j = ((size_t)b * L + t) * N;
-      const float xv = ldb<InT>(p.x, i);
-      const float dt = delta_of(ldb<InT>(p.dt, i) + bias);
       const int k = t - t0;
+      const float xv = active ? ldb<InT>(p.x, idx(t)) : 0.f;
+      const float dt = active ? delta_of(ldb<InT>(p.dt, idx(t)) + bias) : 0.f;
 #pragma unroll
-      for (int n = 0; n < NMAX; ++n)
-        hs[k + 1][n] = n < N ? fmaf(ex2_approx(dt * A2[n]), hs[k][n],
-                                    dt * ldb<InT>(p.B, j + n) * xv)
+      for (int i = 0; i < NPL; ++i)
+        hs[k + 1][i] = on[i] ? fmaf(ex2_approx(dt * A2[i]), hs[k][i],
+                                    dt * ldb<InT>(p.B, tok(t) + i) * xv)
                              : 0.f;
     }
     for (int t = t1 - 1; t >= t0; --t) {
-      const size_t i = ((size_t)b * L + t) * p.D + d, j = ((size_t)b * L + t) * N;
       const int k = t - t0;
-      const float xv = ldb<InT>(p.x, i);
-      const float v = ldb<InT>(p.dt, i) + bias;
+      const size_t i0 = idx(t), j = tok(t);
+      const float xv = active ? ldb<InT>(p.x, i0) : 0.f;
+      const float v = active ? ldb<InT>(p.dt, i0) + bias : 0.f;
       const float dt = delta_of(v);
-      float s = Dd * xv;
+      float sp = 0.f;
 #pragma unroll
-      for (int n = 0; n < NMAX; ++n)
-        if (n < N) s = fmaf(ldb<InT>(p.C, j + n), hs[k + 1][n], s);
-      const float dyv = ldb<GradT>(p.dy, i);
+      for (int i = 0; i < NPL; ++i)
+        if (on[i]) sp = fmaf(ldb<InT>(p.C, j + i), hs[k + 1][i], sp);
+      const float s = group_sum<TPC>(sp) + Dd * xv;
+      const float dyv = active ? ldb<GradT>(p.dy, i0) : 0.f;
       float ds = dyv;
       if (p.has_z) {
-        const float zv = ldb<InT>(p.z, i);
+        const float zv = active ? ldb<InT>(p.z, i0) : 0.f;
         const float sig = __fdividef(1.f, 1.f + __expf(-zv));
-        ds = dyv * zv * sig;                                      // dy * silu(z)
-        p.dz[i] = dyv * s * sig * fmaf(zv, 1.f - sig, 1.f);       // dy * s * silu'(z)
+        ds = dyv * zv * sig;                                          // dy * silu(z)
+        if (active && q == 0) p.dz[i0] = dyv * s * sig * fmaf(zv, 1.f - sig, 1.f);
       }
-      float dxi = ds * Dd;
       dD_acc = fmaf(ds, xv, dD_acc);
-      float ddt = 0.f;
+      float dxp = 0.f, ddtp = 0.f;
 #pragma unroll
-      for (int n = 0; n < NMAX; ++n) {
-        if (n < N) {
-          const float Cn = ldb<InT>(p.C, j + n), Bn = ldb<InT>(p.B, j + n);
-          const float abar = ex2_approx(dt * A2[n]);
-          atomicAdd(p.dC + j + n, ds * hs[k + 1][n]);
-          g[n] = fmaf(ds, Cn, g[n]);
-          const float dabar = g[n] * hs[k][n];
-          ddt += dabar * abar * An[n] + g[n] * Bn * xv;
-          dA_acc[n] = fmaf(dabar * abar, dt, dA_acc[n]);
-          atomicAdd(p.dB + j + n, g[n] * dt * xv);
-          dxi = fmaf(g[n] * dt, Bn, dxi);
-          g[n] *= abar;
+      for (int i = 0; i < NPL; ++i) {
+        if (on[i]) {
+          const float Cn = ldb<InT>(p.C, j + i), Bn = ldb<InT>(p.B, j + i);
+          const float abar = ex2_approx(dt * A2[i]);
+          atomicAdd(p.dC + j + i, ds * hs[k + 1][i]);
+          g[i] = fmaf(ds, Cn, g[i]);
+          const float dabar = g[i] * hs[k][i];
+          ddtp += dabar * abar * An[i] + g[i] * Bn * xv;
+          dA_acc[i] = fmaf(dabar * abar, dt, dA_acc[i]);
+          atomicAdd(p.dB + j + i, g[i] * dt * xv);
+          dxp = fmaf(g[i] * dt, Bn, dxp);
+          g[i] *= abar;
         }
       }
-      p.dx[i] = dxi;
+      const float dxi = group_sum<TPC>(dxp) + ds * Dd;
+      const float ddt = group_sum<TPC>(ddtp);
       const float dv = p.softplus ? ddt * __fdividef(1.f, 1.f + __expf(-v)) : ddt;
-      p.ddelta[i] = dv;
       dbias_acc += dv;
+      if (active && q == 0) {
+        p.dx[i0] = dxi;
+        p.ddelta[i0] = dv;
+      }
     }
   }
   if (p.dh0) {
 #pragma unroll
-    for (int n = 0; n < NMAX; ++n)
-      if (n < N) p.dh0[((size_t)b * p.D + d) * N + n] = g[n];
+    for (int i = 0; i < NPL; ++i)
+      if (on[i]) p.dh0[((size_t)b * p.D + d) * N + q * NPL + i] = g[i];
   }
 #pragma unroll
-  for (int n = 0; n < NMAX; ++n)
-    if (n < N) atomicAdd(p.dA + (size_t)d * N + n, dA_acc[n]);
-  if (p.has_D) atomicAdd(p.dD + d, dD_acc);
-  if (p.has_bias) atomicAdd(p.dbias + d, dbias_acc);
+  for (int i = 0; i < NPL; ++i)
+    if (on[i]) atomicAdd(p.dA + (size_t)d * N + q * NPL + i, dA_acc[i]);
+  if (active && q == 0) {
+    if (p.has_D) atomicAdd(p.dD + d, dD_acc);
+    if (p.has_bias) atomicAdd(p.dbias + d, dbias_acc);
+  }
 }
 
-// One warp per CTA: a layer has only B*D channels (12288 for the 130M
-// layer), so small CTAs spread them over every SM.
-constexpr int kBwdThreads = 32;
+template <typename InT, typename GradT, int NPL, int TPC>
+static void launch_bwd_variant(const BwdParams &p, cudaStream_t stream) {
+  const long long threads = (long long)p.Bsz * p.D * TPC;
+  bwd_kernel<InT, GradT, NPL, TPC, kBwdChunk>
+      <<<(unsigned)((threads + 127) / 128), 128, 0, stream>>>(p);
+}
 
+// Four lanes per channel (N <= 16: up to 4 states each; larger N: 16 each),
+// so a layer's B*D channels fill the SMs four times as densely as one
+// thread per channel.
 template <typename InT, typename GradT>
 static cudaError_t bwd_by_n(const BwdParams &p, cudaStream_t stream) {
-  const long long chans = (long long)p.Bsz * p.D;
-  const unsigned grid = (unsigned)((chans + kBwdThreads - 1) / kBwdThreads);
-  if (p.N <= 4) bwd_kernel<InT, GradT, 4, kBwdChunk><<<grid, kBwdThreads, 0, stream>>>(p);
-  else if (p.N <= 16) bwd_kernel<InT, GradT, 16, kBwdChunk><<<grid, kBwdThreads, 0, stream>>>(p);
-  else bwd_kernel<InT, GradT, 64, kBwdChunk><<<grid, kBwdThreads, 0, stream>>>(p);
+  if (p.N <= 4) launch_bwd_variant<InT, GradT, 1, 4>(p, stream);
+  else if (p.N <= 16) launch_bwd_variant<InT, GradT, 4, 4>(p, stream);
+  else launch_bwd_variant<InT, GradT, 16, 4>(p, stream);
   return cudaGetLastError();
 }
 
