@@ -35,3 +35,28 @@ def test_reference_arm_prints_one_json_line():
     assert out["impl"] == "reference" and out["value"] > 0
     assert out["cpu_baseline"]["kind"] == "oracle" and out["cpu_baseline"]["cores"] >= 1
     assert out["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_reference_arm_with_zero_order_hold():
+    """--zoh reaches the oracle: its rate is measured on the zero-order-hold
+    recurrence (a different program than the default's)."""
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "tiny_fp32", "--steps", "1", "--warmup", "0", "--zoh",
+                        "--cpu-budget-s", "0.3"], capture_output=True, text=True, timeout=600,
+                       cwd=ROOT)
+    assert r.returncode == 0, r.stderr
+    out = json.loads([l for l in r.stdout.splitlines() if l.strip()][0])
+    assert out["impl"] == "reference" and out["value"] > 0
+
+
+def test_cli_flags():
+    sys.path.insert(0, ROOT)
+    import bench
+    argv = sys.argv
+    try:
+        sys.argv = ["bench.py", "--bwd", "--zoh", "--workload", "mamba1p4b_layer"]
+        a = bench.parse_args()
+    finally:
+        sys.argv = argv
+    assert a.bwd and a.zoh and a.workload == "mamba1p4b_layer" and a.gpus == 1
+    assert a.warmup >= 3
