@@ -45,8 +45,12 @@ def _stale(out: str, deps: list[str]) -> bool:
 
 
 def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
-    os.makedirs(BUILD, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+    # a library newer than every source is current even where the object
+    # files were not kept (a copy of the tree without _build/)
+    if not force and not extra and not _stale(LIB, [d for s in srcs for d in _deps(s)]):
+        return LIB
+    os.makedirs(BUILD, exist_ok=True)
     objs = [os.path.join(BUILD, os.path.basename(s)[:-3] + ".o") for s in srcs]
     extra = list(extra or [])
     todo = [(s, o) for s, o in zip(srcs, objs) if force or _stale(o, _deps(s))]
