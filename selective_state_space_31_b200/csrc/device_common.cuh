@@ -217,7 +217,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
   }
 }
 
-// --- TMA (cp.async.bulk.tensor), no multicast -------------------------------
+// --- TMA (cp.async.bulk.tensor) into this CTA's own shared memory ----------
 
 __device__ __forceinline__ void tma_load_3d(void *smem_dst, const void *tmap, uint64_t *bar,
                                             int c0, int c1, int c2) {

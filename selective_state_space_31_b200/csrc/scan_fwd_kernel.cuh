@@ -29,17 +29,17 @@
 //     wait is bounded by a timer.
 //   * One load warp streams the stages' [TT, DT] tiles of x / delta / z and
 //     [TT, N] tiles of B / C into a ring of RAW shared-memory slots with TMA
-//     (cp.async.bulk.tensor, no multicast); slot full / slot empty mbarriers
-//     are the only coupling between warps.  Each scan warp does all the
-//     per-token work of its own channels: lane q of a channel prepares tokens
-//     q, q + LPC, ... (Delta, Delta*x into a warp-private plane that the
-//     channel's LPC lanes read back; silu(z) and D*x*silu(z) stay in the
-//     registers of the lane that finishes those very tokens), scans, and
-//     stores y straight from registers.  B / C are read as stored (bf16 words
-//     are widened with integer ops), which halves the shared-memory
-//     wavefronts of the scan loop against fp32 staging.  Tokens past the end
-//     get Delta = 0, an identity update, so carried states are exact for
-//     ragged tails.
+//     (cp.async.bulk.tensor, every CTA loads its own tiles); slot full / slot
+//     empty mbarriers are the only coupling between warps.  Each scan warp
+//     does all the per-token work of its own channels: lane q of a channel
+//     prepares tokens q, q + LPC, ... (Delta, Delta*x into a warp-private
+//     plane that the channel's LPC lanes read back; silu(z) and D*x*silu(z)
+//     stay in the registers of the lane that finishes those very tokens),
+//     scans, and stores y straight from registers.  B / C are read as stored
+//     (bf16 words are widened with integer ops), which halves the
+//     shared-memory wavefronts of the scan loop against fp32 staging.
+//     Tokens past the end get Delta = 0, an identity update, so carried
+//     states are exact for ragged tails.
 #pragma once
 
 #include "device_common.cuh"
