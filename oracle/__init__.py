@@ -32,18 +32,24 @@ _dp = ctypes.POINTER(ctypes.c_double)
 _build_lock = threading.Lock()
 
 
-def lib_path(mutant: int = 0) -> str:
+def lib_path(mutant: int = 0, fp32: bool = False) -> str:
+    if fp32:
+        return os.path.join(_HERE, "libssm_oracle_fp32.so")
     name = "libssm_oracle.so" if mutant == 0 else f"libssm_oracle_mutant{mutant}.so"
     return os.path.join(_HERE, name)
 
 
-def build(mutant: int = 0, force: bool = False) -> str:
-    """Compile the oracle (optionally with one planted mistake) with gcc."""
-    out = lib_path(mutant)
+def build(mutant: int = 0, force: bool = False, fp32: bool = False) -> str:
+    """Compile the oracle (optionally with one planted mistake) with gcc.
+    ``fp32`` builds the single-precision-accumulate forward loop used only as
+    a timed CPU baseline (never for parity)."""
+    out = lib_path(mutant, fp32)
     with _build_lock:
         if force or not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(_SRC):
-            cmd = ["gcc", "-O2", "-std=c99", "-fPIC", "-shared", f"-DORACLE_MUTANT={mutant}",
-                   "-o", out + ".tmp", _SRC, "-lm"]
+            cmd = ["gcc", "-O2", "-std=c99", "-fPIC", "-shared", f"-DORACLE_MUTANT={mutant}"]
+            if fp32:
+                cmd.append("-DORACLE_FP32")
+            cmd += ["-o", out + ".tmp", _SRC, "-lm"]
             subprocess.check_call(cmd)
             os.replace(out + ".tmp", out)
     return out
@@ -65,22 +71,24 @@ def _ptr(a):
 class Oracle:
     """ctypes front end of one compiled oracle build."""
 
-    def __init__(self, mutant: int = 0):
-        self.mutant = mutant
-        self._lib = ctypes.CDLL(build(mutant))
+    def __init__(self, mutant: int = 0, fp32: bool = False):
+        self.mutant, self.fp32 = mutant, fp32
+        self._lib = ctypes.CDLL(build(mutant, fp32=fp32))
         i64, u32 = ctypes.c_int64, ctypes.c_uint32
         self._lib.ssm_oracle_fwd.argtypes = [i64, i64, i64, i64, u32] + [_dp] * 11
         self._lib.ssm_oracle_fwd.restype = ctypes.c_int
+        self._lib.ssm_oracle_softplus.argtypes = [ctypes.c_double]
+        self._lib.ssm_oracle_softplus.restype = ctypes.c_double
+        self._lib.ssm_oracle_silu.argtypes = [ctypes.c_double]
+        self._lib.ssm_oracle_silu.restype = ctypes.c_double
+        if fp32:   # the timing build has the forward loop only
+            return
         self._lib.ssm_oracle_step.argtypes = [i64, i64, i64, u32] + [_dp] * 10
         self._lib.ssm_oracle_step.restype = ctypes.c_int
         self._lib.ssm_oracle_direct.argtypes = [i64, i64, i64] + [_dp] * 7
         self._lib.ssm_oracle_direct.restype = ctypes.c_int
         self._lib.ssm_oracle_bwd.argtypes = [i64, i64, i64, i64, u32] + [_dp] * 20
         self._lib.ssm_oracle_bwd.restype = ctypes.c_int
-        self._lib.ssm_oracle_softplus.argtypes = [ctypes.c_double]
-        self._lib.ssm_oracle_softplus.restype = ctypes.c_double
-        self._lib.ssm_oracle_silu.argtypes = [ctypes.c_double]
-        self._lib.ssm_oracle_silu.restype = ctypes.c_double
 
     def softplus(self, v: float) -> float:
         return self._lib.ssm_oracle_softplus(float(v))
@@ -200,6 +208,7 @@ class Oracle:
 
 
 _default = None
+_fp32 = None
 
 
 def get() -> Oracle:
@@ -208,6 +217,55 @@ def get() -> Oracle:
     if _default is None:
         _default = Oracle(0)
     return _default
+
+
+def get_fp32() -> Oracle:
+    """The fp32-accumulate timing build (forward loop only)."""
+    global _fp32
+    if _fp32 is None:
+        _fp32 = Oracle(0, fp32=True)
+    return _fp32
+
+
+def channel_blocks(Bsz: int, D: int, width: int = 64):
+    """Every channel of a (Bsz, ., D) problem as blocks (b, d0, d1) of at
+    most ``width`` channels, batch-major."""
+    return [(b, d0, min(D, d0 + width)) for b in range(Bsz) for d0 in range(0, D, width)]
+
+
+def fwd_blocks(x, delta, A, B, C, blocks, consume, D=None, z=None, delta_bias=None, h0=None,
+               delta_softplus=True, zoh=False, threads=None, oracle: Oracle | None = None):
+    """Run the oracle over channel blocks (b, d0, d1) on a pool of host
+    threads (the C loop runs without the GIL).  Each block is an independent
+    sub-problem (batch 1, channels d0..d1) cut out of the full arrays;
+    ``consume((b, d0, d1), y, h_last)`` receives its float64 results
+    (y: (L, d1-d0), h_last: (d1-d0, N)) on a worker thread.  B and C are
+    converted to float64 once per batch element.  Returns the thread count."""
+    import concurrent.futures as cf
+
+    orc = oracle or get()
+    threads = threads or os.cpu_count() or 1
+    bc = {}
+    for b in sorted({blk[0] for blk in blocks}):
+        bc[b] = (np.ascontiguousarray(np.asarray(B)[b:b + 1], dtype=np.float64),
+                 np.ascontiguousarray(np.asarray(C)[b:b + 1], dtype=np.float64))
+    A = np.asarray(A)
+
+    def one(blk):
+        b, d0, d1 = blk
+        sl = lambda a: None if a is None else np.asarray(a)[b:b + 1, :, d0:d1]
+        Bb, Cb = bc[b]
+        y, hl = orc.fwd(sl(x), sl(delta), A[d0:d1], Bb, Cb,
+                        None if D is None else np.asarray(D)[d0:d1], sl(z),
+                        None if delta_bias is None else np.asarray(delta_bias)[d0:d1],
+                        None if h0 is None else np.asarray(h0)[b:b + 1, d0:d1],
+                        delta_softplus=delta_softplus, zoh=zoh)
+        consume(blk, y[0], hl[0])
+
+    with cf.ThreadPoolExecutor(max_workers=threads) as ex:
+        for f in [ex.submit(one, blk) for blk in blocks]:
+            f.result()
+    return threads
 
 
 def fwd_rows(x, delta, A, B, C, rows, D=None, z=None, delta_bias=None, h0=None,

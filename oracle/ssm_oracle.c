@@ -47,6 +47,18 @@
 #define ORACLE_MUTANT 0
 #endif
 
+/* Arithmetic type of the forward recurrence.  The parity oracle is the
+ * default double build.  ORACLE_FP32 (set only by the CPU-baseline timing
+ * build) compiles the same forward loop with a single-precision state and
+ * accumulator, the "fp32-accumulate" CPU baseline; the other entry points
+ * are left out of that build. */
+#ifdef ORACLE_FP32
+#include <tgmath.h>
+typedef float orc_real;
+#else
+typedef double orc_real;
+#endif
+
 /* Option bits understood by the oracle.  They are the oracle's own
  * definitions; the Python wrapper maps keyword arguments onto them. */
 #define ORC_HAS_Z 1u
@@ -79,26 +91,31 @@ double ssm_oracle_silu(double z) {
  * h[0..N) is updated in place; returns y for this token.  [P1] "Selection
  * ...": Abar_t = exp(Delta_t*A), Bbar_t = Delta_t*B_t (or ZOH), h updated
  * first, readout from the updated state ([P3] step 4). */
-static double token_update(int64_t N, uint32_t flags, double xv, double dv,
+static double token_update(int64_t N, uint32_t flags, double xv_in, double dv,
                            double bias, const double *Arow, const double *Bt,
-                           const double *Ct, double Dd, double zv, double *h) {
-  double v = dv + bias;
-  double dt = (flags & ORC_SOFTPLUS) ? ssm_oracle_softplus(v) : v;
+                           const double *Ct, double Dd, double zv, orc_real *h) {
+  const orc_real xv = (orc_real)xv_in;
+  orc_real v = (orc_real)(dv + bias);
+  orc_real dt = (flags & ORC_SOFTPLUS) ? (orc_real)ssm_oracle_softplus(v) : v;
 #if ORACLE_MUTANT == 7
   dt = (flags & ORC_SOFTPLUS) ? ssm_oracle_softplus(dv) : dv; /* bias dropped */
 #endif
-  double acc = 0.0;
+  orc_real acc = 0.0;
   for (int64_t n = 0; n < N; ++n) {
-    double a = Arow[n];
-    double abar = exp(dt * a);
+    orc_real a = (orc_real)Arow[n];
+    orc_real abar = exp(dt * a);
 #if ORACLE_MUTANT == 1
     abar = exp(-dt * a); /* sign flip */
 #endif
-    double bbar;
+    orc_real bbar;
     if (flags & ORC_ZOH)
-      bbar = (a != 0.0 ? expm1(dt * a) / a : dt) * Bt[n];
+#if ORACLE_MUTANT == 16
+      bbar = (a != 0.0 ? expm1(dt * a) / a : 0.0) * (orc_real)Bt[n]; /* A = 0 limit lost */
+#else
+      bbar = (a != 0.0 ? expm1(dt * a) / a : dt) * (orc_real)Bt[n];
+#endif
     else
-      bbar = dt * Bt[n];
+      bbar = dt * (orc_real)Bt[n];
 #if ORACLE_MUTANT == 2
     acc += Ct[n] * h[n]; /* readout from the state before the update */
 #endif
@@ -110,13 +127,13 @@ static double token_update(int64_t N, uint32_t flags, double xv, double dv,
 #if ORACLE_MUTANT == 9
     acc += Bt[n] * h[n]; /* B used as readout instead of C */
 #else
-    acc += Ct[n] * h[n];
+    acc += (orc_real)Ct[n] * h[n];
 #endif
 #endif
   }
   if (flags & ORC_HAS_D) {
 #if ORACLE_MUTANT != 3
-    acc += Dd * xv;
+    acc += (orc_real)Dd * xv;
 #endif
   }
   if (flags & ORC_HAS_Z) {
@@ -143,12 +160,12 @@ int ssm_oracle_fwd(int64_t Bsz, int64_t L, int64_t D, int64_t N, uint32_t flags,
   if ((flags & ORC_HAS_D) && !Dv) return -1;
   if ((flags & ORC_HAS_BIAS) && !bias) return -1;
   if ((flags & ORC_HAS_H0) && !h0) return -1;
-  double *h = (double *)malloc((size_t)N * sizeof(double));
+  orc_real *h = (orc_real *)malloc((size_t)N * sizeof(orc_real));
   if (!h) return -1;
   for (int64_t b = 0; b < Bsz; ++b) {
     for (int64_t d = 0; d < D; ++d) {
       for (int64_t n = 0; n < N; ++n) {
-        h[n] = (flags & ORC_HAS_H0) ? h0[(b * D + d) * N + n] : 0.0;
+        h[n] = (flags & ORC_HAS_H0) ? (orc_real)h0[(b * D + d) * N + n] : 0.0;
 #if ORACLE_MUTANT == 10
         h[n] = 0.0; /* h0 ignored */
 #endif
@@ -173,6 +190,7 @@ int ssm_oracle_fwd(int64_t Bsz, int64_t L, int64_t D, int64_t N, uint32_t flags,
   return 0;
 }
 
+#ifndef ORACLE_FP32
 /* One decode step ([P1] inference section): state (B, D, N) is read, updated
  * with one token and written back; y is (B, D).  x, delta, z: (B, D);
  * Bm, Cm: (B, N). */
@@ -332,3 +350,4 @@ int ssm_oracle_bwd(int64_t Bsz, int64_t L, int64_t D, int64_t N, uint32_t flags,
   free(g);
   return 0;
 }
+#endif /* ORACLE_FP32 */

@@ -216,6 +216,47 @@ def pin_brute_force(orc, seed=12):
     _close(hl, wh, 1e-10, 1e-12, "brute force h_last (plain)")
 
 
+def pin_zoh_limits(orc, seed=19):
+    """[P1] "Vi du Python" discretises with zero-order hold,
+    Bbar = expm1(Delta A) / A * B.  Its value where A = 0 is the limit
+    Delta * B (expm1(u) / u -> 1), and near A = 0 it is continuous.  Checked
+    with every option on against the brute-force products (whose ZOH
+    coefficient takes numpy's expm1 and the limit by an explicit select):
+    some A entries exactly 0, some at +-1e-8, the rest ordinary negative
+    values; then the exact-zero and the 1e-8 runs must agree to ~1e-8
+    relative (continuity of the coefficient at 0)."""
+    rng = np.random.default_rng(seed)
+    Bsz, L, D, N = 2, 11, 3, 4
+    x = rng.standard_normal((Bsz, L, D))
+    dr = rng.standard_normal((Bsz, L, D)) - 0.5
+    z = rng.standard_normal((Bsz, L, D))
+    Bm = rng.standard_normal((Bsz, L, N))
+    Cm = rng.standard_normal((Bsz, L, N))
+    Dv = rng.standard_normal(D)
+    bias = rng.uniform(-2, 1, size=D)
+    h0 = rng.standard_normal((Bsz, D, N))
+    A = -rng.uniform(0.1, 3.0, size=(D, N))
+    A[0, :] = 0.0                    # a whole channel at the limit
+    A[1, 1] = 0.0
+    A[2, 0], A[2, 3] = 1e-8, -1e-8   # next to it, on both sides
+    y, hl = orc.fwd(x, dr, A, Bm, Cm, D=Dv, z=z, delta_bias=bias, h0=h0, zoh=True)
+    wy, wh = brute_force_fwd(x, dr, A, Bm, Cm, D=Dv, z=z, bias=bias, h0=h0, zoh=True)
+    _close(y, wy, 1e-10, 1e-12, "ZOH brute force y (A = 0 and near 0)")
+    _close(hl, wh, 1e-10, 1e-12, "ZOH brute force h_last (A = 0 and near 0)")
+    # A = 0 on every state: Abar = 1, Bbar = Delta * B, so the ZOH scan equals
+    # the Delta*B scan exactly (same prefix sum)
+    A0 = np.zeros((D, N))
+    yz, hz = orc.fwd(x, dr, A0, Bm, Cm, D=Dv, z=z, delta_bias=bias, h0=h0, zoh=True)
+    yd, hd = orc.fwd(x, dr, A0, Bm, Cm, D=Dv, z=z, delta_bias=bias, h0=h0, zoh=False)
+    _close(yz, yd, 1e-15, 1e-15, "ZOH at A = 0 equals Delta*B")
+    _close(hz, hd, 1e-15, 1e-15, "ZOH h_last at A = 0 equals Delta*B")
+    # continuity: A = +-1e-8 moves the result by O(1e-8) relative only
+    ye, he = orc.fwd(x, dr, np.full((D, N), 1e-8), Bm, Cm, D=Dv, z=z, delta_bias=bias, h0=h0,
+                     zoh=True)
+    _normwise(ye, yz, 1e-6, "ZOH continuity at A = 0 (y)")
+    _normwise(he, hz, 1e-6, "ZOH continuity at A = 0 (h_last)")
+
+
 def compose(prefix, cur):
     """[P1] "Scan bien recurrence ...": T2(T1(h)) = A2 A1 h + A2 b1 + b2, i.e.
     (A2, b2) (x) (A1, b1) = (A2*A1, A2*b1 + b2); ``cur`` is applied after
@@ -468,4 +509,4 @@ def pin_backward_finite_differences(orc, seed=18):
 ALL_PINS = [pin_hand_direct, pin_hand_mamba, pin_softplus_values, pin_lti_convolution,
             pin_brute_force, pin_tree_scan, pin_degenerate, pin_skip_and_gate, pin_h0_split,
             pin_decode, pin_p1_numpy_example, pin_p3_shape_example,
-            pin_backward_finite_differences]
+            pin_backward_finite_differences, pin_zoh_limits]

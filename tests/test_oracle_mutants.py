@@ -22,6 +22,7 @@ MUTANTS = {
     13: "backward: state gradient not carried through Abar",
     14: "backward: Delta's input-term gradient dropped",
     15: "backward: sigmoid in place of the silu derivative",
+    16: "zero-order hold: the A = 0 limit Delta*B lost",
 }
 
 
