@@ -203,14 +203,29 @@ SSM_API ssm_status ssm_scan_step(ssm_scan_plan *plan, const void *x, const void 
  * scratch, so calls that overlap on the GPU (other streams or threads) race
  * and give wrong results.  The first call on a device looks the scratch
  * address up (cudaGetSymbolAddress); make that first call before any stream
- * capture.  A device-side wait timeout is not reported by this entry point
- * (outputs are then unspecified).  Nothing is allocated; inputs and outputs
- * are the caller's device buffers. */
+ * capture (a new CUDA context on the device, e.g. after cudaDeviceReset,
+ * makes the next call look it up again).  A device-side wait that runs out
+ * is recorded in the scratch (outputs of that call are then unspecified) and
+ * reported by ssm_scan_noalloc_status.  Nothing is allocated; inputs and
+ * outputs are the caller's device buffers. */
 SSM_API ssm_status ssm_scan_fwd_noalloc(const ssm_scan_desc *desc, const void *x,
                                         const void *delta, const float *delta_bias,
                                         const float *A, const void *B, const void *C,
                                         const float *D, const void *z, const float *h0,
                                         void *y, float *h_last, ssm_stream_t stream);
+
+/* Status of the allocation-free entry point on the caller's current device
+ * (no counterpart on the pages; it belongs to ssm_scan_fwd_noalloc):
+ * synchronises the device, returns the device-side status recorded by the
+ * calls since the last query (SSM_OK or SSM_ERR_TIMEOUT) and resets it.
+ * Allocates nothing. */
+SSM_API ssm_status ssm_scan_noalloc_status(void);
+
+/* Test hook of the allocation-free entry point, process-wide: the bound of
+ * its device-side waits (nanoseconds, 0 = default of 2 s) and the work unit
+ * whose hand-over of its carried state is skipped (-1 = none), as
+ * ssm_scan_set_debug does for a plan. */
+SSM_API ssm_status ssm_scan_noalloc_set_debug(uint64_t wait_timeout_ns, int64_t drop_unit);
 
 /* Synchronise the plan's device, return the device-side status recorded by
  * the last calls (SSM_OK or SSM_ERR_TIMEOUT) and reset it to SSM_OK. */
@@ -229,6 +244,19 @@ SSM_API ssm_status ssm_scan_set_config(ssm_scan_plan *plan, const ssm_scan_confi
  * that row waits until the bound expires.  Used to test the timeout path
  * without hanging the device. */
 SSM_API ssm_status ssm_scan_set_debug(ssm_scan_plan *plan, uint64_t wait_timeout_ns, int64_t drop_unit);
+
+/* Throughput probe for the roofline denominators (a measurement helper; the
+ * pages have no counterpart): launches `blocks` CTAs of 256 threads on
+ * `stream`, each thread running independent chains of kind 0 = ex2.approx
+ * (the special-function unit that computes the exponential of every state
+ * update) or kind 1 = fp32 FMA, `iters` x 64 operations per thread.  *ops
+ * receives the number of operations launched (results per thread x threads);
+ * the caller times the launch (e.g. with CUDA events) and divides.  `sink` is
+ * a device buffer of at least `blocks` floats that the probe may write.
+ * Returns SSM_ERR_INVALID_ARG for a bad argument, SSM_ERR_CUDA if the launch
+ * fails. */
+SSM_API ssm_status ssm_probe_peak(int kind, int64_t iters, int blocks, float *sink,
+                                  int64_t *ops, ssm_stream_t stream);
 
 /* Static description of a status code. */
 SSM_API const char *ssm_status_string(ssm_status s);

@@ -95,6 +95,15 @@ def load_library(path: str | None = None):
         lib.ssm_status_string.restype = ctypes.c_char_p
         lib.ssm_scan_version.argtypes = []
         lib.ssm_scan_version.restype = ctypes.c_int
+        lib.ssm_scan_fwd_noalloc.argtypes = [ctypes.POINTER(Desc)] + [_vp] * 12
+        lib.ssm_scan_fwd_noalloc.restype = st
+        lib.ssm_scan_noalloc_status.argtypes = []
+        lib.ssm_scan_noalloc_status.restype = st
+        lib.ssm_scan_noalloc_set_debug.argtypes = [ctypes.c_uint64, ctypes.c_int64]
+        lib.ssm_scan_noalloc_set_debug.restype = st
+        lib.ssm_probe_peak.argtypes = [ctypes.c_int, ctypes.c_int64, ctypes.c_int, _vp,
+                                       ctypes.POINTER(ctypes.c_int64), _vp]
+        lib.ssm_probe_peak.restype = st
         _lib = lib
         return lib
 
@@ -269,6 +278,18 @@ class Plan:
                                      _stream(dev))
         _check(rc, "ssm_scan_step")
         return y
+
+
+def probe_peak(kind: int, iters: int, blocks: int, sink, stream=None) -> int:
+    """Launch the library's throughput probe (kind 0 = ex2.approx, 1 = fp32
+    FMA) on the current stream; returns the operation count it launched."""
+    ops = ctypes.c_int64(0)
+    dev = sink.device
+    st = ctypes.c_void_p(stream.cuda_stream if stream is not None
+                         else torch.cuda.current_stream(dev).cuda_stream)
+    _check(load_library().ssm_probe_peak(int(kind), int(iters), int(blocks), _ptr(sink),
+                                         ctypes.byref(ops), st), "ssm_probe_peak")
+    return ops.value
 
 
 def flags_for(*, z=None, D=None, delta_bias=None, h0=None, delta_softplus=True,

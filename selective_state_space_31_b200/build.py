@@ -9,6 +9,7 @@ from __future__ import annotations
 
 import concurrent.futures as cf
 import glob
+import hashlib
 import os
 import shutil
 import subprocess
@@ -19,6 +20,9 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libssm_scan_b200.so")
+# sha256 of every source, header and compiler flag the library was linked
+# from, written beside it; a library whose record differs is rebuilt
+STAMP = LIB + ".srchash"
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
@@ -44,16 +48,40 @@ def _stale(out: str, deps: list[str]) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
+def source_hash(extra: list[str] | None = None) -> str:
+    """Hash of everything the library is built from: the sources and headers
+    (by content, in name order) and the nvcc command-line flags."""
+    h = hashlib.sha256()
+    files = sorted(set(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh"))
+                       + glob.glob(os.path.join(CSRC, "*.h"))
+                       + [os.path.join(ROOT, "include", "ssm_scan.h")]))
+    for f in files:
+        h.update(os.path.relpath(f, ROOT).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    h.update(" ".join(ARCH + FLAGS + list(extra or [])).encode())
+    return h.hexdigest()
+
+
+def _current(want: str) -> bool:
+    if not (os.path.exists(LIB) and os.path.exists(STAMP)):
+        return False
+    with open(STAMP) as fh:
+        return fh.read().strip() == want
+
+
 def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
-    # a library newer than every source is current even where the object
-    # files were not kept (a copy of the tree without _build/)
-    if not force and not extra and not _stale(LIB, [d for s in srcs for d in _deps(s)]):
+    # the library is current exactly when it was linked from these very
+    # sources and flags (content hash, not file times: a copied tree keeps
+    # its record, an edited source does not match it)
+    want = source_hash(extra)
+    if not force and _current(want):
         return LIB
     os.makedirs(BUILD, exist_ok=True)
     objs = [os.path.join(BUILD, os.path.basename(s)[:-3] + ".o") for s in srcs]
     extra = list(extra or [])
-    todo = [(s, o) for s, o in zip(srcs, objs) if force or _stale(o, _deps(s))]
+    todo = [(s, o) for s, o in zip(srcs, objs) if force or extra or _stale(o, _deps(s))]
 
     def compile_one(so):
         s, o = so
@@ -67,13 +95,15 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
         for msg in ex.map(compile_one, todo):
             if verbose and msg:
                 print(msg, file=sys.stderr)
-    if force or todo or _stale(LIB, objs):
-        tmp = LIB + ".tmp"
-        cmd = [nvcc()] + ARCH + ["-shared", "-cudart", "static", "-o", tmp] + objs
-        r = subprocess.run(cmd, capture_output=True, text=True)
-        if r.returncode != 0:
-            raise RuntimeError(f"link failed:\n{r.stderr}")
-        os.replace(tmp, LIB)
+    tmp = LIB + ".tmp"
+    cmd = [nvcc()] + ARCH + ["-shared", "-cudart", "static", "-o", tmp] + objs
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    if r.returncode != 0:
+        raise RuntimeError(f"link failed:\n{r.stderr}")
+    os.replace(tmp, LIB)
+    with open(STAMP + ".tmp", "w") as fh:
+        fh.write(want + "\n")
+    os.replace(STAMP + ".tmp", STAMP)
     return LIB
 
 

@@ -16,17 +16,18 @@
 //     LPC lanes (NPL = N / LPC each); the lanes' partial readouts of a group
 //     of LPC tokens are combined by a shuffle butterfly that leaves lane q with
 //     token q, and lane q finishes that token.
-//   * Strided item schedule.  Each row's S stages are cut into parts of PL
-//     stages; item i = part * R + row.  CTA c runs items c, c + P, c + 2P, ...
-//     in order (P = gridDim.x <= R).  The predecessor of an item (same row,
-//     previous part) has index i - R <= i - P, so it belongs to an earlier
-//     slot of some CTA: run in lock-step, no CTA waits, and every CTA gets the
-//     same number of items (to within one).  A part hands its final state to
-//     the next part through a per-(row, warp) flag carrying the stage index
-//     and a launch epoch (release/acquire) -- the pages' associative carry
-//     ("Scan bien recurrence ...": (A2,b2) (x) (A1,b1) = (A2A1, A2b1+b2)): the
-//     state after one part is the exact starting state of the next.  Every
-//     wait is bounded by a timer.
+//   * Ticket schedule.  Each row's S stages are cut into parts of PL stages;
+//     item i = part * R + row.  A CTA's load warp takes item numbers in
+//     increasing order from a device counter (one atomic per item), so the
+//     predecessor of an item (same row, previous part, number i - R) always
+//     went to a CTA that was already running: every wait for a carried state
+//     ends, however few CTAs the device runs at once, and CTAs that finish
+//     early simply take more items.  A part hands its final state to the next
+//     part through a per-(row, warp) flag carrying the stage index and a
+//     launch epoch (release/acquire) -- the pages' associative carry ("Scan
+//     bien recurrence ...": (A2,b2) (x) (A1,b1) = (A2A1, A2b1+b2)): the state
+//     after one part is the exact starting state of the next.  Every wait is
+//     bounded by a timer.
 //   * One load warp streams the stages' [TT, DT] tiles of x / delta / z and
 //     [TT, N] tiles of B / C into a ring of RAW shared-memory slots with TMA
 //     (cp.async.bulk.tensor, every CTA loads its own tiles); slot full / slot
@@ -139,27 +140,18 @@ __device__ __forceinline__ void load_bc(const __nv_bfloat16 *src, float (&dst)[N
   }
 }
 
-// Walks one CTA's items (c, c + P, c + 2P, ...) stage by stage; a division
-// happens only when a new item starts.
-struct ItemCursor {
-  int item, items, P, R, PL, S, nDT;
-  int row, part, st, st_end, b, dtile;
-  __device__ __forceinline__ void load() {
-    if (item >= items) return;
-    part = item / R;
-    row = item - part * R;
-    st = part * PL;
-    st_end = min(S, st + PL);
-    b = row / nDT;
-    dtile = row - b * nDT;
-  }
-  __device__ __forceinline__ void init(int c, const FwdParams &p) {
-    item = c; items = p.items; P = gridDim.x; R = p.rows; PL = p.PL; S = p.S; nDT = p.nDT;
-    row = part = st = st_end = b = dtile = 0;
-    load();
-  }
-  __device__ __forceinline__ void advance() {
-    if (++st == st_end) { item += P; load(); }
+// Position of one stage of work: item (row, part) and stage index, derived
+// from an item number once per item (a division happens only there).
+struct ItemPos {
+  int item = -1, row = 0, part = 0, b = 0, dtile = 0, st_begin = 0, st_end = 0;
+  __device__ __forceinline__ void set(int it, const FwdParams &p) {
+    item = it;
+    part = it / p.rows;
+    row = it - part * p.rows;
+    st_begin = part * p.PL;
+    st_end = min(p.S, st_begin + p.PL);
+    b = row / p.nDT;
+    dtile = row - b * p.nDT;
   }
 };
 
@@ -174,15 +166,12 @@ __global__ void __launch_bounds__((WARPS + 1) * 32)
   uint64_t *rfull = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_BAR);
   uint64_t *rempty = rfull + RAW;  // all scan warps are done with a slot
 
-  const unsigned int epoch = *reinterpret_cast<volatile unsigned int *>(&p.ctl->epoch);
+  // item and stage carried by each ring slot (written by the load warp
+  // before the slot's full barrier completes; item -1 ends the CTA's work)
+  __shared__ int2 slot_work[RAW];
 
-  // ---- strided item schedule: stages this CTA runs ----
+  const unsigned int epoch = *reinterpret_cast<volatile unsigned int *>(&p.ctl->epoch);
   const int S = p.S;
-  int n = 0;
-  for (int it = blockIdx.x; it < p.items; it += gridDim.x) {
-    const int part = it / p.rows;
-    n += min(S, (part + 1) * p.PL) - part * p.PL;
-  }
 
   if (tid == 0) {
 #pragma unroll
@@ -199,18 +188,34 @@ __global__ void __launch_bounds__((WARPS + 1) * 32)
     if (lane == 0) {
       const uint32_t tx_bytes =
           (p.has_z ? 3u : 2u) * TT * DT * sizeof(InT) + 2u * TT * NS * sizeof(InT);
-      ItemCursor iss;
-      iss.init(blockIdx.x, p);
+      // Work items are handed out in increasing order from a device counter
+      // (a ticket per item).  An item's predecessor (same row, previous part)
+      // has a smaller number, so it went to a CTA that was already running
+      // when this one took its ticket: waits on carried states always end,
+      // whatever share of the device this launch gets.
+      ItemPos iss;
+      int st = 0;
       bool ok = true;
       int k = 0;
-      for (; k < n; ++k, iss.advance()) {
+      for (;; ++k) {
         const int r = k % RAW;
         if (k >= RAW &&
             !mbar_wait_bounded(&rempty[r], (uint32_t)(((k / RAW) - 1) & 1), p.timeout_ns)) {
           ok = false;
           break;
         }
-        const int d0 = iss.dtile * DT, t0 = iss.st * TT, b = iss.b;
+        if (iss.item < 0 || st == iss.st_end) {
+          const int it = (int)atomicAdd(&p.ctl->ticket, 1u);
+          if (it >= p.items) {  // no work left: end marker, no data
+            slot_work[r] = make_int2(-1, 0);
+            mbar_arrive(&rfull[r]);
+            break;
+          }
+          iss.set(it, p);
+          st = iss.st_begin;
+        }
+        slot_work[r] = make_int2(iss.item, st);
+        const int d0 = iss.dtile * DT, t0 = st * TT, b = iss.b;
         unsigned char *sb = smem + r * Cfg::SLOT;
         mbar_arrive_expect_tx(&rfull[r], tx_bytes);
         tma_load_3d(sb, &maps.x, &rfull[r], d0, t0, b);
@@ -218,6 +223,7 @@ __global__ void __launch_bounds__((WARPS + 1) * 32)
         if (p.has_z) tma_load_3d(sb + 2 * Cfg::XTILE, &maps.z, &rfull[r], d0, t0, b);
         tma_load_3d(sb + 3 * Cfg::XTILE, &maps.B, &rfull[r], 0, t0, b);
         tma_load_3d(sb + 3 * Cfg::XTILE + Cfg::BCTILE, &maps.C, &rfull[r], 0, t0, b);
+        ++st;
       }
       if (!ok) {
         atomicCAS(&p.ctl->status, 0, kStatusTimeout);
@@ -237,14 +243,21 @@ __global__ void __launch_bounds__((WARPS + 1) * 32)
     for (int i = 0; i < NPL; ++i) { h[i] = 0.f; A2[i] = 0.f; invA[i] = 0.f; }
     float bias = 0.f, dsk = 0.f;
     OutT *const ybase = reinterpret_cast<OutT *>(p.y);
-    ItemCursor cur;
-    cur.init(blockIdx.x, p);
-    for (int k = 0; k < n; ++k, cur.advance()) {
+    ItemPos cur;
+    for (int k = 0;; ++k) {
       const int r = k % RAW;
-      const int row = cur.row, st = cur.st, b = cur.b;
+      if (!__all_sync(FULL_MASK, mbar_wait_bounded(&rfull[r], (uint32_t)((k / RAW) & 1),
+                                                   p.timeout_ns))) {
+        if (lane == 0) atomicCAS(&p.ctl->status, 0, kStatusTimeout);
+        break;
+      }
+      const int2 work = slot_work[r];
+      if (work.x < 0) break;  // end marker
+      if (work.x != cur.item) cur.set(work.x, p);
+      const int row = cur.row, st = work.y, b = cur.b;
       const int d = cur.dtile * DT + ch;
       const bool valid_ch = d < p.D;
-      const bool run_start = st == cur.part * cur.PL;
+      const bool run_start = st == cur.st_begin;
       if (run_start) {  // per-item parameters and starting state of this lane
 #pragma unroll
         for (int i = 0; i < NPL; ++i) {
@@ -279,11 +292,6 @@ __global__ void __launch_bounds__((WARPS + 1) * 32)
         }
       }
 
-      if (!__all_sync(FULL_MASK, mbar_wait_bounded(&rfull[r], (uint32_t)((k / RAW) & 1),
-                                                   p.timeout_ns))) {
-        if (lane == 0) atomicCAS(&p.ctl->status, 0, kStatusTimeout);
-        break;
-      }
       const unsigned char *sb = smem + r * Cfg::SLOT;
       const InT *xs = reinterpret_cast<const InT *>(sb);
       const InT *ds = reinterpret_cast<const InT *>(sb + Cfg::XTILE);
@@ -409,6 +417,7 @@ __global__ void __launch_bounds__((WARPS + 1) * 32)
     const unsigned int prev = atomicAdd(&p.ctl->done, 1u);
     if (prev == gridDim.x - 1) {  // last CTA of this launch: ready the next call
       p.ctl->done = 0u;
+      p.ctl->ticket = 0u;
       p.ctl->epoch = epoch + 1u;
       __threadfence();
     }

@@ -25,6 +25,8 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
+#include <cstddef>
 #include <cstdint>
 #include <mutex>
 
@@ -36,25 +38,93 @@ namespace {
 constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
 constexpr size_t kCtlBytes = 256;
 constexpr int kMaxDevices = 64;
+constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-// Device address of g_noalloc_scratch, looked up once per device with that
-// device current (host code must not use the symbol itself as an address).
+// Test hook (ssm_scan_noalloc_set_debug): wait bound and dropped hand-over.
+std::atomic<uint64_t> g_timeout_ns{kDefaultTimeoutNs};
+std::atomic<int64_t> g_drop_unit{-1};
+
+PFN_cuCtxGetCurrent_v4000 ctx_getter() {
+  static PFN_cuCtxGetCurrent_v4000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 4000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+  });
+  return fn;
+}
+
+// Device address of g_noalloc_scratch in the current context of `device`
+// (host code must not use the symbol itself as an address).  Looked up with
+// that device current and cached per device together with the context it was
+// taken in: a new primary context (after cudaDeviceReset) reloads the module,
+// so the address is looked up again.
 void *scratch_address(int device) {
   static std::mutex mu;
   static void *addr[kMaxDevices] = {};
+  static CUcontext ctx_of[kMaxDevices] = {};
   if (device < 0 || device >= kMaxDevices) return nullptr;
+  CUcontext ctx = nullptr;
+  auto get_ctx = ctx_getter();
+  if (!get_ctx || get_ctx(&ctx) != CUDA_SUCCESS || !ctx) return nullptr;
   std::lock_guard<std::mutex> lock(mu);
-  if (!addr[device]) {
+  if (!addr[device] || ctx_of[device] != ctx) {
     void *p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) {
       cudaGetLastError();
       return nullptr;
     }
     addr[device] = p;
+    ctx_of[device] = ctx;
   }
   return addr[device];
+}
+
+// Launch shapes chosen before, per device and problem: repeat calls only
+// encode tensor maps and launch.
+struct ShapeKey {
+  int device, in_dtype, out_dtype, ns;
+  int64_t batch, seqlen, dim;
+  bool zoh;
+  bool operator==(const ShapeKey &o) const {
+    return device == o.device && in_dtype == o.in_dtype && out_dtype == o.out_dtype &&
+           ns == o.ns && batch == o.batch && seqlen == o.seqlen && dim == o.dim && zoh == o.zoh;
+  }
+};
+constexpr int kShapeCache = 16;
+
+bool cached_shape(const ShapeKey &key, int num_sms, ssm::FwdShape *out) {
+  static std::mutex mu;
+  static ShapeKey keys[kShapeCache];
+  static ssm::FwdShape shapes[kShapeCache];
+  static int used = 0, next = 0;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < used; ++i)
+      if (keys[i] == key) {
+        *out = shapes[i];
+        return true;
+      }
+  }
+  ssm::FwdShape fs;
+  if (ssm::choose_fwd_shape(key.in_dtype, key.out_dtype, key.batch, key.seqlen, key.dim, key.ns,
+                            key.zoh, num_sms, ssm::FwdOverrides{0, 0, 0, 0}, &fs) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  keys[next] = key;
+  shapes[next] = fs;
+  next = (next + 1) % kShapeCache;
+  used = std::min(used + 1, kShapeCache);
+  *out = fs;
+  return true;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encoder_na() {
@@ -97,7 +167,7 @@ extern "C" SSM_API ssm_status ssm_scan_fwd_noalloc(
   if (!desc) return SSM_ERR_INVALID_ARG;
   const ssm_scan_desc &d = *desc;
   const uint32_t f = d.flags;
-  if (d.batch < 1 || d.seqlen < 1 || d.dim < 1) return SSM_ERR_INVALID_ARG;
+  if (d.batch < 1 || d.seqlen < 1 || d.dim < 1 || d.dstate < 1) return SSM_ERR_INVALID_ARG;
   if (d.batch > INT32_MAX || d.seqlen > INT32_MAX || d.dim > INT32_MAX) return SSM_ERR_UNSUPPORTED;
   if ((d.in_dtype != SSM_F32 && d.in_dtype != SSM_BF16) ||
       (d.out_dtype != SSM_F32 && d.out_dtype != SSM_BF16))
@@ -105,10 +175,11 @@ extern "C" SSM_API ssm_status ssm_scan_fwd_noalloc(
   constexpr uint32_t known = SSM_HAS_Z | SSM_HAS_D | SSM_DELTA_SOFTPLUS | SSM_HAS_DELTA_BIAS |
                              SSM_HAS_H0 | SSM_WANT_HLAST | SSM_ZOH;
   if (f & ~known) return SSM_ERR_INVALID_ARG;
-  // the fast-path shape rules of the chunked kernel
+  // the fast-path shape rules of the chunked kernel (dstate checked before
+  // it is narrowed)
+  if (d.dstate != 4 && d.dstate != 8 && d.dstate != 16) return SSM_ERR_UNSUPPORTED;
   const int ns = (int)d.dstate;
   const size_t ei = d.in_dtype == SSM_BF16 ? 2 : 4, eo = d.out_dtype == SSM_BF16 ? 2 : 4;
-  if (ns != 4 && ns != 8 && ns != 16) return SSM_ERR_UNSUPPORTED;
   if (ns == 4 && d.in_dtype == SSM_BF16) return SSM_ERR_UNSUPPORTED;
   if (d.in_dtype == SSM_F32 && d.out_dtype == SSM_BF16) return SSM_ERR_UNSUPPORTED;
   if ((d.dim * ei) % 16 || (ns * ei) % 16 || (d.dim * eo) % 16) return SSM_ERR_UNSUPPORTED;
@@ -127,14 +198,11 @@ extern "C" SSM_API ssm_status ssm_scan_fwd_noalloc(
     cudaGetLastError();
     return SSM_ERR_CUDA;
   }
-  // launch shape: the same choice a plan makes by default
+  // launch shape: the same choice a plan makes by default (cached)
   ssm::FwdShape fs;
-  if (ssm::choose_fwd_shape((int)d.in_dtype, (int)d.out_dtype, d.batch, d.seqlen, d.dim, ns,
-                            (f & SSM_ZOH) != 0, num_sms, ssm::FwdOverrides{0, 0, 0, 0},
-                            &fs) != cudaSuccess) {
-    cudaGetLastError();
-    return SSM_ERR_UNSUPPORTED;
-  }
+  const ShapeKey key{device, (int)d.in_dtype, (int)d.out_dtype, ns, d.batch, d.seqlen, d.dim,
+                     (f & SSM_ZOH) != 0};
+  if (!cached_shape(key, num_sms, &fs)) return SSM_ERR_UNSUPPORTED;
   const int DT = fs.DT, warps = fs.ls.warps, TT = fs.ls.tt;
   const int nDT = (int)((d.dim + DT - 1) / DT);
   const int64_t rows = fs.rows;
@@ -149,7 +217,7 @@ extern "C" SSM_API ssm_status ssm_scan_fwd_noalloc(
   if (!base) return SSM_ERR_CUDA;
 
   ssm::TmaMaps maps;
-  const uint64_t Bn = d.batch, L = d.seqlen, Dm = d.dim, N = d.dstate;
+  const uint64_t Bn = d.batch, L = d.seqlen, Dm = d.dim, N = (uint64_t)ns;
   if (!encode_na(&maps.x, d.in_dtype, x, Dm, L, Bn, DT, TT) ||
       !encode_na(&maps.dt, d.in_dtype, delta, Dm, L, Bn, DT, TT) ||
       !encode_na(&maps.z, d.in_dtype, z ? z : x, Dm, L, Bn, DT, TT) ||
@@ -172,9 +240,34 @@ extern "C" SSM_API ssm_status ssm_scan_fwd_noalloc(
   p.ctl = reinterpret_cast<ssm::Control *>(base);
   p.ws_flags = reinterpret_cast<unsigned long long *>(base + kCtlBytes);
   p.ws_state = reinterpret_cast<float *>(base + st_off);
-  p.timeout_ns = 2000000000ull;
-  p.drop_unit = -1;
+  p.timeout_ns = g_timeout_ns.load();
+  p.drop_unit = g_drop_unit.load();
   const cudaError_t e = ssm::launch_fwd_tma((int)d.in_dtype, (int)d.out_dtype, ls, maps, p,
                                             reinterpret_cast<cudaStream_t>(stream_));
   return e == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+extern "C" SSM_API ssm_status ssm_scan_noalloc_status(void) {
+  int device = 0;
+  if (cudaGetDevice(&device) != cudaSuccess) {
+    cudaGetLastError();
+    return SSM_ERR_CUDA;
+  }
+  if (!scratch_address(device)) return SSM_ERR_CUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) return SSM_ERR_CUDA;
+  const size_t off = offsetof(ssm::Control, status);
+  int st = 0;
+  if (cudaMemcpyFromSymbol(&st, g_noalloc_scratch, sizeof(int), off) != cudaSuccess)
+    return SSM_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_noalloc_scratch, &zero, sizeof(int), off) != cudaSuccess)
+    return SSM_ERR_CUDA;
+  return (ssm_status)st;
+}
+
+extern "C" SSM_API ssm_status ssm_scan_noalloc_set_debug(uint64_t wait_timeout_ns,
+                                                          int64_t drop_unit) {
+  g_timeout_ns.store(wait_timeout_ns ? wait_timeout_ns : kDefaultTimeoutNs);
+  g_drop_unit.store(drop_unit);
+  return SSM_OK;
 }

@@ -16,8 +16,10 @@ struct Control {
   unsigned int done;        // CTAs finished in the current launch
   unsigned int epoch;       // launch counter, tags the carry flags
   int status;               // 0 or a timeout code, sticky until read
-  int pad[3];
+  unsigned int ticket;      // next work item to hand out in the current launch
+  int pad[2];
 };
+static_assert(sizeof(Control) == 32, "control block layout");
 
 struct FwdParams {
   int Bsz, L, D, N;

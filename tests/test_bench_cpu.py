@@ -60,3 +60,42 @@ def test_cli_flags():
         sys.argv = argv
     assert a.bwd and a.zoh and a.workload == "mamba1p4b_layer" and a.gpus == 1
     assert a.warmup >= 3
+
+
+def test_default_headline_is_the_largest_workload():
+    """With no flags the headline is the long sequence, the largest
+    single-GPU workload (B*L*D*N of every forward workload compared)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    a = bench.parse_args([])
+    assert a.workload == "long_seq" and a.steps >= 1 and a.warmup >= 3
+    sizes = {"tiny_fp32": 1 * 512 * 64, "mamba130m_layer": 8 * 2048 * 1536,
+             "mamba1p4b_layer": 4 * 8192 * 4096, "long_seq": 1 * 131072 * 2560}
+    assert max(sizes, key=sizes.get) == a.workload
+
+
+def test_both_arms_name_the_same_config():
+    """The reference arm's config is exactly our arm's for the same workload."""
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "tiny_fp32", "--steps", "1", "--warmup", "0",
+                        "--cpu-budget-s", "0.1"], capture_output=True, text=True, timeout=600,
+                       cwd=ROOT)
+    assert r.returncode == 0, r.stderr
+    ref = json.loads([l for l in r.stdout.splitlines() if l.strip()][0])
+    sys.path.insert(0, ROOT)
+    import bench
+    from selective_state_space_31_b200 import synth
+    assert ref["config"] == bench.arm_config(synth.tiny_fp32(), 1, False)
+
+
+def test_backward_counts():
+    sys.path.insert(0, ROOT)
+    import bench
+    from selective_state_space_31_b200 import synth
+    inp = synth.make_fwd(2, 64, 32, 16, seed=1)
+    f, b = bench.algorithmic_counts(inp), bench.algorithmic_counts(inp, backward=True)
+    B, L, D, N = 2, 64, 32, 16
+    assert b["mufu"] == 3 * B * L * D * N + 2 * 4 * B * L * D
+    # gradients are fp32: the backward moves well over twice the forward's bytes
+    assert b["bytes"] > 2 * f["bytes"]
+    assert b["bytes"] >= 4 * 3 * B * L * D + 4 * 2 * B * L * N + 8 * B * D * (L // 16) * N
