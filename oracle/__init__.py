@@ -89,6 +89,8 @@ class Oracle:
         self._lib.ssm_oracle_direct.restype = ctypes.c_int
         self._lib.ssm_oracle_bwd.argtypes = [i64, i64, i64, i64, u32] + [_dp] * 20
         self._lib.ssm_oracle_bwd.restype = ctypes.c_int
+        self._lib.ssm_oracle_causal_conv_silu.argtypes = [i64, i64, i64, i64] + [_dp] * 4
+        self._lib.ssm_oracle_causal_conv_silu.restype = ctypes.c_int
 
     def softplus(self, v: float) -> float:
         return self._lib.ssm_oracle_softplus(float(v))
@@ -123,6 +125,28 @@ class Oracle:
         if rc != 0:
             raise ValueError("oracle fwd rejected its arguments")
         return y, hl
+
+    def causal_conv_silu(self, x_in, w, bias=None):
+        """silu(causal depthwise conv of x_in (Bsz, L, D) with w (D, K) and
+        bias (D,)), float64 (Bsz, L, D)."""
+        x_in = _arr(x_in)
+        Bsz, L, Dm = x_in.shape
+        w = _arr(w)
+        K = w.shape[1]
+        bias = _arr(bias, (Dm,))
+        out = np.empty_like(x_in)
+        rc = self._lib.ssm_oracle_causal_conv_silu(Bsz, L, Dm, K, _ptr(x_in), _ptr(w), _ptr(bias),
+                                                   _ptr(out))
+        if rc != 0:
+            raise ValueError("oracle conv rejected its arguments")
+        return out
+
+    def fwd_conv(self, x_in, conv_w, conv_b, delta, A, B, C, **kw):
+        """The scan fed by the conv front-end: x = silu(causal_conv(x_in));
+        returns (y, h_last, x)."""
+        x = self.causal_conv_silu(x_in, conv_w, conv_b)
+        y, hl = self.fwd(x, delta, A, B, C, **kw)
+        return y, hl, x
 
     def bwd(self, x, delta, A, B, C, dy, D=None, z=None, delta_bias=None, h0=None,
             dh_last=None, delta_softplus=True):

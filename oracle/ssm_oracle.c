@@ -191,6 +191,42 @@ int ssm_oracle_fwd(int64_t Bsz, int64_t L, int64_t D, int64_t N, uint32_t flags,
 }
 
 #ifndef ORACLE_FP32
+/* Causal depthwise convolution of the x branch followed by silu, the
+ * front-end that feeds the scan's x ([P5] section 5.3 names the fused
+ * causal_conv1d + selective_scan_fn kernels; the operation is read as the
+ * standard one of that name): per channel d, with x_in = 0 before t = 0,
+ *   u[b,t,d] = bias[d] + sum_{k=0}^{K-1} w[d,k] * x_in[b, t-(K-1)+k, d],
+ *   out[b,t,d] = silu(u[b,t,d]).
+ * w[d, K-1] multiplies the current token.  x_in, out: (B, L, D); w: (D, K);
+ * bias: (D) or NULL.  Returns 0, or -1 on a bad argument. */
+int ssm_oracle_causal_conv_silu(int64_t Bsz, int64_t L, int64_t D, int64_t K,
+                                const double *x_in, const double *w, const double *bias,
+                                double *out) {
+  if (Bsz < 0 || L < 0 || D < 0 || K < 1 || !x_in || !w || !out) return -1;
+  for (int64_t b = 0; b < Bsz; ++b)
+    for (int64_t t = 0; t < L; ++t)
+      for (int64_t d = 0; d < D; ++d) {
+        double u = bias ? bias[d] : 0.0;
+#if ORACLE_MUTANT == 18
+        u = 0.0; /* bias dropped */
+#endif
+        for (int64_t k = 0; k < K; ++k) {
+          int64_t src = t - (K - 1) + k;
+#if ORACLE_MUTANT == 19
+          src += 1; /* window shifted one token into the future */
+#endif
+          if (src < 0 || src >= L) continue;
+#if ORACLE_MUTANT == 17
+          u += w[d * K + (K - 1 - k)] * x_in[(b * L + src) * D + d]; /* taps reversed */
+#else
+          u += w[d * K + k] * x_in[(b * L + src) * D + d];
+#endif
+        }
+        out[(b * L + t) * D + d] = ssm_oracle_silu(u);
+      }
+  return 0;
+}
+
 /* One decode step ([P1] inference section): state (B, D, N) is read, updated
  * with one token and written back; y is (B, D).  x, delta, z: (B, D);
  * Bm, Cm: (B, N). */

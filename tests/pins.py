@@ -506,7 +506,50 @@ def pin_backward_finite_differences(orc, seed=18):
     _fd_case(orc, rng, False)
 
 
+def pin_causal_conv(orc, seed=20):
+    """The conv front-end of the x branch ([P5] section 5.3 names the fused
+    causal_conv1d): per channel u_t = bias + sum_k w[k] x_{t-(K-1)+k} with
+    x = 0 before the sequence, then silu.
+    (i) identity taps (0, 0, 0, 1), no bias: the output is silu(x) itself;
+    (ii) a hand-computed dyadic case (K = 4, one channel):
+         x = (1, 2, -1, 4, 0.5), w = (0.5, -1, 0.25, 2), bias = 0.5:
+         u_0 = 0.5 + 2*1                              = 2.5
+         u_1 = 0.5 + 0.25*1 + 2*2                     = 4.75
+         u_2 = 0.5 - 1*1 + 0.25*2 + 2*(-1)            = -2
+         u_3 = 0.5 + 0.5*1 - 1*2 + 0.25*(-1) + 2*4    = 6.75
+         u_4 = 0.5 + 0.5*2 - 1*(-1) + 0.25*4 + 2*0.5  = 4.5
+    (iii) random taps against numpy's full convolution with the taps
+    reversed (a library routine), truncated to the first L outputs;
+    (iv) causality: changing x at t0 leaves every output before t0 alone."""
+    silu = _silu_ref
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((2, 9, 3))
+    w = np.zeros((3, 4))
+    w[:, 3] = 1.0
+    _close(orc.causal_conv_silu(x, w), silu(x), 1e-15, 1e-15, "identity taps")
+    xh = np.array([1.0, 2.0, -1.0, 4.0, 0.5]).reshape(1, 5, 1)
+    wh = np.array([[0.5, -1.0, 0.25, 2.0]])
+    u = np.array([2.5, 4.75, -2.0, 6.75, 4.5])
+    _close(orc.causal_conv_silu(xh, wh, np.array([0.5])).ravel(), silu(u), 1e-15, 1e-15,
+           "hand conv")
+    Bsz, L, D, K = 2, 17, 5, 4
+    x = rng.standard_normal((Bsz, L, D))
+    w = rng.standard_normal((D, K))
+    bias = rng.standard_normal(D)
+    got = orc.causal_conv_silu(x, w, bias)
+    want = np.zeros_like(x)
+    for b in range(Bsz):
+        for d in range(D):
+            want[b, :, d] = silu(bias[d] + np.convolve(x[b, :, d], w[d, ::-1])[:L])
+    _close(got, want, 1e-13, 1e-14, "conv vs numpy.convolve")
+    x2 = x.copy()
+    x2[:, 9] += 3.0
+    got2 = orc.causal_conv_silu(x2, w, bias)
+    _close(got2[:, :9], got[:, :9], 0, 0, "causality")
+    assert np.all(np.abs(got2[:, 9] - got[:, 9]) > 0), "the changed token itself moves"
+
+
 ALL_PINS = [pin_hand_direct, pin_hand_mamba, pin_softplus_values, pin_lti_convolution,
             pin_brute_force, pin_tree_scan, pin_degenerate, pin_skip_and_gate, pin_h0_split,
             pin_decode, pin_p1_numpy_example, pin_p3_shape_example,
-            pin_backward_finite_differences, pin_zoh_limits]
+            pin_backward_finite_differences, pin_zoh_limits, pin_causal_conv]

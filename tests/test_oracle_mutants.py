@@ -23,6 +23,9 @@ MUTANTS = {
     14: "backward: Delta's input-term gradient dropped",
     15: "backward: sigmoid in place of the silu derivative",
     16: "zero-order hold: the A = 0 limit Delta*B lost",
+    17: "conv front-end: taps reversed",
+    18: "conv front-end: bias dropped",
+    19: "conv front-end: window shifted one token",
 }
 
 
