@@ -71,6 +71,10 @@ def parse_args(argv=None):
                     help="time the backward pass (ssm_scan_bwd) instead of the forward")
     ap.add_argument("--zoh", action="store_true",
                     help="zero-order-hold input matrix (exp(Delta A) - 1)/A * B instead of Delta * B")
+    ap.add_argument("--shape", default="",
+                    help="B,L,D: a resized copy of --workload (profiling on smaller inputs)")
+    ap.add_argument("--segments", type=int, default=0, help="segments per row (launch override)")
+    ap.add_argument("--kc", type=int, default=0, help="channels per lane (launch override)")
     return ap.parse_args(argv)
 
 
@@ -113,8 +117,7 @@ def algorithmic_counts(inp, backward=False):
 # sources that define the forward kernel and its launch shape: a committed
 # ncu summary's traffic figure is used only while these are unchanged
 FWD_KERNEL_SOURCES = ("device_common.cuh", "scan_params.h", "scan_fwd_kernel.cuh",
-                      "scan_fwd_bf16.cu", "scan_fwd_f32.cu", "scan_fwd_bf16_f32.cu",
-                      "scan_fwd_dispatch.cu")
+                      "scan_fwd_variants.h", "scan_fwd_dispatch.cu")
 STEP_KERNEL_SOURCES = ("device_common.cuh", "scan_params.h", "scan_step.cu")
 
 
@@ -397,7 +400,9 @@ def run_fwd(name, steps, warmup, args, rank, world, device, peaks, e2e_steps,
     from selective_state_space_31_b200 import synth
 
     torch.cuda.set_device(device)
-    make = synth.FWD_WORKLOADS[name]
+    shape = tuple(int(v) for v in args.shape.split(",")) if args.shape and \
+        name == args.workload else None
+    make = lambda **kw: synth.FWD_WORKLOADS[name](shape=shape, **kw)
     inp = make()
     inp.zoh = bool(args.zoh)
     tdt = {"f32": torch.float32, "bf16": torch.bfloat16}
@@ -423,8 +428,8 @@ def run_fwd(name, steps, warmup, args, rank, world, device, peaks, e2e_steps,
                           delta_softplus=inp.delta_softplus, want_h_last=True, zoh=inp.zoh)
     plan = bnd.Plan(inp.Bsz, inp.L, inp.D, inp.N, tdt[inp.in_dtype], tdt[inp.out_dtype], flags,
                     device)
-    if args.lpc or args.warps or args.grid or args.tile_t:
-        plan.set_config(args.lpc, args.warps, args.grid, args.tile_t)
+    if args.lpc or args.warps or args.grid or args.tile_t or args.segments or args.kc:
+        plan.set_config(args.lpc, args.warps, args.grid, args.tile_t, args.kc, args.segments)
     outs = [(torch.empty((inp.Bsz, inp.L, inp.D), dtype=tdt[inp.out_dtype], device=device),
              torch.empty((inp.Bsz, inp.D, inp.N), dtype=torch.float32, device=device))
             for _ in range(n_sets)]
@@ -555,9 +560,10 @@ def run_fwd(name, steps, warmup, args, rank, world, device, peaks, e2e_steps,
         "dtype": "bf16" if inp.in_dtype == "bf16" else "f32",
         "data": "synthetic (seeded normal draws, shapes and distributions of the workload)",
         "config": arm_config(inp, world, args.bwd),
-        "launch": {k: info[k] for k in ("lanes_per_chan", "warps_per_cta", "tile_t",
-                                        "chans_per_cta", "grid", "rows", "units",
-                                        "parts_per_row") if k in info},
+        "launch": {k: info[k] for k in ("lanes_per_chan", "chans_per_lane", "warps_per_cta",
+                                        "tile_t", "chans_per_cta", "grid", "rows", "units",
+                                        "parts_per_row", "segments", "stages_per_segment",
+                                        "carry_grid", "launches_per_call") if k in info},
         "roofline": {"bound": "alu", "achieved": achieved_mufu / 1e9, "peak": peak_mufu / 1e9,
                      "unit": "G MUFU-op/s (ex2, lg2, rcp)", "frac": achieved_mufu / peak_mufu,
                      "traffic": traffic, "peak_basis": basis,

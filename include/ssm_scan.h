@@ -95,9 +95,11 @@ enum {
   SSM_HAS_H0 = 16,          /* start from h0 (else from 0) */
   SSM_WANT_HLAST = 32,      /* write h_last */
   SSM_A_DIRECT = 64,        /* elementwise variant: N = 1, A/B/C per (b,t,d), no delta/D/z */
-  SSM_ZOH = 128             /* zero-order-hold input matrix: Bbar = (exp(Delta*A) - 1) / A * B
+  SSM_ZOH = 128,            /* zero-order-hold input matrix: Bbar = (exp(Delta*A) - 1) / A * B
                                ("Vi du Python" of the first page) instead of Delta * B;
                                Bbar -> Delta * B where A = 0.  Not with SSM_A_DIRECT. */
+  SSM_CONV_X = 256          /* the x branch passes through the causal conv front-end first
+                               (ssm_scan_fwd_conv); not with SSM_A_DIRECT or SSM_ZOH */
 };
 
 typedef struct {
@@ -118,22 +120,31 @@ typedef struct {
   int stages;          /* stage slots in the TMA ring (fused kernel) */
   int stages_per_row;  /* ceil(seqlen / tile_t) */
   int chans_per_cta;   /* channels per row tile */
-  int grid;            /* CTAs launched (CTA c runs items c, c + grid, ...) */
+  int grid;            /* CTAs launched (each takes work items by ticket) */
   int64_t rows;        /* independent (batch, channel-tile) rows */
   int64_t units;       /* stages in all = rows * stages_per_row */
-  int parts_per_row;   /* work items per row (a row's parts hand their state on) */
+  int parts_per_row;   /* work items per segment (a segment's parts hand their state on) */
   int stages_per_part;
   size_t smem_bytes;
   size_t workspace_bytes;
+  int chans_per_lane;  /* channels a lane owns (1 or 2) */
+  int segments;        /* segments per row scanned at the same time (1 = none) */
+  int stages_per_segment;
+  int carry_grid;      /* CTAs of the carry pass (segments > 1) */
+  int launches_per_call; /* kernels one ssm_scan_fwd launches (2 with segments) */
 } ssm_scan_info;
 
 /* Optional overrides of the launch shape (0 = keep the default). */
 typedef struct {
   int lanes_per_chan; /* 1, 2, 4, 8, 16 (<= dstate) */
   int warps_per_cta;  /* scan warps: 2, 4 or 8 (plus one load warp) */
-  int grid;           /* CTAs (clamped to what is co-resident on the device) */
-  int tile_t;         /* tokens per pipeline stage: 16, 32 or 64 */
+  int grid;           /* CTAs (any number: work items go out by ticket; capped by the items) */
+  int tile_t;         /* tokens per pipeline stage: 32 or 64 */
+  int chans_per_lane; /* 1 or 2 */
+  int segments;       /* segments per row: 1, 2, 4 or 8 (1 = none) */
 } ssm_scan_config;
+/* Only the combinations compiled into the library exist; ssm_scan_set_config
+ * returns SSM_ERR_UNSUPPORTED for others (ssm_scan_list_variants lists them). */
 
 /* Create a plan for one problem shape on `device`; allocates the workspace.
  * Returns SSM_ERR_INVALID_ARG / SSM_ERR_UNSUPPORTED for a bad desc (checked
@@ -154,6 +165,53 @@ SSM_API ssm_status ssm_scan_fwd(ssm_scan_plan *plan, const void *x, const void *
                         const float *delta_bias, const void *A, const void *B,
                         const void *C, const float *D, const void *z,
                         const float *h0, void *y, float *h_last, ssm_stream_t stream);
+
+/* Forward pass fed by the causal conv front-end of the x branch, fused into
+ * the scan kernel so the conv output never goes through HBM unless asked
+ * for.  "Tong quan ..." (vietitpro.vn), section 5.3 "Toi uu hoa Kernel
+ * Fusion cho Mamba SSM", names causal_conv1d with selective_scan_fn as the
+ * fused pair; the operation is the depthwise causal convolution over L with
+ * 4 taps per channel, then silu:
+ *   x[b,t,d] = silu(conv_b[d] + sum_{k=0..3} conv_w[d,k] * x_in[b, t-3+k, d])
+ * with x_in = 0 before t = 0 (conv_w[d,3] weighs the current token).  That x
+ * is the scan's x everywhere (the Delta*x input term and the D skip).  The
+ * plan must have SSM_CONV_X.  x_in: (batch, seqlen, dim) in_dtype;
+ * conv_w: (dim, 4) fp32; conv_b: (dim) fp32 or NULL (0); x_conv: NULL, or
+ * (batch, seqlen, dim) out_dtype to receive x.  The other arguments,
+ * ownership and errors are those of ssm_scan_fwd, which refuses SSM_CONV_X
+ * plans (SSM_ERR_INVALID_ARG).  ssm_scan_step and ssm_scan_bwd return
+ * SSM_ERR_UNSUPPORTED for such plans. */
+SSM_API ssm_status ssm_scan_fwd_conv(ssm_scan_plan *plan, const void *x_in, const float *conv_w,
+                                     const float *conv_b, const void *delta,
+                                     const float *delta_bias, const float *A, const void *B,
+                                     const void *C, const float *D, const void *z,
+                                     const float *h0, void *y, float *h_last, void *x_conv,
+                                     ssm_stream_t stream);
+
+/* Map of the plan's whole sequence, for a scan whose L is split over several
+ * devices or calls.  The tokens act on each channel's state as one affine
+ * map h -> P h + e per state ("Scan bien recurrence thanh phep toan co the
+ * song song hoa ra sao?": per-token maps compose associatively,
+ * (A2,b2) (x) (A1,b1) = (A2 A1, A2 b1 + b2)), where P = exp(A * sum_t Delta_t)
+ * and e is the state the sequence reaches from h = 0.  Writes
+ * map_h (batch, dim, dstate) fp32 = e and map_s (batch, dim) fp32 =
+ * sum_t Delta_t.  Inputs as for ssm_scan_fwd (x, delta, delta_bias, A, B;
+ * C, D, z are not needed).  The first call on a plan allocates a workspace
+ * (about 4*(dstate+1) bytes per channel and sub-chunk) and may return
+ * SSM_ERR_OOM.  Plans with SSM_A_DIRECT or SSM_CONV_X: SSM_ERR_UNSUPPORTED. */
+SSM_API ssm_status ssm_scan_seq_map(ssm_scan_plan *plan, const void *x, const void *delta,
+                                    const float *delta_bias, const float *A, const void *B,
+                                    float *map_h, float *map_s, ssm_stream_t stream);
+
+/* Composition of `count` sequence maps, in order, onto a starting state:
+ * h = h0 (NULL = 0); for j = 0 .. count-1: h = exp(A * s_j) * h + e_j; writes
+ * h_out (batch, dim, dstate) fp32.  maps_h: (count, batch, dim, dstate),
+ * maps_s: (count, batch, dim), fp32, as ssm_scan_seq_map writes them (one
+ * map per earlier piece of the sequence).  The result is the exact state at
+ * the start of the next piece, to pass as h0 to ssm_scan_fwd. */
+SSM_API ssm_status ssm_scan_fold_maps(ssm_scan_plan *plan, int count, const float *maps_h,
+                                      const float *maps_s, const float *A, const float *h0,
+                                      float *h_out, ssm_stream_t stream);
 
 /* Backward pass of ssm_scan_fwd (Delta*B input coefficient; plans with
  * SSM_ZOH or SSM_A_DIRECT get SSM_ERR_UNSUPPORTED): gradients of a loss
@@ -257,6 +315,20 @@ SSM_API ssm_status ssm_scan_set_debug(ssm_scan_plan *plan, uint64_t wait_timeout
  * fails. */
 SSM_API ssm_status ssm_probe_peak(int kind, int64_t iters, int blocks, float *sink,
                                   int64_t *ops, ssm_stream_t stream);
+
+/* One compiled variant of the fused kernel. */
+typedef struct {
+  int dstate, lanes_per_chan, chans_per_lane, warps_per_cta, tile_t;
+  int zoh;   /* zero-order-hold input coefficient */
+  int carry; /* the carry pass of a segmented launch (not a full scan) */
+  int conv;  /* with the causal conv front-end of the x branch */
+} ssm_scan_variant;
+
+/* The compiled variants of the fused kernel for a dtype pair (a tuning and
+ * test aid; the pages have no counterpart): fills up to `max` entries of
+ * `out` (which may be NULL) and returns how many exist. */
+SSM_API int ssm_scan_list_variants(ssm_dtype in_dtype, ssm_dtype out_dtype,
+                                   ssm_scan_variant *out, int max);
 
 /* Static description of a status code. */
 SSM_API const char *ssm_status_string(ssm_status s);

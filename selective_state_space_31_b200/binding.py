@@ -23,6 +23,8 @@ F32, BF16 = 0, 1
 # flags
 HAS_Z, HAS_D, DELTA_SOFTPLUS, HAS_DELTA_BIAS, HAS_H0, WANT_HLAST, A_DIRECT = 1, 2, 4, 8, 16, 32, 64
 ZOH = 128  # zero-order-hold input matrix: Bbar = (exp(Delta A) - 1) / A * B
+CONV_X = 256  # x branch through the causal conv front-end (ssm_scan_fwd_conv)
+CONV_WIDTH = 4
 
 _TORCH_TO_SSM = {torch.float32: F32, torch.bfloat16: BF16}
 
@@ -45,7 +47,10 @@ class Info(ctypes.Structure):
                 ("stages_per_row", ctypes.c_int), ("chans_per_cta", ctypes.c_int),
                 ("grid", ctypes.c_int), ("rows", ctypes.c_int64), ("units", ctypes.c_int64),
                 ("parts_per_row", ctypes.c_int), ("stages_per_part", ctypes.c_int),
-                ("smem_bytes", ctypes.c_size_t), ("workspace_bytes", ctypes.c_size_t)]
+                ("smem_bytes", ctypes.c_size_t), ("workspace_bytes", ctypes.c_size_t),
+                ("chans_per_lane", ctypes.c_int), ("segments", ctypes.c_int),
+                ("stages_per_segment", ctypes.c_int), ("carry_grid", ctypes.c_int),
+                ("launches_per_call", ctypes.c_int)]
 
     def as_dict(self):
         return {k: getattr(self, k) for k, _ in self._fields_}
@@ -53,7 +58,18 @@ class Info(ctypes.Structure):
 
 class Config(ctypes.Structure):
     _fields_ = [("lanes_per_chan", ctypes.c_int), ("warps_per_cta", ctypes.c_int),
-                ("grid", ctypes.c_int), ("tile_t", ctypes.c_int)]
+                ("grid", ctypes.c_int), ("tile_t", ctypes.c_int),
+                ("chans_per_lane", ctypes.c_int), ("segments", ctypes.c_int)]
+
+
+class Variant(ctypes.Structure):
+    _fields_ = [("dstate", ctypes.c_int), ("lanes_per_chan", ctypes.c_int),
+                ("chans_per_lane", ctypes.c_int), ("warps_per_cta", ctypes.c_int),
+                ("tile_t", ctypes.c_int), ("zoh", ctypes.c_int), ("carry", ctypes.c_int),
+                ("conv", ctypes.c_int)]
+
+    def as_dict(self):
+        return {k: getattr(self, k) for k, _ in self._fields_}
 
 
 _lib = None
@@ -79,6 +95,12 @@ def load_library(path: str | None = None):
         lib.ssm_scan_destroy.restype = st
         lib.ssm_scan_fwd.argtypes = [_vp] * 13
         lib.ssm_scan_fwd.restype = st
+        lib.ssm_scan_fwd_conv.argtypes = [_vp] * 16
+        lib.ssm_scan_fwd_conv.restype = st
+        lib.ssm_scan_seq_map.argtypes = [_vp] * 9
+        lib.ssm_scan_seq_map.restype = st
+        lib.ssm_scan_fold_maps.argtypes = [_vp, ctypes.c_int] + [_vp] * 6
+        lib.ssm_scan_fold_maps.restype = st
         lib.ssm_scan_step.argtypes = [_vp] * 12
         lib.ssm_scan_step.restype = st
         lib.ssm_scan_bwd.argtypes = [_vp] * 22
@@ -104,6 +126,9 @@ def load_library(path: str | None = None):
         lib.ssm_probe_peak.argtypes = [ctypes.c_int, ctypes.c_int64, ctypes.c_int, _vp,
                                        ctypes.POINTER(ctypes.c_int64), _vp]
         lib.ssm_probe_peak.restype = st
+        lib.ssm_scan_list_variants.argtypes = [ctypes.c_int, ctypes.c_int,
+                                               ctypes.POINTER(Variant), ctypes.c_int]
+        lib.ssm_scan_list_variants.restype = ctypes.c_int
         _lib = lib
         return lib
 
@@ -175,8 +200,9 @@ class Plan:
         _check(self._lib.ssm_scan_get_info(self._h, ctypes.byref(i)), "ssm_scan_get_info")
         return i.as_dict()
 
-    def set_config(self, lanes_per_chan=0, warps_per_cta=0, grid=0, tile_t=0):
-        c = Config(lanes_per_chan, warps_per_cta, grid, tile_t)
+    def set_config(self, lanes_per_chan=0, warps_per_cta=0, grid=0, tile_t=0,
+                   chans_per_lane=0, segments=0):
+        c = Config(lanes_per_chan, warps_per_cta, grid, tile_t, chans_per_lane, segments)
         _check(self._lib.ssm_scan_set_config(self._h, ctypes.byref(c)), "ssm_scan_set_config")
 
     def set_debug(self, wait_timeout_ns=0, drop_unit=-1):
@@ -219,6 +245,84 @@ class Plan:
                                     _ptr(h_last), _stream(dev))
         _check(rc, "ssm_scan_fwd")
         return y, h_last
+
+    def fwd_conv(self, x_in, conv_w, delta, A, B, C, conv_b=None, D=None, z=None,
+                 delta_bias=None, h0=None, y=None, h_last=None, x_conv=None):
+        """Forward pass with the causal conv front-end of the x branch: x_in
+        (B, L, D) in_dtype, conv_w (D, 4) fp32, conv_b (D,) fp32.  x_conv,
+        when given ((B, L, D) out dtype), receives silu(conv(x_in)).
+        Returns (y, h_last)."""
+        d, f, dev = self.desc, self.flags, self.device
+        if not f & CONV_X:
+            raise ValueError("the plan was created without CONV_X")
+        Bz, L, Dm, N = d.batch, d.seqlen, d.dim, d.dstate
+        _need(x_in, "x_in", (Bz, L, Dm), self.in_dtype, dev)
+        _need(conv_w, "conv_w", (Dm, CONV_WIDTH), torch.float32, dev)
+        _need(conv_b, "conv_b", (Dm,), torch.float32, dev)
+        _need(delta, "delta", (Bz, L, Dm), self.in_dtype, dev)
+        _need(A, "A", (Dm, N), torch.float32, dev)
+        _need(D, "D", (Dm,), torch.float32, dev)
+        _need(z, "z", (Bz, L, Dm), self.in_dtype, dev)
+        _need(delta_bias, "delta_bias", (Dm,), torch.float32, dev)
+        _need(h0, "h0", (Bz, Dm, N), torch.float32, dev)
+        _need(B, "B", (Bz, L, N), self.in_dtype, dev)
+        _need(C, "C", (Bz, L, N), self.in_dtype, dev)
+        if y is None:
+            y = torch.empty((Bz, L, Dm), dtype=self.out_dtype, device=dev)
+        _need(y, "y", (Bz, L, Dm), self.out_dtype, dev)
+        if f & WANT_HLAST and h_last is None:
+            h_last = torch.empty((Bz, Dm, N), dtype=torch.float32, device=dev)
+        _need(h_last, "h_last", (Bz, Dm, N), torch.float32, dev)
+        _need(x_conv, "x_conv", (Bz, L, Dm), self.out_dtype, dev)
+        rc = self._lib.ssm_scan_fwd_conv(self._h, _ptr(x_in), _ptr(conv_w), _ptr(conv_b),
+                                         _ptr(delta), _ptr(delta_bias), _ptr(A), _ptr(B),
+                                         _ptr(C), _ptr(D), _ptr(z), _ptr(h0), _ptr(y),
+                                         _ptr(h_last), _ptr(x_conv), _stream(dev))
+        _check(rc, "ssm_scan_fwd_conv")
+        return y, h_last
+
+    def seq_map(self, x, delta, A, B, delta_bias=None, map_h=None, map_s=None):
+        """Map of the plan's whole sequence: (map_h (B, D, N) = the state
+        reached from 0, map_s (B, D) = the sum of Delta), fp32."""
+        d, dev = self.desc, self.device
+        Bz, L, Dm, N = d.batch, d.seqlen, d.dim, d.dstate
+        _need(x, "x", (Bz, L, Dm), self.in_dtype, dev)
+        _need(delta, "delta", (Bz, L, Dm), self.in_dtype, dev)
+        _need(A, "A", (Dm, N), torch.float32, dev)
+        _need(B, "B", (Bz, L, N), self.in_dtype, dev)
+        _need(delta_bias, "delta_bias", (Dm,), torch.float32, dev)
+        if map_h is None:
+            map_h = torch.empty((Bz, Dm, N), dtype=torch.float32, device=dev)
+        if map_s is None:
+            map_s = torch.empty((Bz, Dm), dtype=torch.float32, device=dev)
+        _need(map_h, "map_h", (Bz, Dm, N), torch.float32, dev)
+        _need(map_s, "map_s", (Bz, Dm), torch.float32, dev)
+        _check(self._lib.ssm_scan_seq_map(self._h, _ptr(x), _ptr(delta), _ptr(delta_bias),
+                                          _ptr(A), _ptr(B), _ptr(map_h), _ptr(map_s),
+                                          _stream(dev)), "ssm_scan_seq_map")
+        return map_h, map_s
+
+    def fold_maps(self, count, maps_h, maps_s, A, h0=None, h_out=None):
+        """Compose the first `count` maps (maps_h (>= count, B, D, N), maps_s
+        (>= count, B, D)) in order onto h0 (None = 0); returns h (B, D, N)."""
+        d, dev = self.desc, self.device
+        Bz, Dm, N = d.batch, d.dim, d.dstate
+        _need(A, "A", (Dm, N), torch.float32, dev)
+        _need(h0, "h0", (Bz, Dm, N), torch.float32, dev)
+        for name, t, tail in (("maps_h", maps_h, (Bz, Dm, N)), ("maps_s", maps_s, (Bz, Dm))):
+            if count > 0:
+                if t.dtype != torch.float32 or t.device != dev or not t.is_contiguous() or \
+                        tuple(t.shape[1:]) != tail or t.shape[0] < count:
+                    raise ValueError(f"{name} must be contiguous fp32 (>= {count}, {tail})")
+        if h_out is None:
+            h_out = torch.empty((Bz, Dm, N), dtype=torch.float32, device=dev)
+        _need(h_out, "h_out", (Bz, Dm, N), torch.float32, dev)
+        _check(self._lib.ssm_scan_fold_maps(self._h, int(count),
+                                            _ptr(maps_h) if count > 0 else None,
+                                            _ptr(maps_s) if count > 0 else None, _ptr(A),
+                                            _ptr(h0), _ptr(h_out), _stream(dev)),
+               "ssm_scan_fold_maps")
+        return h_out
 
     def bwd(self, x, delta, A, B, C, dy, D=None, z=None, delta_bias=None, h0=None,
             dh_last=None, want_dh0=True):
@@ -280,6 +384,16 @@ class Plan:
         return y
 
 
+def list_variants(in_dtype=torch.bfloat16, out_dtype=None) -> list:
+    """The compiled variants of the fused kernel for a dtype pair (dicts)."""
+    lib = load_library()
+    a, b = _TORCH_TO_SSM[in_dtype], _TORCH_TO_SSM[out_dtype or in_dtype]
+    n = lib.ssm_scan_list_variants(a, b, None, 0)
+    arr = (Variant * max(n, 1))()
+    lib.ssm_scan_list_variants(a, b, arr, n)
+    return [arr[i].as_dict() for i in range(n)]
+
+
 def probe_peak(kind: int, iters: int, blocks: int, sink, stream=None) -> int:
     """Launch the library's throughput probe (kind 0 = ex2.approx, 1 = fp32
     FMA) on the current stream; returns the operation count it launched."""
@@ -293,12 +407,12 @@ def probe_peak(kind: int, iters: int, blocks: int, sink, stream=None) -> int:
 
 
 def flags_for(*, z=None, D=None, delta_bias=None, h0=None, delta_softplus=True,
-              want_h_last=True, zoh=False) -> int:
+              want_h_last=True, zoh=False, conv=False) -> int:
     return ((HAS_Z if z is not None else 0) | (HAS_D if D is not None else 0)
             | (DELTA_SOFTPLUS if delta_softplus else 0)
             | (HAS_DELTA_BIAS if delta_bias is not None else 0)
             | (HAS_H0 if h0 is not None else 0) | (WANT_HLAST if want_h_last else 0)
-            | (ZOH if zoh else 0))
+            | (ZOH if zoh else 0) | (CONV_X if conv else 0))
 
 
 _plans: dict = {}

@@ -4,7 +4,8 @@
 // the pages' third pillar, recomputation instead of storing the (B, L, D, N)
 // states, "Tai sao chi parallel scan van chua du nhanh?").
 //
-// Four lanes share one channel (b, d) and split its N states.  Pass 1 runs
+// Four lanes share one channel (b, d) and split its N states.  The chunk's
+// states stay in registers (its loops are unrolled).  Pass 1 runs
 // the recurrence forward and checkpoints the state at the start of every
 // chunk of K tokens (the only state written to HBM: B*D*ceil(L/K)*N floats).
 // Pass 2 walks the chunks backwards: it recomputes the chunk's K + 1 states
@@ -12,9 +13,10 @@
 // chunk's end, carrying g = dL/dh_t (g <- g * Abar_t after each token).
 // Gradients of per-channel parameters (A, D, bias) are summed in registers
 // and added once per thread; gradients of the per-token B_t, C_t (shared by
-// every channel) are added with atomics.  This is the correctness-first form
-// of the backward: it costs three exps per state update (forward pass,
-// recomputation, reverse) and keeps the chunk's states in local memory.
+// every channel) are first summed over the warp's channels by a shuffle
+// reduce-scatter, then added with one atomic per (token, state) and warp.
+// It costs three exps per state update (forward pass, recomputation,
+// reverse).
 #include "device_common.cuh"
 #include "scan_bwd.h"
 
@@ -32,6 +34,28 @@ __device__ __forceinline__ float group_sum(float v) {
 #pragma unroll
   for (int m = TPC / 2; m >= 1; m >>= 1) v += __shfl_xor_sync(FULL_MASK, v, m);
   return v;
+}
+
+// Reduce-scatter over the G = 32 / TPC channels of a warp that hold the same
+// state group: on entry every lane holds V values (its channel's
+// contributions to V per-token sums), on exit lane (channel c) holds the sum
+// over the warp's channels of value c (c < V).  log2(G) rounds of shuffles
+// across lanes TPC, 2 TPC, ... apart.
+template <int TPC, int V>
+__device__ __forceinline__ float channel_reduce_scatter(float (&v)[V], int c) {
+  constexpr int G = 32 / TPC;
+  static_assert(V == G, "one value per channel of the warp");
+#pragma unroll
+  for (int m = G / 2; m >= 1; m >>= 1) {
+    const bool upper = (c & m) != 0;
+#pragma unroll
+    for (int i = 0; i < m; ++i) {
+      const float send = upper ? v[i] : v[i + m];
+      const float keep = upper ? v[i + m] : v[i];
+      v[i] = keep + __shfl_xor_sync(FULL_MASK, send, m * TPC);
+    }
+  }
+  return v[0];
 }
 
 template <typename InT, typename GradT, int NPL, int TPC, int K>
@@ -88,23 +112,33 @@ __global__ void __launch_bounds__(128) bwd_kernel(const BwdParams p) {
     dA_acc[i] = 0.f;
   }
   float dD_acc = 0.f, dbias_acc = 0.f;
-  float hs[K + 1][NPL];  // this lane's states h_{t0} .. h_{t1} of the chunk
+  // channel of this lane within the warp, for the dB / dC reduction
+  constexpr int G = 32 / TPC;
+  constexpr bool kWarpRed = 2 * NPL <= G;  // the warp's channels reduce dB, dC first
+  const int cw = (threadIdx.x & 31) / TPC;
+  float hs[K + 1][NPL];  // this lane's states h_{t0} .. h_{t1} of the chunk (registers:
+                         // the chunk loops are unrolled, tokens past the end skipped)
   for (int c = nck - 1; c >= 0; --c) {
     const int t0 = c * K, t1 = min(L, t0 + K);
 #pragma unroll
     for (int i = 0; i < NPL; ++i) hs[0][i] = on[i] ? ck[(size_t)c * N + i] : 0.f;
-    for (int t = t0; t < t1; ++t) {
-      const int k = t - t0;
-      const float xv = active ? ldb<InT>(p.x, idx(t)) : 0.f;
-      const float dt = active ? delta_of(ldb<InT>(p.dt, idx(t)) + bias) : 0.f;
 #pragma unroll
-      for (int i = 0; i < NPL; ++i)
-        hs[k + 1][i] = on[i] ? fmaf(ex2_approx(dt * A2[i]), hs[k][i],
-                                    dt * ldb<InT>(p.B, tok(t) + i) * xv)
-                             : 0.f;
+    for (int k = 0; k < K; ++k) {
+      const int t = t0 + k;
+      if (t < t1) {
+        const float xv = active ? ldb<InT>(p.x, idx(t)) : 0.f;
+        const float dt = active ? delta_of(ldb<InT>(p.dt, idx(t)) + bias) : 0.f;
+#pragma unroll
+        for (int i = 0; i < NPL; ++i)
+          hs[k + 1][i] = on[i] ? fmaf(ex2_approx(dt * A2[i]), hs[k][i],
+                                      dt * ldb<InT>(p.B, tok(t) + i) * xv)
+                               : 0.f;
+      }
     }
-    for (int t = t1 - 1; t >= t0; --t) {
-      const int k = t - t0;
+#pragma unroll
+    for (int k = K - 1; k >= 0; --k) {
+      const int t = t0 + k;
+      if (t >= t1) continue;  // (uniform over the warp: every lane has the same t1)
       const size_t i0 = idx(t), j = tok(t);
       const float xv = active ? ldb<InT>(p.x, i0) : 0.f;
       const float v = active ? ldb<InT>(p.dt, i0) + bias : 0.f;
@@ -124,20 +158,46 @@ __global__ void __launch_bounds__(128) bwd_kernel(const BwdParams p) {
       }
       dD_acc = fmaf(ds, xv, dD_acc);
       float dxp = 0.f, ddtp = 0.f;
+      // this channel's shares of dC_t and dB_t (NPL states each); summed over
+      // the warp's channels below, then one atomic per (token, state) and warp
+      float red[kWarpRed ? G : 2 * NPL];
+#pragma unroll
+      for (int i = 0; i < (kWarpRed ? G : 2 * NPL); ++i) red[i] = 0.f;
 #pragma unroll
       for (int i = 0; i < NPL; ++i) {
         if (on[i]) {
           const float Cn = ldb<InT>(p.C, j + i), Bn = ldb<InT>(p.B, j + i);
           const float abar = ex2_approx(dt * A2[i]);
-          atomicAdd(p.dC + j + i, ds * hs[k + 1][i]);
+          red[i] = ds * hs[k + 1][i];
           g[i] = fmaf(ds, Cn, g[i]);
           const float dabar = g[i] * hs[k][i];
           ddtp += dabar * abar * An[i] + g[i] * Bn * xv;
           dA_acc[i] = fmaf(dabar * abar, dt, dA_acc[i]);
-          atomicAdd(p.dB + j + i, g[i] * dt * xv);
+          red[NPL + i] = g[i] * dt * xv;
           dxp = fmaf(g[i] * dt, Bn, dxp);
           g[i] *= abar;
         }
+      }
+      bool reduced = false;
+      if constexpr (kWarpRed) {
+        if (p.warp_uniform_b) {
+          // lane of channel cw ends with value cw summed over the warp's
+          // channels (values 0..NPL-1 are dC, NPL..2NPL-1 are dB of its
+          // states); every channel of the warp belongs to one batch element
+          const float tot = channel_reduce_scatter<TPC, G>(red, cw);
+          const int i = cw < NPL ? cw : cw - NPL;
+          if (active && cw < 2 * NPL && q * NPL + i < N)
+            atomicAdd((cw < NPL ? p.dC : p.dB) + j + i, tot);
+          reduced = true;
+        }
+      }
+      if (!reduced) {
+#pragma unroll
+        for (int i = 0; i < NPL; ++i)
+          if (on[i]) {
+            atomicAdd(p.dC + j + i, red[i]);
+            atomicAdd(p.dB + j + i, red[NPL + i]);
+          }
       }
       const float dxi = group_sum<TPC>(dxp) + ds * Dd;
       const float ddt = group_sum<TPC>(ddtp);
@@ -164,8 +224,11 @@ __global__ void __launch_bounds__(128) bwd_kernel(const BwdParams p) {
 }
 
 template <typename InT, typename GradT, int NPL, int TPC>
-static void launch_bwd_variant(const BwdParams &p, cudaStream_t stream) {
+static void launch_bwd_variant(BwdParams p, cudaStream_t stream) {
   const long long threads = (long long)p.Bsz * p.D * TPC;
+  // a warp holds 32 / TPC consecutive channels: one batch element when D is
+  // a multiple of that
+  p.warp_uniform_b = p.D % (32 / TPC) == 0;
   bwd_kernel<InT, GradT, NPL, TPC, kBwdChunk>
       <<<(unsigned)((threads + 127) / 128), 128, 0, stream>>>(p);
 }

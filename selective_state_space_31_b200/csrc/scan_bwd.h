@@ -16,6 +16,7 @@ struct BwdParams {
   const float *A, *Dv, *bias, *h0, *dh_last;
   float *dx, *ddelta, *dz, *dB, *dC, *dA, *dD, *dbias, *dh0;
   float *ws_ck;                          // B * D * ceil(L / kBwdChunk) * N checkpoints
+  bool warp_uniform_b;                   // every warp's channels share one batch element
 };
 cudaError_t launch_bwd(const BwdParams &p, cudaStream_t stream);
 

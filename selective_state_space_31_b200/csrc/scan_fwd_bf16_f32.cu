@@ -1,0 +1,29 @@
+// scan_fwd_bf16_f32.cu -- compiled variants of the fused forward kernel for bf16 inputs, fp32 outputs
+// (the variant tables are split over translation units so they compile in
+// parallel).
+#include "scan_fwd_kernel.cuh"
+#include "scan_fwd_variants.h"
+
+namespace ssm {
+
+cudaError_t fwd_table_bf16_f32(const LaunchShape *ls, const TmaMaps *maps, const FwdParams *p,
+                           cudaStream_t st, VariantInfo *vi) {
+#define SSM_X(NS, LPC, KC, W, TT, ZOH, CARRY, CONV)                                    \
+  if (shape_is(ls, NS, LPC, KC, W, TT, ZOH, CARRY, CONV))                               \
+    return run_variant<__nv_bfloat16, float, NS, LPC, KC, W, TT, ZOH, CARRY, CONV>(ls, maps, p, st, vi);
+  SSM_FWD_BF16_F32(SSM_X)
+#undef SSM_X
+  return cudaErrorNotSupported;
+}
+
+int fwd_list_bf16_f32(VariantDesc *out, int max) {
+  int n = 0;
+#define SSM_X(NS, LPC, KC, W, TT, ZOH, CARRY, CONV)                                    \
+  if (n < max) out[n] = VariantDesc{NS, LPC, KC, W, TT, ZOH, CARRY, CONV};             \
+  ++n;
+  SSM_FWD_BF16_F32(SSM_X)
+#undef SSM_X
+  return n;
+}
+
+}  // namespace ssm

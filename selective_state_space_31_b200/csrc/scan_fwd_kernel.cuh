@@ -12,35 +12,45 @@
 //
 // Work decomposition
 //   * A "row" is DT consecutive channels of one batch element; its L tokens
-//     are cut into stages of TT tokens.  A channel's N states are split over
-//     LPC lanes (NPL = N / LPC each); the lanes' partial readouts of a group
-//     of LPC tokens are combined by a shuffle butterfly that leaves lane q with
+//     are cut into stages of TT tokens.  A lane owns KC adjacent channels
+//     (1 or 2) and NPL = N / LPC of their states, so LPC lanes share a
+//     channel group; with two channels a lane loads and widens each B_t / C_t
+//     value once for both.  The lanes' partial readouts of a group of LPC
+//     tokens are combined by a shuffle butterfly that leaves lane q with
 //     token q, and lane q finishes that token.
-//   * Ticket schedule.  Each row's S stages are cut into parts of PL stages;
-//     item i = part * R + row.  A CTA's load warp takes item numbers in
-//     increasing order from a device counter (one atomic per item), so the
-//     predecessor of an item (same row, previous part, number i - R) always
-//     went to a CTA that was already running: every wait for a carried state
-//     ends, however few CTAs the device runs at once, and CTAs that finish
-//     early simply take more items.  A part hands its final state to the next
-//     part through a per-(row, warp) flag carrying the stage index and a
-//     launch epoch (release/acquire) -- the pages' associative carry ("Scan
-//     bien recurrence ...": (A2,b2) (x) (A1,b1) = (A2A1, A2b1+b2)): the state
-//     after one part is the exact starting state of the next.  Every wait is
-//     bounded by a timer.
+//   * Segments.  A row's stages may be cut into M segments that run at the
+//     same time.  Segment k > 0 starts from the exact state at its first
+//     token, obtained with the pages' associative composition ("Scan bien
+//     recurrence ...": (A2,b2) (x) (A1,b1) = (A2A1, A2b1+b2)): a carry pass
+//     (this kernel with CARRY set) scans every sub-chunk of the earlier
+//     segments from h = 0 and records its map (prod Abar, h_end), where
+//     prod_t exp(Delta_t A) = exp(A sum_t Delta_t) needs only the sum of
+//     Delta; the segment's first part folds those maps onto h0.  Long
+//     sequences gain parallelism this way at the cost of a second exponential
+//     for the tokens of the earlier segments.
+//   * Ticket schedule.  Each segment's stages are cut into parts of PL
+//     stages; item i = part * VR + (row, segment) with VR = rows * M.  A
+//     CTA's load warp takes item numbers in increasing order from a device
+//     counter (one atomic per item), so the predecessor of an item (same row
+//     and segment, previous part, number i - VR) always went to a CTA that
+//     was already running: every wait for a carried state ends, however few
+//     CTAs the device runs at once, and CTAs that finish early simply take
+//     more items.  A part hands its final state to the next part through a
+//     per-(row, segment, warp) flag carrying the stage index and a launch
+//     epoch (release/acquire): the state after one part is the exact starting
+//     state of the next.  Every wait is bounded by a timer.
 //   * One load warp streams the stages' [TT, DT] tiles of x / delta / z and
 //     [TT, N] tiles of B / C into a ring of RAW shared-memory slots with TMA
 //     (cp.async.bulk.tensor, every CTA loads its own tiles); slot full / slot
 //     empty mbarriers are the only coupling between warps.  Each scan warp
 //     does all the per-token work of its own channels: lane q of a channel
-//     prepares tokens q, q + LPC, ... (Delta, Delta*x into a warp-private
-//     plane that the channel's LPC lanes read back; silu(z) and D*x*silu(z)
-//     stay in the registers of the lane that finishes those very tokens),
-//     scans, and stores y straight from registers.  B / C are read as stored
-//     (bf16 words are widened with integer ops), which halves the
-//     shared-memory wavefronts of the scan loop against fp32 staging.
-//     Tokens past the end get Delta = 0, an identity update, so carried
-//     states are exact for ragged tails.
+//     group prepares tokens q, q + LPC, ... (Delta, Delta*x into a
+//     warp-private plane that the group's LPC lanes read back; silu(z) and
+//     D*x*silu(z) stay in the registers of the lane that finishes those very
+//     tokens), scans, and stores y straight from registers.  B / C are read
+//     as stored (bf16 words are widened with integer ops).  Tokens past the
+//     end get Delta = 0, an identity update, so carried states are exact for
+//     ragged tails.
 #pragma once
 
 #include "device_common.cuh"
@@ -51,35 +61,47 @@ namespace ssm {
 constexpr int align_up(int v, int a) { return (v + a - 1) / a * a; }
 constexpr int clamp_int(int v, int lo, int hi) { return v < lo ? lo : (v > hi ? hi : v); }
 
-template <typename InT, typename OutT, int NS, int LPC, int WARPS, int TT>
+template <typename InT, typename OutT, int NS, int LPC, int KC, int WARPS, int TT,
+          bool CONV = false>
 struct FwdCfg {
-  static constexpr int NPL = NS / LPC;    // states per lane
-  static constexpr int DTW = 32 / LPC;    // channels per scan warp
+  static constexpr int NPL = NS / LPC;    // states per lane and channel
+  static constexpr int GPW = 32 / LPC;    // channel groups per scan warp
+  static constexpr int DTW = GPW * KC;    // channels per scan warp
   static constexpr int DT = WARPS * DTW;  // channels per row tile
   static constexpr int TPL = TT / LPC;    // tokens a lane prepares and finishes per stage
   static constexpr int THREADS = (WARPS + 1) * 32;  // scan warps + the load warp
+  // the conv front-end reads the x branch from kConvWidth tokens before the
+  // stage on (zero-filled by TMA before the sequence)
+  static constexpr int XHALO = CONV ? kConvWidth : 0;
   static constexpr int XTILE = align_up(TT * DT * (int)sizeof(InT), 128);
+  static constexpr int XTILE_X = align_up((TT + XHALO) * DT * (int)sizeof(InT), 128);
   static constexpr int BCTILE = align_up(TT * NS * (int)sizeof(InT), 128);
-  static constexpr int SLOT = 3 * XTILE + 2 * BCTILE;
+  static constexpr int OFF_DT = XTILE_X, OFF_Z = XTILE_X + XTILE, OFF_B = XTILE_X + 2 * XTILE,
+                       OFF_C = OFF_B + BCTILE;
+  static constexpr int SLOT = OFF_C + BCTILE;
   // ring depth: ~128 tokens of prefetch, within ~64 KB, at least 3 slots
   static constexpr int RAW = clamp_int(65536 / SLOT, 3, 128 / TT > 3 ? 128 / TT : 3);
-  // (Delta, Delta*x) per warp, channel-major: row c holds tokens 0..TT-1 of
-  // channel c, rows TTP float2 apart (TTP - TT spreads the rows over the
-  // shared-memory banks; TTP even keeps token pairs 16-byte aligned)
-  static constexpr int TTP = TT + (LPC > 2 ? LPC : 2);
-  static constexpr int PLANE = align_up(TTP * DTW * 8, 128);
+  // Per warp, channel-group-major plane of per-token values: KC = 1 keeps
+  // (Delta, Delta*x) as a float2, KC = 2 (Delta0, Delta1, Delta*x0, Delta*x1)
+  // as a float4.  Row g holds tokens 0..TT-1 of group g; the TTP - TT pad
+  // spreads the rows and the prologue's writes over the shared-memory banks.
+  static constexpr int ESZ = 8 * KC;  // bytes per token and group
+  static constexpr int TTP = KC == 1 ? TT + (LPC > 2 ? LPC : 2) : TT + (LPC > 1 ? LPC : 2);
+  static constexpr int PLANE = align_up(TTP * GPW * ESZ, 128);
   static constexpr int OFF_PLANE = RAW * SLOT;
   static constexpr int OFF_BAR = OFF_PLANE + WARPS * PLANE;
   static constexpr int SMEM = OFF_BAR + 2 * RAW * 8;
   static_assert(NS % LPC == 0, "LPC must divide N");
   static_assert(TT % LPC == 0, "LPC must divide the stage length");
+  static_assert(KC == 1 || KC == 2, "one or two channels per lane");
+  static_assert(KC == 1 || NPL % 2 == 0, "two channels per lane pair up their states");
   static_assert(DT * (int)sizeof(InT) % 16 == 0, "TMA rows need 16-byte multiples");
   static_assert(SLOT % 128 == 0 && OFF_PLANE % 128 == 0, "slot alignment");
 };
 
-// Butterfly reduce-scatter over the LPC lanes of a channel: on entry lane q
-// holds partial sums v[j] (its NPL states) of the group's LPC tokens; on exit
-// it returns the full sum (all N states) of token q.
+// Butterfly reduce-scatter over the LPC lanes of a channel group: on entry
+// lane q holds partial sums v[j] (its NPL states) of the group's LPC tokens;
+// on exit it returns the full sum (all N states) of token q.
 template <int LPC>
 __device__ __forceinline__ float reduce_scatter(float (&v)[LPC], int q) {
 #pragma unroll
@@ -90,6 +112,23 @@ __device__ __forceinline__ float reduce_scatter(float (&v)[LPC], int q) {
       const float send = upper ? v[i] : v[i + m];
       const float keep = upper ? v[i + m] : v[i];
       v[i] = keep + __shfl_xor_sync(FULL_MASK, send, m);
+    }
+  }
+  return v[0];
+}
+// The same for a lane's two channels at once (.x and .y).
+template <int LPC>
+__device__ __forceinline__ float2 reduce_scatter2(float2 (&v)[LPC], int q) {
+#pragma unroll
+  for (int m = LPC / 2; m >= 1; m >>= 1) {
+    const bool upper = (q & m) != 0;
+#pragma unroll
+    for (int i = 0; i < m; ++i) {
+      const float2 send = upper ? v[i] : v[i + m];
+      const float2 keep = upper ? v[i + m] : v[i];
+      const float2 got = make_float2(__shfl_xor_sync(FULL_MASK, send.x, m),
+                                     __shfl_xor_sync(FULL_MASK, send.y, m));
+      v[i] = fadd2(keep, got);
     }
   }
   return v[0];
@@ -140,26 +179,54 @@ __device__ __forceinline__ void load_bc(const __nv_bfloat16 *src, float (&dst)[N
   }
 }
 
-// Position of one stage of work: item (row, part) and stage index, derived
-// from an item number once per item (a division happens only there).
+// Two adjacent channels' values of one token (x, delta or z) as fp32.
+__device__ __forceinline__ float2 load_pair(const float *src) {
+  return *reinterpret_cast<const float2 *>(src);
+}
+__device__ __forceinline__ float2 load_pair(const __nv_bfloat16 *src) {
+  float2 v;
+  widen_bf16x2(*reinterpret_cast<const uint32_t *>(src), v.x, v.y);
+  return v;
+}
+// Store two adjacent channels' outputs.
+__device__ __forceinline__ void store_pair(float *dst, float2 v) {
+  *reinterpret_cast<float2 *>(dst) = v;
+}
+__device__ __forceinline__ void store_pair(__nv_bfloat16 *dst, float2 v) {
+  *reinterpret_cast<__nv_bfloat162 *>(dst) = __floats2bfloat162_rn(v.x, v.y);
+}
+
+// Position of one stage of work: item (row, segment, part) and its stages,
+// derived from an item number once per item (divisions happen only there).
 struct ItemPos {
-  int item = -1, row = 0, part = 0, b = 0, dtile = 0, st_begin = 0, st_end = 0;
+  int item = -1, row = 0, seg = 0, vrow = 0, part = 0, b = 0, dtile = 0;
+  int seg_begin = 0, seg_end = 0, st_begin = 0, st_end = 0;
   __device__ __forceinline__ void set(int it, const FwdParams &p) {
+    const int VR = p.rows * p.M;
     item = it;
-    part = it / p.rows;
-    row = it - part * p.rows;
-    st_begin = part * p.PL;
-    st_end = min(p.S, st_begin + p.PL);
+    part = it / VR;
+    vrow = it - part * VR;
+    row = vrow / p.M;
+    seg = vrow - row * p.M;
+    seg_begin = seg * p.SPS;
+    seg_end = min(p.S, seg_begin + p.SPS);
+    st_begin = seg_begin + part * p.PL;
+    st_end = min(seg_end, st_begin + p.PL);
     b = row / p.nDT;
     dtile = row - b * p.nDT;
   }
 };
 
-template <typename InT, typename OutT, int NS, int LPC, int WARPS, int TT, bool ZOH>
+// CARRY = false: the fused forward scan.  CARRY = true: the carry pass over
+// sub-chunks of PL stages (items independent, no readout): each item scans
+// its stages from h = 0 and records (sum of Delta, h_end) per channel.
+template <typename InT, typename OutT, int NS, int LPC, int KC, int WARPS, int TT, bool ZOH,
+          bool CARRY, bool CONV>
 __global__ void __launch_bounds__((WARPS + 1) * 32)
     fwd_kernel(const __grid_constant__ TmaMaps maps, const FwdParams p) {
-  using Cfg = FwdCfg<InT, OutT, NS, LPC, WARPS, TT>;
-  constexpr int NPL = Cfg::NPL, DTW = Cfg::DTW, DT = Cfg::DT, RAW = Cfg::RAW, TPL = Cfg::TPL;
+  using Cfg = FwdCfg<InT, OutT, NS, LPC, KC, WARPS, TT, CONV>;
+  constexpr int NPL = Cfg::NPL, GPW = Cfg::GPW, DT = Cfg::DT, RAW = Cfg::RAW,
+                TPL = Cfg::TPL;
   extern __shared__ __align__(1024) unsigned char smem[];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -186,13 +253,9 @@ __global__ void __launch_bounds__((WARPS + 1) * 32)
   if (warp == WARPS) {
     // =================== load warp (one thread issues) ===================
     if (lane == 0) {
-      const uint32_t tx_bytes =
-          (p.has_z ? 3u : 2u) * TT * DT * sizeof(InT) + 2u * TT * NS * sizeof(InT);
-      // Work items are handed out in increasing order from a device counter
-      // (a ticket per item).  An item's predecessor (same row, previous part)
-      // has a smaller number, so it went to a CTA that was already running
-      // when this one took its ticket: waits on carried states always end,
-      // whatever share of the device this launch gets.
+      const bool with_z = !CARRY && p.has_z;
+      const uint32_t tx_bytes = (TT + Cfg::XHALO + (with_z ? 2u : 1u) * TT) * DT * sizeof(InT) +
+                                (CARRY ? 1u : 2u) * TT * NS * sizeof(InT);
       ItemPos iss;
       int st = 0;
       bool ok = true;
@@ -204,25 +267,32 @@ __global__ void __launch_bounds__((WARPS + 1) * 32)
           ok = false;
           break;
         }
-        if (iss.item < 0 || st == iss.st_end) {
+        // next item when this one is done (parts past a short segment's end
+        // have no stages and are skipped)
+        bool done = false;
+        while (iss.item < 0 || st == iss.st_end) {
           const int it = (int)atomicAdd(&p.ctl->ticket, 1u);
-          if (it >= p.items) {  // no work left: end marker, no data
-            slot_work[r] = make_int2(-1, 0);
-            mbar_arrive(&rfull[r]);
+          if (it >= p.items) {
+            done = true;
             break;
           }
           iss.set(it, p);
           st = iss.st_begin;
         }
+        if (done) {  // no work left: end marker, no data
+          slot_work[r] = make_int2(-1, 0);
+          mbar_arrive(&rfull[r]);
+          break;
+        }
         slot_work[r] = make_int2(iss.item, st);
         const int d0 = iss.dtile * DT, t0 = st * TT, b = iss.b;
         unsigned char *sb = smem + r * Cfg::SLOT;
         mbar_arrive_expect_tx(&rfull[r], tx_bytes);
-        tma_load_3d(sb, &maps.x, &rfull[r], d0, t0, b);
-        tma_load_3d(sb + Cfg::XTILE, &maps.dt, &rfull[r], d0, t0, b);
-        if (p.has_z) tma_load_3d(sb + 2 * Cfg::XTILE, &maps.z, &rfull[r], d0, t0, b);
-        tma_load_3d(sb + 3 * Cfg::XTILE, &maps.B, &rfull[r], 0, t0, b);
-        tma_load_3d(sb + 3 * Cfg::XTILE + Cfg::BCTILE, &maps.C, &rfull[r], 0, t0, b);
+        tma_load_3d(sb, &maps.x, &rfull[r], d0, t0 - Cfg::XHALO, b);
+        tma_load_3d(sb + Cfg::OFF_DT, &maps.dt, &rfull[r], d0, t0, b);
+        if (with_z) tma_load_3d(sb + Cfg::OFF_Z, &maps.z, &rfull[r], d0, t0, b);
+        tma_load_3d(sb + Cfg::OFF_B, &maps.B, &rfull[r], 0, t0, b);
+        if (!CARRY) tma_load_3d(sb + Cfg::OFF_C, &maps.C, &rfull[r], 0, t0, b);
         ++st;
       }
       if (!ok) {
@@ -234,14 +304,24 @@ __global__ void __launch_bounds__((WARPS + 1) * 32)
     }
   } else {
     // =================== scan warps ===================
-    const int c_loc = lane / LPC;       // channel within the warp
-    const int q = lane % LPC;           // state group of this lane
-    const int ch = warp * DTW + c_loc;  // channel within the row tile
-    float2 *plane = reinterpret_cast<float2 *>(smem + Cfg::OFF_PLANE + warp * Cfg::PLANE);
-    float h[NPL], A2[NPL], invA[NPL];  // invA: 1/A (0 where A = 0), zero-order hold only
+    const int g_loc = lane / LPC;        // channel group within the warp
+    const int q = lane % LPC;            // state group of this lane
+    const int grp = warp * GPW + g_loc;  // channel group within the row tile
+    const int ch0 = grp * KC;            // first channel of this lane within the row tile
+    unsigned char *plane_base = smem + Cfg::OFF_PLANE + warp * Cfg::PLANE;
+    float h[KC][NPL], A2[KC][NPL], invA[KC][NPL];  // invA: 1/A (0 where A = 0), ZOH only
 #pragma unroll
-    for (int i = 0; i < NPL; ++i) { h[i] = 0.f; A2[i] = 0.f; invA[i] = 0.f; }
-    float bias = 0.f, dsk = 0.f;
+    for (int c = 0; c < KC; ++c)
+#pragma unroll
+      for (int i = 0; i < NPL; ++i) { h[c][i] = 0.f; A2[c][i] = 0.f; invA[c][i] = 0.f; }
+    float bias[KC], dsk[KC], dsum[KC];
+    float cw[KC][CONV ? kConvWidth : 1], cb[KC];  // conv taps and bias of each channel
+#pragma unroll
+    for (int c = 0; c < KC; ++c) {
+      bias[c] = 0.f; dsk[c] = 0.f; dsum[c] = 0.f; cb[c] = 0.f;
+#pragma unroll
+      for (int k = 0; k < (CONV ? kConvWidth : 1); ++k) cw[c][k] = 0.f;
+    }
     OutT *const ybase = reinterpret_cast<OutT *>(p.y);
     ItemPos cur;
     for (int k = 0;; ++k) {
@@ -254,27 +334,54 @@ __global__ void __launch_bounds__((WARPS + 1) * 32)
       const int2 work = slot_work[r];
       if (work.x < 0) break;  // end marker
       if (work.x != cur.item) cur.set(work.x, p);
-      const int row = cur.row, st = work.y, b = cur.b;
-      const int d = cur.dtile * DT + ch;
-      const bool valid_ch = d < p.D;
-      const bool run_start = st == cur.st_begin;
-      if (run_start) {  // per-item parameters and starting state of this lane
+      const int st = work.y, b = cur.b;
+      const int d = cur.dtile * DT + ch0;  // first channel (of KC) in the tensor
+      const bool valid_ch = d < p.D;       // KC = 2: D is even there, so d + 1 < D too
+      if (st == cur.st_begin) {  // per-item parameters and starting state of this lane
 #pragma unroll
-        for (int i = 0; i < NPL; ++i) {
-          const float a = valid_ch ? __ldg(p.A + (size_t)d * NS + q * NPL + i) : 0.f;
-          A2[i] = a * kLog2e;
-          if constexpr (ZOH) invA[i] = a != 0.f ? 1.f / a : 0.f;
+        for (int c = 0; c < KC; ++c) {
+#pragma unroll
+          for (int i = 0; i < NPL; ++i) {
+            const float a = valid_ch ? __ldg(p.A + (size_t)(d + c) * NS + q * NPL + i) : 0.f;
+            A2[c][i] = a * kLog2e;
+            if constexpr (ZOH) invA[c][i] = a != 0.f ? 1.f / a : 0.f;
+          }
+          bias[c] = (p.has_bias && valid_ch) ? __ldg(p.bias + d + c) : 0.f;
+          dsk[c] = (!CARRY && p.has_D && valid_ch) ? __ldg(p.Dv + d + c) : 0.f;
+          dsum[c] = 0.f;
+          if constexpr (CONV) {
+#pragma unroll
+            for (int k = 0; k < kConvWidth; ++k)
+              cw[c][k] = valid_ch ? __ldg(p.conv_w + (size_t)(d + c) * kConvWidth + k) : 0.f;
+            cb[c] = (valid_ch && p.conv_b) ? __ldg(p.conv_b + d + c) : 0.f;
+          }
         }
-        bias = (p.has_bias && valid_ch) ? __ldg(p.bias + d) : 0.f;
-        dsk = (p.has_D && valid_ch) ? __ldg(p.Dv + d) : 0.f;
-        if (st == 0) {
+        if (CARRY || st == cur.seg_begin) {
+          // start of a carry sub-chunk (from 0) or of a segment: h0, then the
+          // maps of all sub-chunks before this segment, in order
 #pragma unroll
-          for (int i = 0; i < NPL; ++i)
-            h[i] = (p.has_h0 && valid_ch)
-                       ? __ldg(p.h0 + ((size_t)b * p.D + d) * NS + q * NPL + i) : 0.f;
-        } else {  // carried state of this row from the CTA that ran the previous part
+          for (int c = 0; c < KC; ++c)
+#pragma unroll
+            for (int i = 0; i < NPL; ++i)
+              h[c][i] = (!CARRY && p.has_h0 && valid_ch)
+                            ? __ldg(p.h0 + ((size_t)b * p.D + d + c) * NS + q * NPL + i) : 0.f;
+          if (!CARRY && cur.seg > 0 && valid_ch) {
+            const int nsub = cur.seg * p.nq;
+            for (int j = 0; j < nsub; ++j) {
+              const size_t base = ((size_t)b * p.nsub_row + j) * p.D + d;
+#pragma unroll
+              for (int c = 0; c < KC; ++c) {
+                const float s = __ldcg(p.agg_s + base + c);
+                const float *ah = p.agg_h + (base + c) * NS + q * NPL;
+#pragma unroll
+                for (int i = 0; i < NPL; ++i)
+                  h[c][i] = fmaf(ex2_approx(A2[c][i] * s), h[c][i], __ldcg(ah + i));
+              }
+            }
+          }
+        } else {  // carried state of this (row, segment) from the CTA that ran the previous part
           const unsigned long long want = ((unsigned long long)epoch << 32) | (unsigned)st;
-          unsigned long long *flag = p.ws_flags + (size_t)row * WARPS + warp;
+          unsigned long long *flag = p.ws_flags + (size_t)cur.vrow * WARPS + warp;
           bool got = ld_acquire_u64(flag) == want;
           if (!got) {
             const uint64_t tstart = globaltimer_ns();
@@ -286,125 +393,266 @@ __global__ void __launch_bounds__((WARPS + 1) * 32)
           }
           if (!__all_sync(FULL_MASK, got) && lane == 0)
             atomicCAS(&p.ctl->status, 0, kStatusTimeout);
-          const float *src = p.ws_state + ((size_t)row * DT + ch) * NS + q * NPL;
 #pragma unroll
-          for (int i = 0; i < NPL; ++i) h[i] = __ldcg(src + i);
+          for (int c = 0; c < KC; ++c) {
+            const float *src = p.ws_state + ((size_t)cur.vrow * DT + ch0 + c) * NS + q * NPL;
+#pragma unroll
+            for (int i = 0; i < NPL; ++i) h[c][i] = __ldcg(src + i);
+          }
         }
       }
 
       const unsigned char *sb = smem + r * Cfg::SLOT;
+      // x rows: token t of the stage is row t + XHALO (conv front-end: rows
+      // t + 1 .. t + 4 are tokens t - 3 .. t)
       const InT *xs = reinterpret_cast<const InT *>(sb);
-      const InT *ds = reinterpret_cast<const InT *>(sb + Cfg::XTILE);
-      const InT *zs = reinterpret_cast<const InT *>(sb + 2 * Cfg::XTILE);
-      const InT *Bs = reinterpret_cast<const InT *>(sb + 3 * Cfg::XTILE);
-      const InT *Cs = reinterpret_cast<const InT *>(sb + 3 * Cfg::XTILE + Cfg::BCTILE);
+      const InT *ds = reinterpret_cast<const InT *>(sb + Cfg::OFF_DT);
+      const InT *zs = reinterpret_cast<const InT *>(sb + Cfg::OFF_Z);
+      const InT *Bs = reinterpret_cast<const InT *>(sb + Cfg::OFF_B);
+      const InT *Cs = reinterpret_cast<const InT *>(sb + Cfg::OFF_C);
       const int t0 = st * TT;
+      OutT *xcrow = CONV && p.xconv
+                        ? reinterpret_cast<OutT *>(p.xconv) + ((size_t)b * p.L + t0) * p.D + d
+                        : nullptr;
       const int nvalid = min(TT, p.L - t0);
+      OutT *yrow = ybase + ((size_t)b * p.L + t0) * p.D + d;
 
-      // -- per-token prologue of this lane's tokens j * LPC + q --
-      float g1[TPL], g2[TPL];
-      if constexpr (TPL % 2 == 0) {
+      if constexpr (KC == 1) {
+        float2 *plane = reinterpret_cast<float2 *>(plane_base);
+        const int ch = ch0;
+        // -- per-token prologue of this lane's tokens j * LPC + q --
+        float g1[CARRY ? 1 : TPL], g2[CARRY ? 1 : TPL];
+        if constexpr (TPL % 2 == 0) {
 #pragma unroll
-        for (int j = 0; j < TPL; j += 2) {
-          const int ta = j * LPC + q, tb = ta + LPC;
-          const float2 xv = make_float2(to_f32(xs[ta * DT + ch]), to_f32(xs[tb * DT + ch]));
-          float2 v = fadd2(make_float2(to_f32(ds[ta * DT + ch]), to_f32(ds[tb * DT + ch])),
-                           make_float2(bias, bias));
-          if (p.softplus) v = softplus_f2(v);
-          if (ta >= nvalid) v.x = 0.f;  // past the end: identity update
-          if (tb >= nvalid) v.y = 0.f;
-          const float2 dx = fmul2(v, xv);
-          // zero-order hold keeps x itself: its input term is not a multiple of Delta
-          plane[c_loc * Cfg::TTP + ta] = make_float2(v.x, ZOH ? xv.x : dx.x);
-          plane[c_loc * Cfg::TTP + tb] = make_float2(v.y, ZOH ? xv.y : dx.y);
-          float2 g = make_float2(1.f, 1.f);
-          if (p.has_z) g = silu_f2(make_float2(to_f32(zs[ta * DT + ch]), to_f32(zs[tb * DT + ch])));
-          const float2 gd = fmul2(fmul2(make_float2(dsk, dsk), xv), g);
-          g1[j] = g.x; g1[j + 1] = g.y;
-          g2[j] = gd.x; g2[j + 1] = gd.y;
+          for (int j = 0; j < TPL; j += 2) {
+            const int ta = j * LPC + q, tb = ta + LPC;
+            float2 xv;
+            if constexpr (CONV) {
+              float2 u = make_float2(cb[0], cb[0]);
+#pragma unroll
+              for (int k = 0; k < kConvWidth; ++k)
+                u = ffma2(make_float2(cw[0][k], cw[0][k]),
+                          make_float2(to_f32(xs[(ta + 1 + k) * DT + ch]),
+                                      to_f32(xs[(tb + 1 + k) * DT + ch])), u);
+              xv = silu_f2(u);
+              if (xcrow && valid_ch && !CARRY) {
+                if (ta < nvalid) xcrow[(size_t)ta * p.D] = from_f32<OutT>(xv.x);
+                if (tb < nvalid) xcrow[(size_t)tb * p.D] = from_f32<OutT>(xv.y);
+              }
+            } else {
+              xv = make_float2(to_f32(xs[ta * DT + ch]), to_f32(xs[tb * DT + ch]));
+            }
+            float2 v = fadd2(make_float2(to_f32(ds[ta * DT + ch]), to_f32(ds[tb * DT + ch])),
+                             make_float2(bias[0], bias[0]));
+            if (p.softplus) v = softplus_f2(v);
+            if (ta >= nvalid) v.x = 0.f;  // past the end: identity update
+            if (tb >= nvalid) v.y = 0.f;
+            const float2 dx = fmul2(v, xv);
+            // zero-order hold keeps x itself: its input term is not a multiple of Delta
+            plane[g_loc * Cfg::TTP + ta] = make_float2(v.x, ZOH ? xv.x : dx.x);
+            plane[g_loc * Cfg::TTP + tb] = make_float2(v.y, ZOH ? xv.y : dx.y);
+            if constexpr (!CARRY) {
+              float2 g = make_float2(1.f, 1.f);
+              if (p.has_z)
+                g = silu_f2(make_float2(to_f32(zs[ta * DT + ch]), to_f32(zs[tb * DT + ch])));
+              const float2 gd = fmul2(fmul2(make_float2(dsk[0], dsk[0]), xv), g);
+              g1[j] = g.x; g1[j + 1] = g.y;
+              g2[j] = gd.x; g2[j + 1] = gd.y;
+            }
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < TPL; ++j) {
+            const int ta = j * LPC + q;
+            float xv;
+            if constexpr (CONV) {
+              float u = cb[0];
+#pragma unroll
+              for (int k = 0; k < kConvWidth; ++k)
+                u = fmaf(cw[0][k], to_f32(xs[(ta + 1 + k) * DT + ch]), u);
+              xv = silu_f(u);
+              if (xcrow && valid_ch && !CARRY && ta < nvalid)
+                xcrow[(size_t)ta * p.D] = from_f32<OutT>(xv);
+            } else {
+              xv = to_f32(xs[ta * DT + ch]);
+            }
+            float v = to_f32(ds[ta * DT + ch]) + bias[0];
+            if (p.softplus) v = softplus_f(v);
+            if (ta >= nvalid) v = 0.f;
+            plane[g_loc * Cfg::TTP + ta] = make_float2(v, ZOH ? xv : v * xv);
+            if constexpr (!CARRY) {
+              const float g = p.has_z ? silu_f(to_f32(zs[ta * DT + ch])) : 1.f;
+              g1[j] = g;
+              g2[j] = dsk[0] * xv * g;
+            }
+          }
+        }
+        __syncwarp();
+
+        // -- the scan over TT tokens of this lane's channel --
+        const float2 *prow = plane + g_loc * Cfg::TTP;
+        float4 dpair;  // (Delta, Delta*x) of an even token and the next, one 16-byte load
+#pragma unroll
+        for (int tt = 0; tt < TT; tt += LPC) {
+          float yp[LPC];
+#pragma unroll
+          for (int j = 0; j < LPC; ++j) {
+            const int t = tt + j;
+            if ((t & 1) == 0) dpair = *reinterpret_cast<const float4 *>(prow + t);
+            const float2 dd =
+                (t & 1) ? make_float2(dpair.z, dpair.w) : make_float2(dpair.x, dpair.y);
+            if constexpr (CARRY) dsum[0] += dd.x;
+            float bv[NPL], cv[NPL];
+            load_bc<NPL>(Bs + t * NS + q * NPL, bv);
+            if constexpr (!CARRY) load_bc<NPL>(Cs + t * NS + q * NPL, cv);
+            if constexpr (NPL % 2 == 0) {
+              const float2 dA = make_float2(dd.x, dd.x), dX = make_float2(dd.y, dd.y);
+              float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+              for (int i = 0; i < NPL; i += 2) {
+                const float2 arg = fmul2(dA, make_float2(A2[0][i], A2[0][i + 1]));
+                const float2 a = make_float2(ex2_approx(arg.x), ex2_approx(arg.y));
+                float2 bx = fmul2(dX, make_float2(bv[i], bv[i + 1]));
+                if constexpr (ZOH)  // dX holds x: Bbar x = ((e^u - 1) / A) * (B x)
+                  bx = fmul2(zoh_coef2(fmul2(arg, make_float2(kLn2, kLn2)), a, dA,
+                                       make_float2(invA[0][i], invA[0][i + 1])),
+                             bx);
+                const float2 hn = ffma2(a, make_float2(h[0][i], h[0][i + 1]), bx);
+                h[0][i] = hn.x;
+                h[0][i + 1] = hn.y;
+                if constexpr (!CARRY) acc = ffma2(make_float2(cv[i], cv[i + 1]), hn, acc);
+              }
+              yp[j] = acc.x + acc.y;
+            } else {
+              const float arg = dd.x * A2[0][0];
+              const float a = ex2_approx(arg);
+              float bx = dd.y * bv[0];
+              if constexpr (ZOH) bx *= zoh_coef(arg * kLn2, a, dd.x, invA[0][0]);
+              h[0][0] = fmaf(a, h[0][0], bx);
+              yp[j] = CARRY ? 0.f : cv[0] * h[0][0];
+            }
+          }
+          if constexpr (!CARRY) {
+            const float ys = reduce_scatter<LPC>(yp, q);
+            const int to = tt + q;  // this lane's own token of the group: prologue slot tt / LPC
+            if (to < nvalid && valid_ch)
+              yrow[(size_t)to * p.D] = from_f32<OutT>(fmaf(ys, g1[tt / LPC], g2[tt / LPC]));
+          }
         }
       } else {
+        // ------------- two channels per lane: ch0 and ch0 + 1 -------------
+        float4 *plane = reinterpret_cast<float4 *>(plane_base);
+        float2 g1[CARRY ? 1 : TPL], g2[CARRY ? 1 : TPL];
 #pragma unroll
         for (int j = 0; j < TPL; ++j) {
           const int ta = j * LPC + q;
-          const float xv = to_f32(xs[ta * DT + ch]);
-          float v = to_f32(ds[ta * DT + ch]) + bias;
-          if (p.softplus) v = softplus_f(v);
-          if (ta >= nvalid) v = 0.f;
-          plane[c_loc * Cfg::TTP + ta] = make_float2(v, ZOH ? xv : v * xv);
-          const float g = p.has_z ? silu_f(to_f32(zs[ta * DT + ch])) : 1.f;
-          g1[j] = g;
-          g2[j] = dsk * xv * g;
-        }
-      }
-      __syncwarp();
-
-      // -- the scan over TT tokens of this lane's channel --
-      OutT *yrow = ybase + ((size_t)b * p.L + t0) * p.D + d;
-      const float2 *prow = plane + c_loc * Cfg::TTP;
-      float4 dpair;  // (Delta, Delta*x) of an even token and the next, one 16-byte load
+          float2 xv;
+          if constexpr (CONV) {
+            float2 u = make_float2(cb[0], cb[1]);
 #pragma unroll
-      for (int tt = 0; tt < TT; tt += LPC) {
-        float yp[LPC];
-#pragma unroll
-        for (int j = 0; j < LPC; ++j) {
-          const int t = tt + j;
-          if ((t & 1) == 0) dpair = *reinterpret_cast<const float4 *>(prow + t);
-          const float2 dd = (t & 1) ? make_float2(dpair.z, dpair.w) : make_float2(dpair.x, dpair.y);
-          float bv[NPL], cv[NPL];
-          load_bc<NPL>(Bs + (tt + j) * NS + q * NPL, bv);
-          load_bc<NPL>(Cs + (tt + j) * NS + q * NPL, cv);
-          if constexpr (NPL % 2 == 0) {
-            const float2 dA = make_float2(dd.x, dd.x), dX = make_float2(dd.y, dd.y);
-            float2 acc = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int i = 0; i < NPL; i += 2) {
-              const float2 arg = fmul2(dA, make_float2(A2[i], A2[i + 1]));
-              const float2 a = make_float2(ex2_approx(arg.x), ex2_approx(arg.y));
-              float2 bx = fmul2(dX, make_float2(bv[i], bv[i + 1]));
-              if constexpr (ZOH)  // dX holds x: Bbar x = ((e^u - 1) / A) * (B x)
-                bx = fmul2(zoh_coef2(fmul2(arg, make_float2(kLn2, kLn2)), a, dA,
-                                     make_float2(invA[i], invA[i + 1])),
-                           bx);
-              const float2 hn = ffma2(a, make_float2(h[i], h[i + 1]), bx);
-              h[i] = hn.x;
-              h[i + 1] = hn.y;
-              acc = ffma2(make_float2(cv[i], cv[i + 1]), hn, acc);
-            }
-            yp[j] = acc.x + acc.y;
+            for (int k = 0; k < kConvWidth; ++k)
+              u = ffma2(make_float2(cw[0][k], cw[1][k]), load_pair(xs + (ta + 1 + k) * DT + ch0),
+                        u);
+            xv = silu_f2(u);
+            if (xcrow && valid_ch && !CARRY && ta < nvalid)
+              store_pair(xcrow + (size_t)ta * p.D, xv);
           } else {
-            const float arg = dd.x * A2[0];
-            const float a = ex2_approx(arg);
-            float bx = dd.y * bv[0];
-            if constexpr (ZOH) bx *= zoh_coef(arg * kLn2, a, dd.x, invA[0]);
-            h[0] = fmaf(a, h[0], bx);
-            yp[j] = cv[0] * h[0];
+            xv = load_pair(xs + ta * DT + ch0);
+          }
+          float2 v = fadd2(load_pair(ds + ta * DT + ch0), make_float2(bias[0], bias[1]));
+          if (p.softplus) v = softplus_f2(v);
+          if (ta >= nvalid) v = make_float2(0.f, 0.f);  // past the end: identity update
+          const float2 dx = ZOH ? xv : fmul2(v, xv);
+          plane[g_loc * Cfg::TTP + ta] = make_float4(v.x, v.y, dx.x, dx.y);
+          if constexpr (!CARRY) {
+            const float2 g = p.has_z ? silu_f2(load_pair(zs + ta * DT + ch0))
+                                     : make_float2(1.f, 1.f);
+            g1[j] = g;
+            g2[j] = fmul2(fmul2(make_float2(dsk[0], dsk[1]), xv), g);
           }
         }
-        const float ys = reduce_scatter<LPC>(yp, q);
-        const int to = tt + q;  // this lane's own token of the group: prologue slot tt / LPC
-        if (to < nvalid && valid_ch)
-          yrow[(size_t)to * p.D] = from_f32<OutT>(fmaf(ys, g1[tt / LPC], g2[tt / LPC]));
+        __syncwarp();
+
+        const float4 *prow = plane + g_loc * Cfg::TTP;
+#pragma unroll
+        for (int tt = 0; tt < TT; tt += LPC) {
+          float2 yp[LPC];
+#pragma unroll
+          for (int j = 0; j < LPC; ++j) {
+            const int t = tt + j;
+            const float4 dd = prow[t];  // (Delta0, Delta1, X0, X1)
+            float bv[NPL], cv[NPL];
+            load_bc<NPL>(Bs + t * NS + q * NPL, bv);
+            if constexpr (!CARRY) load_bc<NPL>(Cs + t * NS + q * NPL, cv);
+            float ypc[2];
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              const float dl = c ? dd.y : dd.x, xx = c ? dd.w : dd.z;
+              if constexpr (CARRY) dsum[c] += dl;
+              const float2 dA = make_float2(dl, dl), dX = make_float2(xx, xx);
+              float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+              for (int i = 0; i < NPL; i += 2) {
+                const float2 arg = fmul2(dA, make_float2(A2[c][i], A2[c][i + 1]));
+                const float2 a = make_float2(ex2_approx(arg.x), ex2_approx(arg.y));
+                float2 bx = fmul2(dX, make_float2(bv[i], bv[i + 1]));
+                if constexpr (ZOH)
+                  bx = fmul2(zoh_coef2(fmul2(arg, make_float2(kLn2, kLn2)), a, dA,
+                                       make_float2(invA[c][i], invA[c][i + 1])),
+                             bx);
+                const float2 hn = ffma2(a, make_float2(h[c][i], h[c][i + 1]), bx);
+                h[c][i] = hn.x;
+                h[c][i + 1] = hn.y;
+                if constexpr (!CARRY) acc = ffma2(make_float2(cv[i], cv[i + 1]), hn, acc);
+              }
+              ypc[c] = acc.x + acc.y;
+            }
+            yp[j] = make_float2(ypc[0], ypc[1]);
+          }
+          if constexpr (!CARRY) {
+            const float2 ys = reduce_scatter2<LPC>(yp, q);
+            const int to = tt + q;
+            if (to < nvalid && valid_ch)
+              store_pair(yrow + (size_t)to * p.D, ffma2(ys, g1[tt / LPC], g2[tt / LPC]));
+          }
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&rempty[r]);  // this warp is done with slot r
 
-      const bool run_end = st + 1 == cur.st_end;
-      if (run_end) {
-        if (st == S - 1) {
-          if (p.want_hlast && valid_ch) {
-            float *dst = p.h_last + ((size_t)b * p.D + d) * NS + q * NPL;
+      if (st + 1 == cur.st_end) {  // end of this item's stages
+        if constexpr (CARRY) {
+          // the sub-chunk's map: (sum of Delta, state reached from 0)
+          if (valid_ch) {
+            const size_t base = ((size_t)b * p.nsub_row + cur.part) * p.D + d;
 #pragma unroll
-            for (int i = 0; i < NPL; ++i) dst[i] = h[i];
+            for (int c = 0; c < KC; ++c) {
+              float *dst = p.agg_h + (base + c) * NS + q * NPL;
+#pragma unroll
+              for (int i = 0; i < NPL; ++i) __stcg(dst + i, h[c][i]);
+              if (q == 0) __stcg(p.agg_s + base + c, dsum[c]);
+            }
           }
-        } else if ((long long)row * S + st != p.drop_unit) {  // hand the state on
-          float *dst = p.ws_state + ((size_t)row * DT + ch) * NS + q * NPL;
+        } else if (st + 1 == cur.seg_end) {
+          if (st == S - 1 && p.want_hlast && valid_ch) {  // the last segment's end
 #pragma unroll
-          for (int i = 0; i < NPL; ++i) __stcg(dst + i, h[i]);
+            for (int c = 0; c < KC; ++c) {
+              float *dst = p.h_last + ((size_t)b * p.D + d + c) * NS + q * NPL;
+#pragma unroll
+              for (int i = 0; i < NPL; ++i) dst[i] = h[c][i];
+            }
+          }
+        } else if ((long long)cur.row * S + st != p.drop_unit) {  // hand the state on
+#pragma unroll
+          for (int c = 0; c < KC; ++c) {
+            float *dst = p.ws_state + ((size_t)cur.vrow * DT + ch0 + c) * NS + q * NPL;
+#pragma unroll
+            for (int i = 0; i < NPL; ++i) __stcg(dst + i, h[c][i]);
+          }
           __threadfence();
           __syncwarp();
           if (lane == 0)
-            st_release_u64(p.ws_flags + (size_t)row * WARPS + warp,
+            st_release_u64(p.ws_flags + (size_t)cur.vrow * WARPS + warp,
                            ((unsigned long long)epoch << 32) | (unsigned)(st + 1));
         }
       }
@@ -425,15 +673,16 @@ __global__ void __launch_bounds__((WARPS + 1) * 32)
 }
 
 // ---------------------------------------------------------------------------
-// host-side variant table (one translation unit per dtype pair)
+// host side: one compiled variant
 // ---------------------------------------------------------------------------
 
-template <typename InT, typename OutT, int NS, int LPC, int WARPS, int TT, bool ZOH>
+template <typename InT, typename OutT, int NS, int LPC, int KC, int WARPS, int TT, bool ZOH,
+          bool CARRY, bool CONV>
 static cudaError_t run_variant(const LaunchShape *ls, const TmaMaps *maps, const FwdParams *p,
                                cudaStream_t stream, VariantInfo *vi) {
-  using Cfg = FwdCfg<InT, OutT, NS, LPC, WARPS, TT>;
-  auto kern = fwd_kernel<InT, OutT, NS, LPC, WARPS, TT, ZOH>;
-  if (Cfg::SMEM > 227 * 1024) return cudaErrorInvalidValue;
+  using Cfg = FwdCfg<InT, OutT, NS, LPC, KC, WARPS, TT, CONV>;
+  auto kern = fwd_kernel<InT, OutT, NS, LPC, KC, WARPS, TT, ZOH, CARRY, CONV>;
+  if (Cfg::SMEM + 8 * Cfg::RAW > 227 * 1024) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
   if (e != cudaSuccess) {
     cudaGetLastError();
@@ -450,80 +699,11 @@ static cudaError_t run_variant(const LaunchShape *ls, const TmaMaps *maps, const
   return cudaGetLastError();
 }
 
-template <typename InT, typename OutT, int NS, int LPC, int WARPS, bool ZOH>
-static cudaError_t by_tt(const LaunchShape *ls, const TmaMaps *maps, const FwdParams *p,
-                         cudaStream_t st, VariantInfo *vi) {
-  // a row tile's x / delta / z rows must be whole 16-byte TMA units
-  if constexpr ((WARPS * (32 / LPC) * (int)sizeof(InT)) % 16 != 0) {
-    return cudaErrorInvalidValue;
-  } else {
-    switch (ls->tt) {
-      case 16:
-        if constexpr (!ZOH) return run_variant<InT, OutT, NS, LPC, WARPS, 16, ZOH>(ls, maps, p, st, vi);
-        return cudaErrorInvalidValue;
-      case 32: return run_variant<InT, OutT, NS, LPC, WARPS, 32, ZOH>(ls, maps, p, st, vi);
-      case 64: return run_variant<InT, OutT, NS, LPC, WARPS, 64, ZOH>(ls, maps, p, st, vi);
-      default: return cudaErrorInvalidValue;
-    }
-  }
+// Does a launch shape ask for this compiled variant?
+inline bool shape_is(const LaunchShape *ls, int ns, int lpc, int kc, int warps, int tt, bool zoh,
+                     bool carry, bool conv) {
+  return ls->ns == ns && ls->lpc == lpc && ls->kc == kc && ls->warps == warps && ls->tt == tt &&
+         ls->zoh == zoh && ls->carry == carry && ls->conv == conv;
 }
-
-template <typename InT, typename OutT, int NS, int LPC, bool ZOH>
-static cudaError_t by_warps(const LaunchShape *ls, const TmaMaps *maps, const FwdParams *p,
-                            cudaStream_t st, VariantInfo *vi) {
-  switch (ls->warps) {
-    case 2: return by_tt<InT, OutT, NS, LPC, 2, ZOH>(ls, maps, p, st, vi);
-    case 4: return by_tt<InT, OutT, NS, LPC, 4, ZOH>(ls, maps, p, st, vi);
-    case 8: return by_tt<InT, OutT, NS, LPC, 8, ZOH>(ls, maps, p, st, vi);
-    default: return cudaErrorInvalidValue;
-  }
-}
-
-template <typename InT, typename OutT, int NS, bool ZOH>
-static cudaError_t by_lpc(const LaunchShape *ls, const TmaMaps *maps, const FwdParams *p,
-                          cudaStream_t st, VariantInfo *vi) {
-  switch (ls->lpc) {
-    case 1: return by_warps<InT, OutT, NS, 1, ZOH>(ls, maps, p, st, vi);
-    case 2: return by_warps<InT, OutT, NS, 2, ZOH>(ls, maps, p, st, vi);
-    case 4: return by_warps<InT, OutT, NS, 4, ZOH>(ls, maps, p, st, vi);
-    case 8:
-      if constexpr (NS >= 8) return by_warps<InT, OutT, NS, 8, ZOH>(ls, maps, p, st, vi);
-      return cudaErrorInvalidValue;
-    case 16:
-      if constexpr (NS >= 16) return by_warps<InT, OutT, NS, 16, ZOH>(ls, maps, p, st, vi);
-      return cudaErrorInvalidValue;
-    default: return cudaErrorInvalidValue;
-  }
-}
-
-template <typename InT, typename OutT, bool ZOH>
-static cudaError_t by_ns_zoh(const LaunchShape *ls, const TmaMaps *maps, const FwdParams *p,
-                             cudaStream_t st, VariantInfo *vi) {
-  switch (ls->ns) {
-    case 4:
-      if constexpr (sizeof(InT) == 4) return by_lpc<InT, OutT, 4, ZOH>(ls, maps, p, st, vi);
-      return cudaErrorInvalidValue;
-    case 8: return by_lpc<InT, OutT, 8, ZOH>(ls, maps, p, st, vi);
-    case 16: return by_lpc<InT, OutT, 16, ZOH>(ls, maps, p, st, vi);
-    default: return cudaErrorInvalidValue;
-  }
-}
-
-template <typename InT, typename OutT>
-static cudaError_t by_ns(const LaunchShape *ls, const TmaMaps *maps, const FwdParams *p,
-                         cudaStream_t st, VariantInfo *vi) {
-  if (ls->stages != kStages) return cudaErrorInvalidValue;
-  if (p && p->zoh != ls->zoh) return cudaErrorInvalidValue;
-  return ls->zoh ? by_ns_zoh<InT, OutT, true>(ls, maps, p, st, vi)
-                 : by_ns_zoh<InT, OutT, false>(ls, maps, p, st, vi);
-}
-
-// per-dtype entry points (defined in scan_fwd_<dtypes>.cu)
-cudaError_t fwd_dispatch_f32(const LaunchShape *, const TmaMaps *, const FwdParams *, cudaStream_t,
-                             VariantInfo *);
-cudaError_t fwd_dispatch_bf16(const LaunchShape *, const TmaMaps *, const FwdParams *,
-                              cudaStream_t, VariantInfo *);
-cudaError_t fwd_dispatch_bf16_f32(const LaunchShape *, const TmaMaps *, const FwdParams *,
-                                  cudaStream_t, VariantInfo *);
 
 }  // namespace ssm

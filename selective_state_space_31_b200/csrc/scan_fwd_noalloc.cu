@@ -113,8 +113,10 @@ bool cached_shape(const ShapeKey &key, int num_sms, ssm::FwdShape *out) {
       }
   }
   ssm::FwdShape fs;
+  ssm::FwdOverrides o{0, 0, 0, 0};
+  o.segments = 1;  // no carry pass: its maps would need more scratch
   if (ssm::choose_fwd_shape(key.in_dtype, key.out_dtype, key.batch, key.seqlen, key.dim, key.ns,
-                            key.zoh, num_sms, ssm::FwdOverrides{0, 0, 0, 0}, &fs) != cudaSuccess) {
+                            key.zoh, false, num_sms, o, &fs) != cudaSuccess) {
     cudaGetLastError();
     return false;
   }
@@ -228,6 +230,9 @@ extern "C" SSM_API ssm_status ssm_scan_fwd_noalloc(
   ssm::FwdParams p{};
   p.Bsz = (int)d.batch; p.L = (int)d.seqlen; p.D = (int)d.dim; p.N = ns;
   p.DT = DT; p.nDT = nDT; p.rows = (int)rows; p.S = fs.S;
+  p.M = 1; p.SPS = fs.S; p.nq = 0; p.nsub_row = 0;
+  p.agg_h = nullptr; p.agg_s = nullptr;
+  p.conv_w = nullptr; p.conv_b = nullptr; p.xconv = nullptr;
   p.PL = fs.PL; p.items = (int)(rows * fs.parts);
   p.softplus = (f & SSM_DELTA_SOFTPLUS) != 0;
   p.has_z = (f & SSM_HAS_Z) != 0;

@@ -38,10 +38,26 @@ __global__ void __launch_bounds__(128) fwd_general_kernel(const GenericParams p)
   }
   const float Dd = p.has_D ? p.Dv[d] : 0.f;
   const float bias = p.has_bias ? p.bias[d] : 0.f;
+  // conv front-end: x_t = silu(cb + sum_k w_k x_in[t - 3 + k]), the last
+  // three inputs kept in registers (zero before the sequence)
+  float w[kConvWidth] = {0.f, 0.f, 0.f, 0.f}, cb = 0.f, xh[kConvWidth - 1] = {0.f, 0.f, 0.f};
+  if (p.conv_w) {
+#pragma unroll
+    for (int k = 0; k < kConvWidth; ++k) w[k] = p.conv_w[(size_t)d * kConvWidth + k];
+    cb = p.conv_b ? p.conv_b[d] : 0.f;
+  }
   for (int t = 0; t < p.L; ++t) {
     const size_t i = ((size_t)b * p.L + t) * p.D + d;
     const size_t j = ((size_t)b * p.L + t) * N;
-    const float xv = ldf<InT>(p.x, i);
+    float xv = ldf<InT>(p.x, i);
+    if (p.conv_w) {
+      const float u = fmaf(w[3], xv, fmaf(w[2], xh[2], fmaf(w[1], xh[1], fmaf(w[0], xh[0], cb))));
+      xh[0] = xh[1];
+      xh[1] = xh[2];
+      xh[2] = xv;
+      xv = silu_f(u);
+      if (p.xconv) reinterpret_cast<OutT *>(p.xconv)[i] = from_f32<OutT>(xv);
+    }
     const float v = ldf<InT>(p.dt, i) + bias;
     const float dlt = p.softplus ? softplus_f(v) : v;
     const float dtx = dlt * xv;

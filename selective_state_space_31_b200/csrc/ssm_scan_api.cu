@@ -19,7 +19,8 @@
 namespace {
 
 constexpr uint32_t kKnownFlags = SSM_HAS_Z | SSM_HAS_D | SSM_DELTA_SOFTPLUS | SSM_HAS_DELTA_BIAS |
-                                 SSM_HAS_H0 | SSM_WANT_HLAST | SSM_A_DIRECT | SSM_ZOH;
+                                 SSM_HAS_H0 | SSM_WANT_HLAST | SSM_A_DIRECT | SSM_ZOH |
+                                 SSM_CONV_X;
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
 constexpr int kMaxDstate = 64;
 
@@ -80,9 +81,14 @@ struct ssm_scan_plan {
   int device = 0;
   int num_sms = 0;
   int path = PATH_GENERAL;
+  ssm::FwdShape fs{};  // launch shape of the fused kernel (and of its carry pass)
   ssm::LaunchShape ls{};
   int DT = 0, nDT = 0, S = 0, PL = 0, parts = 0;
   int64_t rows = 0, units = 0;
+  float *ws_agg = nullptr;  // carry-pass maps: (B, nsub, D, N) states then (B, nsub, D) sums
+  size_t ws_agg_bytes = 0;
+  float *ws_map = nullptr;  // sub-chunk maps of ssm_scan_seq_map (allocated by its first call)
+  size_t ws_map_bytes = 0;
   ssm_scan_config cfg{};  // user overrides
   ssm::Control *ctl = nullptr;
   int ring = 0;  // stage slots of the fused kernel's TMA ring
@@ -107,9 +113,11 @@ ssm_status validate_desc(const ssm_scan_desc *d) {
   if (d->flags & ~kKnownFlags) return SSM_ERR_INVALID_ARG;
   if (d->flags & SSM_A_DIRECT) {
     if (d->dstate != 1) return SSM_ERR_INVALID_ARG;
-    if (d->flags & (SSM_HAS_Z | SSM_HAS_D | SSM_DELTA_SOFTPLUS | SSM_HAS_DELTA_BIAS | SSM_ZOH))
+    if (d->flags & (SSM_HAS_Z | SSM_HAS_D | SSM_DELTA_SOFTPLUS | SSM_HAS_DELTA_BIAS | SSM_ZOH |
+                    SSM_CONV_X))
       return SSM_ERR_INVALID_ARG;
   }
+  if ((d->flags & SSM_CONV_X) && (d->flags & SSM_ZOH)) return SSM_ERR_UNSUPPORTED;
   if (d->dstate > kMaxDstate) return SSM_ERR_UNSUPPORTED;
   return SSM_OK;
 }
@@ -133,17 +141,36 @@ ssm_status plan_tma(ssm_scan_plan *pl) {
   const int ns = (int)d.dstate;
   if (pl->cfg.tile_t && pl->cfg.tile_t != 16 && pl->cfg.tile_t != 32 && pl->cfg.tile_t != 64)
     return SSM_ERR_INVALID_ARG;
-  const ssm::FwdOverrides o{pl->cfg.lanes_per_chan, pl->cfg.warps_per_cta, pl->cfg.tile_t,
-                            pl->cfg.grid};
+  if (pl->cfg.chans_per_lane && pl->cfg.chans_per_lane != 1 && pl->cfg.chans_per_lane != 2)
+    return SSM_ERR_INVALID_ARG;
+  if (pl->cfg.segments && pl->cfg.segments != 1 && pl->cfg.segments != 2 &&
+      pl->cfg.segments != 4 && pl->cfg.segments != 8)
+    return SSM_ERR_INVALID_ARG;
+  ssm::FwdOverrides o{pl->cfg.lanes_per_chan, pl->cfg.warps_per_cta, pl->cfg.tile_t,
+                      pl->cfg.grid};
+  o.kc = pl->cfg.chans_per_lane;
+  o.segments = pl->cfg.segments;
   ssm::FwdShape fs;
   if (ssm::choose_fwd_shape((int)d.in_dtype, (int)d.out_dtype, d.batch, d.seqlen, d.dim, ns,
-                            (d.flags & SSM_ZOH) != 0, pl->num_sms, o, &fs) != cudaSuccess) {
+                            (d.flags & SSM_ZOH) != 0, (d.flags & SSM_CONV_X) != 0, pl->num_sms, o,
+                            &fs) != cudaSuccess) {
     cudaGetLastError();
     return SSM_ERR_UNSUPPORTED;  // no variant fits (or bad override)
   }
-  // workspace: carried state per (row, channel, n) and a flag per (row, warp)
-  const size_t st_bytes = (size_t)fs.rows * fs.DT * ns * sizeof(float);
-  const size_t fl_bytes = (size_t)fs.rows * fs.ls.warps * sizeof(unsigned long long);
+  // workspace: carried state per (row, segment, channel, n), a flag per
+  // (row, segment, warp), and the carry pass's maps per (batch, sub-chunk, channel)
+  const int64_t vrows = fs.rows * fs.M;
+  const size_t st_bytes = (size_t)vrows * fs.DT * ns * sizeof(float);
+  const size_t fl_bytes = (size_t)vrows * fs.ls.warps * sizeof(unsigned long long);
+  const int64_t nsub = fs.M > 1 ? (int64_t)(fs.M - 1) * fs.nq : 0;
+  const size_t agg_bytes = (size_t)(d.batch * nsub * d.dim * (ns + 1)) * sizeof(float);
+  if (agg_bytes > pl->ws_agg_bytes) {
+    if (pl->ws_agg) cudaFree(pl->ws_agg);
+    pl->ws_agg = nullptr;
+    pl->ws_agg_bytes = 0;
+    if (cudaMalloc(&pl->ws_agg, agg_bytes) != cudaSuccess) return SSM_ERR_OOM;
+    pl->ws_agg_bytes = agg_bytes;
+  }
   if (st_bytes > pl->ws_state_bytes) {
     if (pl->ws_state) cudaFree(pl->ws_state);
     pl->ws_state = nullptr;
@@ -160,6 +187,7 @@ ssm_status plan_tma(ssm_scan_plan *pl) {
   }
   // flags start below every epoch tag (epochs start at 1)
   if (cudaMemset(pl->ws_flags, 0, pl->ws_flag_bytes) != cudaSuccess) return SSM_ERR_CUDA;
+  pl->fs = fs;
   pl->ls = fs.ls;
   pl->DT = fs.DT;
   pl->nDT = (int)((d.dim + fs.DT - 1) / fs.DT);
@@ -204,7 +232,19 @@ const char *ssm_status_string(ssm_status s) {
   }
 }
 
-int ssm_scan_version(void) { return 100; }
+int ssm_scan_version(void) { return 200; }
+
+int ssm_scan_list_variants(ssm_dtype in_dtype, ssm_dtype out_dtype, ssm_scan_variant *out,
+                           int max) {
+  constexpr int kMax = 512;
+  ssm::VariantDesc v[kMax];
+  const int n = std::min(kMax, ssm::fwd_variants((int)in_dtype, (int)out_dtype, v, kMax));
+  if (out)
+    for (int i = 0; i < n && i < max; ++i)
+      out[i] = ssm_scan_variant{v[i].ns, v[i].lpc, v[i].kc, v[i].warps, v[i].tt,
+                                v[i].zoh ? 1 : 0, v[i].carry ? 1 : 0, v[i].conv ? 1 : 0};
+  return n;
+}
 
 ssm_status ssm_scan_create(ssm_scan_plan **plan, const ssm_scan_desc *desc, int device) {
   if (!plan) return SSM_ERR_INVALID_ARG;
@@ -255,6 +295,8 @@ ssm_status ssm_scan_destroy(ssm_scan_plan *pl) {
     if (pl->ws_ck) cudaFree(pl->ws_ck);
     if (pl->ws_state) cudaFree(pl->ws_state);
     if (pl->ws_flags) cudaFree(pl->ws_flags);
+    if (pl->ws_agg) cudaFree(pl->ws_agg);
+    if (pl->ws_map) cudaFree(pl->ws_map);
   }
   delete pl;
   return SSM_OK;
@@ -277,14 +319,21 @@ ssm_status ssm_scan_get_info(const ssm_scan_plan *pl, ssm_scan_info *info) {
     info->parts_per_row = pl->parts;
     info->stages_per_part = pl->PL;
     info->smem_bytes = pl->ls.smem;
+    info->chans_per_lane = pl->ls.kc;
+    info->segments = pl->fs.M;
+    info->stages_per_segment = pl->fs.SPS;
+    info->carry_grid = pl->fs.M > 1 ? pl->fs.cls.grid : 0;
   }
-  info->workspace_bytes = pl->ws_state_bytes + pl->ws_flag_bytes + sizeof(ssm::Control);
+  info->launches_per_call = pl->path == PATH_TMA && pl->fs.M > 1 ? 2 : 1;
+  info->workspace_bytes =
+      pl->ws_state_bytes + pl->ws_flag_bytes + pl->ws_agg_bytes + sizeof(ssm::Control);
   return SSM_OK;
 }
 
 ssm_status ssm_scan_set_config(ssm_scan_plan *pl, const ssm_scan_config *cfg) {
   if (!pl || !cfg) return SSM_ERR_INVALID_ARG;
-  if (cfg->lanes_per_chan < 0 || cfg->warps_per_cta < 0 || cfg->grid < 0 || cfg->tile_t < 0)
+  if (cfg->lanes_per_chan < 0 || cfg->warps_per_cta < 0 || cfg->grid < 0 || cfg->tile_t < 0 ||
+      cfg->chans_per_lane < 0 || cfg->segments < 0)
     return SSM_ERR_INVALID_ARG;
   DeviceGuard guard(pl->device);
   if (!guard.ok) return SSM_ERR_CUDA;
@@ -321,12 +370,18 @@ ssm_status ssm_scan_get_status(ssm_scan_plan *pl) {
   return (ssm_status)st;
 }
 
-ssm_status ssm_scan_fwd(ssm_scan_plan *pl, const void *x, const void *delta,
-                        const float *delta_bias, const void *A, const void *B, const void *C,
-                        const float *D, const void *z, const float *h0, void *y, float *h_last,
-                        ssm_stream_t stream_) {
-  if (!pl) return SSM_ERR_INVALID_ARG;
+}  // extern "C"
+
+namespace {
+
+// Both forward entry points: conv_w non-null selects the conv front-end (x
+// then holds the raw x branch).
+ssm_status fwd_impl(ssm_scan_plan *pl, const void *x, const float *conv_w, const float *conv_b,
+                    void *xconv, const void *delta, const float *delta_bias, const void *A,
+                    const void *B, const void *C, const float *D, const void *z, const float *h0,
+                    void *y, float *h_last, ssm_stream_t stream_) {
   const ssm_scan_desc &d = pl->desc;
+  const bool conv = conv_w != nullptr;
   const uint32_t f = d.flags;
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   // Pointer checks apply to tensors that have elements: a zero-size tensor
@@ -363,12 +418,15 @@ ssm_status ssm_scan_fwd(ssm_scan_plan *pl, const void *x, const void *delta,
   }
 
   const bool aligned = aligned16(x) && aligned16(delta) && aligned16(z) && aligned16(B) &&
-                       aligned16(C) && aligned16(y);
+                       aligned16(C) && aligned16(y) && aligned16(xconv);
   if (pl->path == PATH_TMA && aligned) {
+    const ssm::FwdShape &fs = pl->fs;
     ssm::TmaMaps maps;
     const uint64_t Bn = d.batch, L = d.seqlen, Dm = d.dim, N = d.dstate;
     const uint32_t DT = (uint32_t)pl->DT, TT = (uint32_t)pl->ls.tt;
-    if (!encode3d(&maps.x, d.in_dtype, x, Dm, L, Bn, DT, TT) ||
+    // the conv front-end's x tiles carry kConvWidth earlier tokens
+    const uint32_t XT = TT + (conv ? (uint32_t)ssm::kConvWidth : 0u);
+    if (!encode3d(&maps.x, d.in_dtype, x, Dm, L, Bn, DT, XT) ||
         !encode3d(&maps.dt, d.in_dtype, delta, Dm, L, Bn, DT, TT) ||
         !encode3d(&maps.z, d.in_dtype, z ? z : x, Dm, L, Bn, DT, TT) ||
         !encode3d(&maps.B, d.in_dtype, B, N, L, Bn, (uint32_t)N, TT) ||
@@ -377,7 +435,12 @@ ssm_status ssm_scan_fwd(ssm_scan_plan *pl, const void *x, const void *delta,
     ssm::FwdParams p{};
     p.Bsz = (int)d.batch; p.L = (int)d.seqlen; p.D = (int)d.dim; p.N = (int)d.dstate;
     p.DT = pl->DT; p.nDT = pl->nDT; p.rows = (int)pl->rows; p.S = pl->S;
-    p.PL = pl->PL; p.items = (int)(pl->rows * pl->parts);
+    p.M = fs.M; p.SPS = fs.SPS;
+    p.PL = pl->PL; p.items = (int)(pl->rows * fs.M * pl->parts);
+    p.nq = fs.nq; p.nsub_row = fs.M > 1 ? (fs.M - 1) * fs.nq : 0;
+    const size_t nagg = (size_t)d.batch * p.nsub_row * d.dim;
+    p.agg_h = pl->ws_agg;
+    p.agg_s = pl->ws_agg ? pl->ws_agg + nagg * d.dstate : nullptr;
     p.softplus = (f & SSM_DELTA_SOFTPLUS) != 0;
     p.has_z = (f & SSM_HAS_Z) != 0;
     p.has_D = (f & SSM_HAS_D) != 0;
@@ -387,9 +450,31 @@ ssm_status ssm_scan_fwd(ssm_scan_plan *pl, const void *x, const void *delta,
     p.zoh = (f & SSM_ZOH) != 0;
     p.A = static_cast<const float *>(A);
     p.Dv = D; p.bias = delta_bias; p.h0 = h0; p.h_last = h_last; p.y = y;
+    p.conv_w = conv_w; p.conv_b = conv_b; p.xconv = xconv;
     p.ws_state = pl->ws_state; p.ws_flags = pl->ws_flags; p.ctl = pl->ctl;
     p.timeout_ns = pl->timeout_ns;
     p.drop_unit = pl->drop_unit;
+    if (fs.M > 1) {
+      // carry pass: the map of every sub-chunk of segments 0 .. M-2, from 0
+      ssm::TmaMaps cmaps = maps;
+      const uint32_t cDT = (uint32_t)fs.cDT;
+      if (cDT != DT && (!encode3d(&cmaps.x, d.in_dtype, x, Dm, L, Bn, cDT, XT) ||
+                        !encode3d(&cmaps.dt, d.in_dtype, delta, Dm, L, Bn, cDT, TT)))
+        return SSM_ERR_CUDA;
+      ssm::FwdParams c = p;
+      c.DT = fs.cDT;
+      c.nDT = (int)((d.dim + fs.cDT - 1) / fs.cDT);
+      c.rows = (int)fs.crows;
+      c.M = 1;
+      c.SPS = pl->S;
+      c.PL = fs.Q;
+      c.items = (int)(fs.crows * p.nsub_row);
+      c.drop_unit = -1;
+      c.xconv = nullptr;
+      const cudaError_t e =
+          ssm::launch_fwd_tma((int)d.in_dtype, (int)d.out_dtype, fs.cls, cmaps, c, stream);
+      if (e != cudaSuccess) return SSM_ERR_CUDA;
+    }
     return map_cuda(ssm::launch_fwd_tma((int)d.in_dtype, (int)d.out_dtype, pl->ls, maps, p, stream));
   }
 
@@ -407,7 +492,131 @@ ssm_status ssm_scan_fwd(ssm_scan_plan *pl, const void *x, const void *delta,
   p.x = x; p.dt = delta; p.z = z; p.B = B; p.C = C;
   p.A = static_cast<const float *>(A);
   p.Dv = D; p.bias = delta_bias; p.h0 = h0; p.y = y; p.h_last = h_last;
+  p.conv_w = conv_w; p.conv_b = conv_b; p.xconv = xconv;
   return map_cuda(ssm::launch_fwd_general(p, stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+ssm_status ssm_scan_fwd(ssm_scan_plan *pl, const void *x, const void *delta,
+                        const float *delta_bias, const void *A, const void *B, const void *C,
+                        const float *D, const void *z, const float *h0, void *y, float *h_last,
+                        ssm_stream_t stream) {
+  if (!pl) return SSM_ERR_INVALID_ARG;
+  if (pl->desc.flags & SSM_CONV_X) return SSM_ERR_INVALID_ARG;  // needs ssm_scan_fwd_conv
+  return fwd_impl(pl, x, nullptr, nullptr, nullptr, delta, delta_bias, A, B, C, D, z, h0, y,
+                  h_last, stream);
+}
+
+ssm_status ssm_scan_seq_map(ssm_scan_plan *pl, const void *x, const void *delta,
+                            const float *delta_bias, const float *A, const void *B, float *map_h,
+                            float *map_s, ssm_stream_t stream_) {
+  if (!pl) return SSM_ERR_INVALID_ARG;
+  const ssm_scan_desc &d = pl->desc;
+  const uint32_t f = d.flags;
+  if (f & (SSM_A_DIRECT | SSM_CONV_X)) return SSM_ERR_UNSUPPORTED;
+  const bool has_chans = d.batch * d.dim != 0;
+  if (has_chans && (!A || !map_h || !map_s)) return SSM_ERR_INVALID_ARG;
+  if (d.batch * d.seqlen * d.dim != 0 && (!x || !delta || !B)) return SSM_ERR_INVALID_ARG;
+  if (has_chans && ((f & SSM_HAS_DELTA_BIAS) != 0) != (delta_bias != nullptr))
+    return SSM_ERR_INVALID_ARG;
+  if (!has_chans) return SSM_OK;
+  DeviceGuard guard(pl->device);
+  if (!guard.ok) return SSM_ERR_CUDA;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  const uint64_t Bn = d.batch, L = d.seqlen, Dm = d.dim, N = d.dstate;
+  const bool aligned = aligned16(x) && aligned16(delta) && aligned16(B);
+  ssm::MapShape ms{};
+  if (pl->path == PATH_TMA && aligned && d.seqlen > 0 &&
+      ssm::choose_map_shape((int)d.in_dtype, (int)d.out_dtype, d.batch, d.dim, pl->fs,
+                            pl->num_sms, &ms) == cudaSuccess) {
+    const size_t nagg = (size_t)d.batch * ms.nsub * d.dim;
+    const size_t need = nagg * (d.dstate + 1) * sizeof(float);
+    if (need > pl->ws_map_bytes) {
+      if (pl->ws_map) cudaFree(pl->ws_map);
+      pl->ws_map = nullptr;
+      pl->ws_map_bytes = 0;
+      if (cudaMalloc(&pl->ws_map, need) != cudaSuccess) {
+        cudaGetLastError();
+        return SSM_ERR_OOM;
+      }
+      pl->ws_map_bytes = need;
+    }
+    const uint32_t TT = (uint32_t)pl->fs.ls.tt, cDT = (uint32_t)ms.DT;
+    ssm::TmaMaps maps;
+    if (!encode3d(&maps.x, d.in_dtype, x, Dm, L, Bn, cDT, TT) ||
+        !encode3d(&maps.dt, d.in_dtype, delta, Dm, L, Bn, cDT, TT) ||
+        !encode3d(&maps.z, d.in_dtype, x, Dm, L, Bn, cDT, TT) ||
+        !encode3d(&maps.B, d.in_dtype, B, N, L, Bn, (uint32_t)N, TT) ||
+        !encode3d(&maps.C, d.in_dtype, B, N, L, Bn, (uint32_t)N, TT))
+      return SSM_ERR_CUDA;
+    ssm::FwdParams c{};
+    c.Bsz = (int)d.batch; c.L = (int)d.seqlen; c.D = (int)d.dim; c.N = (int)d.dstate;
+    c.DT = ms.DT; c.nDT = (int)((d.dim + ms.DT - 1) / ms.DT); c.rows = (int)ms.rows;
+    c.S = pl->fs.S; c.M = 1; c.SPS = pl->fs.S; c.PL = ms.Q;
+    c.items = (int)(ms.rows * ms.nsub);
+    c.nq = ms.nsub; c.nsub_row = ms.nsub;
+    c.agg_h = pl->ws_map;
+    c.agg_s = pl->ws_map + nagg * d.dstate;
+    c.softplus = (f & SSM_DELTA_SOFTPLUS) != 0;
+    c.has_bias = (f & SSM_HAS_DELTA_BIAS) != 0;
+    c.zoh = (f & SSM_ZOH) != 0;
+    c.A = A; c.bias = delta_bias;
+    c.ws_state = pl->ws_state; c.ws_flags = pl->ws_flags; c.ctl = pl->ctl;
+    c.timeout_ns = pl->timeout_ns;
+    c.drop_unit = -1;
+    if (ssm::launch_fwd_tma((int)d.in_dtype, (int)d.out_dtype, ms.ls, maps, c, stream) !=
+        cudaSuccess)
+      return SSM_ERR_CUDA;
+    ssm::FoldParams fp{};
+    fp.Bsz = (int)d.batch; fp.D = (int)d.dim; fp.N = (int)d.dstate; fp.count = ms.nsub;
+    fp.stride_b = (long long)ms.nsub * d.dim;
+    fp.stride_j = d.dim;
+    fp.A = A; fp.maps_h = c.agg_h; fp.maps_s = c.agg_s; fp.h0 = nullptr;
+    fp.h_out = map_h; fp.s_out = map_s;
+    return map_cuda(ssm::launch_fold_maps(fp, stream));
+  }
+  ssm::MapParams mp{};
+  mp.Bsz = (int)d.batch; mp.L = (int)d.seqlen; mp.D = (int)d.dim; mp.N = (int)d.dstate;
+  mp.softplus = (f & SSM_DELTA_SOFTPLUS) != 0;
+  mp.zoh = (f & SSM_ZOH) != 0;
+  mp.in_bf16 = d.in_dtype == SSM_BF16;
+  mp.x = x; mp.dt = delta; mp.B = B; mp.A = A; mp.bias = delta_bias;
+  mp.map_h = map_h; mp.map_s = map_s;
+  return map_cuda(ssm::launch_map_general(mp, stream));
+}
+
+ssm_status ssm_scan_fold_maps(ssm_scan_plan *pl, int count, const float *maps_h,
+                              const float *maps_s, const float *A, const float *h0, float *h_out,
+                              ssm_stream_t stream) {
+  if (!pl || count < 0) return SSM_ERR_INVALID_ARG;
+  const ssm_scan_desc &d = pl->desc;
+  if (d.flags & SSM_A_DIRECT) return SSM_ERR_UNSUPPORTED;
+  if (d.batch * d.dim == 0) return SSM_OK;
+  if (!A || !h_out || (count > 0 && (!maps_h || !maps_s))) return SSM_ERR_INVALID_ARG;
+  DeviceGuard guard(pl->device);
+  if (!guard.ok) return SSM_ERR_CUDA;
+  ssm::FoldParams fp{};
+  fp.Bsz = (int)d.batch; fp.D = (int)d.dim; fp.N = (int)d.dstate; fp.count = count;
+  fp.stride_b = d.dim;
+  fp.stride_j = d.batch * d.dim;
+  fp.A = A; fp.maps_h = maps_h; fp.maps_s = maps_s; fp.h0 = h0; fp.h_out = h_out;
+  fp.s_out = nullptr;
+  return map_cuda(ssm::launch_fold_maps(fp, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+ssm_status ssm_scan_fwd_conv(ssm_scan_plan *pl, const void *x_in, const float *conv_w,
+                             const float *conv_b, const void *delta, const float *delta_bias,
+                             const float *A, const void *B, const void *C, const float *D,
+                             const void *z, const float *h0, void *y, float *h_last,
+                             void *x_conv, ssm_stream_t stream) {
+  if (!pl) return SSM_ERR_INVALID_ARG;
+  if (!(pl->desc.flags & SSM_CONV_X)) return SSM_ERR_INVALID_ARG;
+  if (!conv_w && pl->desc.dim * pl->desc.batch * pl->desc.seqlen != 0) return SSM_ERR_INVALID_ARG;
+  return fwd_impl(pl, x_in, conv_w, conv_b, x_conv, delta, delta_bias, A, B, C, D, z, h0, y,
+                  h_last, stream);
 }
 
 ssm_status ssm_scan_bwd(ssm_scan_plan *pl, const void *x, const void *delta,
@@ -419,7 +628,7 @@ ssm_status ssm_scan_bwd(ssm_scan_plan *pl, const void *x, const void *delta,
   if (!pl) return SSM_ERR_INVALID_ARG;
   const ssm_scan_desc &d = pl->desc;
   const uint32_t f = d.flags;
-  if (f & (SSM_ZOH | SSM_A_DIRECT)) return SSM_ERR_UNSUPPORTED;
+  if (f & (SSM_ZOH | SSM_A_DIRECT | SSM_CONV_X)) return SSM_ERR_UNSUPPORTED;
   const bool has_tokens = d.batch * d.seqlen * d.dim != 0;
   const bool has_chans = d.batch * d.dim != 0;
   if (has_tokens && (!x || !delta || !B || !C || !dy || !dx || !ddelta || !dB || !dC))
@@ -473,6 +682,7 @@ ssm_status ssm_scan_step(ssm_scan_plan *pl, const void *x, const void *delta,
   const ssm_scan_desc &d = pl->desc;
   const uint32_t f = d.flags;
   if (f & SSM_A_DIRECT) return SSM_ERR_INVALID_ARG;
+  if (f & SSM_CONV_X) return SSM_ERR_UNSUPPORTED;  // the conv's token history is not kept
   const bool empty = d.batch * d.dim == 0;
   if (!empty && (!x || !delta || !A || !B || !C || !state || !y)) return SSM_ERR_INVALID_ARG;
   if (((f & SSM_HAS_Z) != 0) != (z != nullptr)) return SSM_ERR_INVALID_ARG;

@@ -33,7 +33,7 @@ from dataclasses import dataclass, field
 import numpy as np
 
 # field ids: one independent random stream per field
-_F_X, _F_DELTA, _F_Z, _F_B, _F_C, _F_BIAS, _F_D, _F_H0, _F_A = range(9)
+_F_X, _F_DELTA, _F_Z, _F_B, _F_C, _F_BIAS, _F_D, _F_H0, _F_A, _F_CONV_W, _F_CONV_B = range(11)
 
 
 def round_bf16(a: np.ndarray) -> np.ndarray:
@@ -123,22 +123,28 @@ def make_fwd(Bsz, L, D, N, *, in_dtype="bf16", out_dtype=None, seed=0, has_z=Tru
                       bias, h0, delta_softplus, True, zoh)
 
 
-def tiny_fp32(seed=0):
-    """B=1, L=512, D=64, N=16 fp32; delta_raw = N(0,1) - 1; no gate, no bias."""
-    return make_fwd(1, 512, 64, 16, in_dtype="f32", seed=seed, has_z=False, has_bias=False,
+def tiny_fp32(seed=0, shape=None):
+    """B=1, L=512, D=64, N=16 fp32; delta_raw = N(0,1) - 1; no gate, no bias.
+    ``shape`` = (B, L, D) resizes any workload with its distributions kept
+    (for profiling on smaller copies)."""
+    B, L, D = shape or (1, 512, 64)
+    return make_fwd(B, L, D, 16, in_dtype="f32", seed=seed, has_z=False, has_bias=False,
                     has_h0=False, delta_shift=-1.0, name="tiny_fp32")
 
 
-def mamba130m_layer(seed=1):
-    return make_fwd(8, 2048, 1536, 16, seed=seed, name="mamba130m_layer")
+def mamba130m_layer(seed=1, shape=None):
+    B, L, D = shape or (8, 2048, 1536)
+    return make_fwd(B, L, D, 16, seed=seed, name="mamba130m_layer")
 
 
-def mamba1p4b_layer(seed=2):
-    return make_fwd(4, 8192, 4096, 16, seed=seed, has_h0=True, name="mamba1p4b_layer")
+def mamba1p4b_layer(seed=2, shape=None):
+    B, L, D = shape or (4, 8192, 4096)
+    return make_fwd(B, L, D, 16, seed=seed, has_h0=True, name="mamba1p4b_layer")
 
 
-def long_seq(seed=3):
-    return make_fwd(1, 131072, 2560, 16, seed=seed, name="long_seq")
+def long_seq(seed=3, shape=None):
+    B, L, D = shape or (1, 131072, 2560)
+    return make_fwd(B, L, D, 16, seed=seed, name="long_seq")
 
 
 FWD_WORKLOADS = {
@@ -201,3 +207,13 @@ def make_direct(Bsz, L, D, *, seed=0, in_dtype="f32", has_h0=True, a_zero=False)
         A = round_bf16(A) if in_dtype == "bf16" else A
     h0 = _rng(seed, _F_H0).standard_normal((Bsz, D), dtype=np.float32) if has_h0 else None
     return {"x": x, "A": A, "B": Bm, "C": Cm, "h0": h0, "in_dtype": in_dtype}
+
+
+def make_conv(D: int, width: int = 4, seed: int = 0):
+    """Taps and bias of the causal conv front-end of the x branch, fp32:
+    w (D, width) and b (D,) ~ U(-1/sqrt(width), 1/sqrt(width)) (the uniform
+    fan-in initialisation of a depthwise convolution with `width` taps)."""
+    bound = 1.0 / np.sqrt(width)
+    w = _rng(seed, _F_CONV_W).uniform(-bound, bound, size=(D, width)).astype(np.float32)
+    b = _rng(seed, _F_CONV_B).uniform(-bound, bound, size=D).astype(np.float32)
+    return w, b

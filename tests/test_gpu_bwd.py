@@ -80,3 +80,41 @@ def test_bwd_refuses_zero_order_hold():
         plan.bwd(dev["x"], dev["delta"], dev["A"], dev["B"], dev["C"], dy, D=dev["D"],
                  z=dev["z"], delta_bias=dev["delta_bias"])
     assert e.value.status == bnd.ERR_UNSUPPORTED
+
+
+def test_bwd_channels_not_a_multiple_of_the_warp_group():
+    """dim % 8 != 0: a warp's channels span two batch elements, so dB and dC
+    take one atomic per lane instead of the warp's reduce-scatter."""
+    _check(synth.make_fwd(2, 70, 37, 16, in_dtype="f32", seed=56, has_h0=True), seed=5)
+
+
+def test_bwd_large_dstate():
+    """dstate 32: sixteen states per lane (no warp reduction of dB / dC)."""
+    _check(synth.make_fwd(1, 40, 16, 32, in_dtype="f32", seed=57, has_h0=True), seed=6)
+
+
+def test_bwd_130m_layer_sampled():
+    """The 130M-layer shape at full size in bf16: finite gradients, and the
+    per-channel ones (dA, dD, delta bias) and dh0 on sampled channels
+    against the oracle run over those channels only.  (dB / dC sum over
+    every channel, so they are checked on the small shapes above.)"""
+    inp = synth.make_fwd(8, 2048, 1536, 16, seed=58)
+    rng = np.random.default_rng(7)
+    dy = _round_bf16(rng.standard_normal((inp.Bsz, inp.L, inp.D)).astype(np.float32))
+    plan = gu.make_plan(inp)
+    dev = gu.upload(inp)
+    g = plan.bwd(dev["x"], dev["delta"], dev["A"], dev["B"], dev["C"],
+                 gu.dev_tensor(dy, "bf16"), D=dev["D"], z=dev["z"],
+                 delta_bias=dev["delta_bias"])
+    torch.cuda.synchronize()
+    for name, t in g.items():
+        assert bool(torch.isfinite(t).all()), name
+    chans = [0, 7, 8, 777, 1535]
+    sub = lambda a: np.ascontiguousarray(a[:, :, chans])
+    ref = oracle.get().bwd(sub(inp.x), sub(inp.delta), inp.A[chans], inp.B, inp.C, sub(dy),
+                           D=inp.Dskip[chans], z=sub(inp.z), delta_bias=inp.delta_bias[chans])
+    got_x = g["x"].cpu().numpy()[:, :, chans]
+    assert gu.normwise(got_x, ref["x"]) <= 2e-2
+    assert gu.normwise(g["delta"].cpu().numpy()[:, :, chans], ref["delta"]) <= 2e-2
+    assert gu.normwise(g["A"].cpu().numpy()[chans], ref["A"]) <= 2e-2
+    assert gu.normwise(g["D"].cpu().numpy()[chans], ref["D"]) <= 2e-2

@@ -31,47 +31,22 @@ def test_tiny_fp32_workload():
     _case(synth.tiny_fp32(), expect_path=0)
 
 
-@pytest.mark.parametrize("lpc", [1, 2, 4, 8, 16])
-@pytest.mark.parametrize("warps", [2, 4, 8])
-@pytest.mark.parametrize("tile_t", [16, 32, 64])
-@pytest.mark.parametrize("grid", [0, 2])
-def test_bf16_all_options_every_variant(lpc, warps, tile_t, grid):
-    """Every kernel variant (lanes per channel x scan warps x stage length)
-    with bf16 in/out, gate, skip, bias, h0 and a ragged L (not a multiple of
-    any stage length).  grid=2 makes each CTA run several parts of several
-    rows, handing carried states between CTAs.  The plan refuses variants
-    whose channel tile is not a whole 16-byte TMA row, and the one whose ring
-    of three stage slots (256 channels x 64 tokens) exceeds 227 KB of shared
-    memory."""
-    from selective_state_space_31_b200 import binding as bnd
-    inp = synth.make_fwd(3, 389, 64, 16, seed=21, has_h0=True)
-    cfg = dict(lanes_per_chan=lpc, warps_per_cta=warps, grid=grid, tile_t=tile_t)
-    if (warps * 32 // lpc) * 2 % 16 or (lpc, warps, tile_t) == (1, 8, 64):
-        plan = gu.make_plan(inp)
-        with pytest.raises(bnd.SsmError):
-            plan.set_config(**cfg)
-        return
-    plan = _case(inp, cfg, expect_path=0)
-    info = plan.info()
-    assert (info["lanes_per_chan"], info["warps_per_cta"], info["tile_t"]) == (lpc, warps, tile_t)
-
-
 @pytest.mark.parametrize("lpc,warps", [(4, 4), (8, 2), (16, 4)])
 @pytest.mark.parametrize("grid", [5, 40])
 def test_parts_chained_across_ctas(lpc, warps, grid):
     """grid=5 splits rows between CTAs; grid=40 gives CTAs less than a row
     each, so a row passes through a chain of CTAs."""
     inp = synth.make_fwd(3, 389, 64, 16, seed=21, has_h0=True)
-    _case(inp, dict(lanes_per_chan=lpc, warps_per_cta=warps, grid=grid, tile_t=16),
-          expect_path=0)
+    _case(inp, dict(lanes_per_chan=lpc, warps_per_cta=warps, grid=grid, tile_t=32,
+                    chans_per_lane=1, segments=1), expect_path=0)
 
 
 @pytest.mark.parametrize("grid", [1, 2, 7, 0, 64, 5000])
 def test_schedule_grid_sizes(grid):
     """One CTA walking every unit, small grids, the default, and grids
-    larger than the rows (clamped to what is co-resident)."""
+    larger than the work (capped by the number of items)."""
     inp = synth.make_fwd(2, 1000, 128, 16, seed=22, has_h0=True)
-    _case(inp, dict(grid=grid), expect_path=0)
+    _case(inp, dict(grid=grid, segments=1), expect_path=0)
 
 
 @pytest.mark.parametrize("N", [4, 8, 16])
@@ -320,7 +295,8 @@ def test_fwd_replayed_from_a_cuda_graph():
     correctly and reproduces the eager result bit for bit."""
     inp = synth.make_fwd(3, 389, 64, 16, seed=46, has_h0=True)
     plan = gu.make_plan(inp)
-    plan.set_config(lanes_per_chan=4, warps_per_cta=4, grid=4, tile_t=32)  # 6 rows on 4 CTAs
+    plan.set_config(lanes_per_chan=4, warps_per_cta=4, grid=4, tile_t=32, chans_per_lane=1,
+                    segments=1)  # 6 rows on 4 CTAs
     assert plan.info()["parts_per_row"] >= 2
     dev = gu.upload(inp)
     y = torch.empty((inp.Bsz, inp.L, inp.D), dtype=torch.bfloat16, device="cuda")
@@ -361,7 +337,7 @@ def test_timeout_is_reported_without_hanging():
     exact again."""
     inp = synth.make_fwd(4, 512, 32, 16, seed=34)
     plan = gu.make_plan(inp)
-    plan.set_config(lanes_per_chan=4, warps_per_cta=4, grid=3)
+    plan.set_config(lanes_per_chan=4, warps_per_cta=4, grid=3, chans_per_lane=1, segments=1)
     info = plan.info()
     S, PL = info["stages_per_row"], info["stages_per_part"]
     assert info["rows"] == 4 and info["grid"] == 3 and info["parts_per_row"] >= 2, info

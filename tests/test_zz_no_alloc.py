@@ -53,6 +53,7 @@ def test_noalloc_matches_plan_entry_point(shape, dt, zoh):
     inp = synth.make_fwd(Bz, L, D, N, in_dtype=dt, seed=41, has_h0=True, zoh=zoh)
     dev = gu.upload(inp)
     plan = gu.make_plan(inp)
+    plan.set_config(segments=1)   # the launch shape the allocation-free entry point takes
     y_ref, h_ref = gu.run_gpu(inp, plan, dev)
     lib = _lib()
     for call in range(2):
@@ -92,7 +93,8 @@ def test_noalloc_timeout_is_reported():
     reports SSM_ERR_TIMEOUT, and the next call is exact again."""
     inp = synth.make_fwd(8, 512, 1536, 16, seed=43)
     dev = gu.upload(inp)
-    plan = gu.make_plan(inp)   # same default launch shape as the noalloc entry point
+    plan = gu.make_plan(inp)
+    plan.set_config(segments=1)   # the launch shape the allocation-free entry point takes
     info = plan.info()
     assert info["parts_per_row"] >= 2, info
     y_ref, h_ref = gu.run_gpu(inp, plan, dev)
