@@ -132,6 +132,8 @@ typedef struct {
   int stages_per_segment;
   int carry_grid;      /* CTAs of the carry pass (segments > 1) */
   int launches_per_call; /* kernels one ssm_scan_fwd launches (2 with segments) */
+  int scan_loop;       /* 1 + variant options: bit 0 software-pipelined scan loop,
+                          bit 1 registers capped for five CTAs per SM */
 } ssm_scan_info;
 
 /* Optional overrides of the launch shape (0 = keep the default). */
@@ -142,6 +144,10 @@ typedef struct {
   int tile_t;         /* tokens per pipeline stage: 32 or 64 */
   int chans_per_lane; /* 1 or 2 */
   int segments;       /* segments per row: 1, 2, 4 or 8 (1 = none) */
+  int scan_loop;      /* 1 + variant options (0 = free choice): option bit 0 =
+                         software-pipelined scan loop (the next token's exponentials and
+                         loads issued before this token's update), bit 1 = registers
+                         capped so five CTAs fit on an SM */
 } ssm_scan_config;
 /* Only the combinations compiled into the library exist; ssm_scan_set_config
  * returns SSM_ERR_UNSUPPORTED for others (ssm_scan_list_variants lists them). */
@@ -322,6 +328,7 @@ typedef struct {
   int zoh;   /* zero-order-hold input coefficient */
   int carry; /* the carry pass of a segmented launch (not a full scan) */
   int conv;  /* with the causal conv front-end of the x branch */
+  int opt;   /* options: bit 0 software-pipelined scan loop, bit 1 five CTAs per SM */
 } ssm_scan_variant;
 
 /* The compiled variants of the fused kernel for a dtype pair (a tuning and

@@ -8,9 +8,9 @@ namespace ssm {
 
 cudaError_t fwd_table_bf16_a(const LaunchShape *ls, const TmaMaps *maps, const FwdParams *p,
                            cudaStream_t st, VariantInfo *vi) {
-#define SSM_X(NS, LPC, KC, W, TT, ZOH, CARRY, CONV)                                    \
-  if (shape_is(ls, NS, LPC, KC, W, TT, ZOH, CARRY, CONV))                               \
-    return run_variant<__nv_bfloat16, __nv_bfloat16, NS, LPC, KC, W, TT, ZOH, CARRY, CONV>(ls, maps, p, st, vi);
+#define SSM_X(NS, LPC, KC, W, TT, ZOH, CARRY, CONV, OPT)                                  \
+  if (shape_is(ls, NS, LPC, KC, W, TT, ZOH, CARRY, CONV, OPT))                              \
+    return run_variant<__nv_bfloat16, __nv_bfloat16, NS, LPC, KC, W, TT, ZOH, CARRY, CONV, OPT>(ls, maps, p, st, vi);
   SSM_FWD_BF16_N16(SSM_X)
 #undef SSM_X
   return cudaErrorNotSupported;
@@ -18,8 +18,8 @@ cudaError_t fwd_table_bf16_a(const LaunchShape *ls, const TmaMaps *maps, const F
 
 int fwd_list_bf16_a(VariantDesc *out, int max) {
   int n = 0;
-#define SSM_X(NS, LPC, KC, W, TT, ZOH, CARRY, CONV)                                    \
-  if (n < max) out[n] = VariantDesc{NS, LPC, KC, W, TT, ZOH, CARRY, CONV};             \
+#define SSM_X(NS, LPC, KC, W, TT, ZOH, CARRY, CONV, OPT)                                  \
+  if (n < max) out[n] = VariantDesc{NS, LPC, KC, W, TT, ZOH, CARRY, CONV, OPT};              \
   ++n;
   SSM_FWD_BF16_N16(SSM_X)
 #undef SSM_X

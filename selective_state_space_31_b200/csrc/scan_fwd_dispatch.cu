@@ -90,13 +90,14 @@ namespace {
 // (bf16 layer workloads).  One channel per lane: splitting a channel over 4
 // lanes balances the per-lane B / C loads against the shuffle readout best;
 // longer stages amortise the per-stage waits but raise register pressure.
-// Two channels per lane load and widen each B / C value once for both, which
-// removes about a third of the instructions per state update.
+// Two channels per lane load and widen each B / C value once for both
+// (fewer instructions per update) but halve the lanes; measured on B200 they
+// run at about the speed of one channel per lane with the same warps busy.
 double shape_weight(int lpc, int kc, int tt) {
   const int i = tt == 16 ? 0 : tt == 32 ? 1 : 2;
   if (kc == 2) {
-    static const double v2[3] = {1.1, 1.15, 1.1}, v4[3] = {1.25, 1.3, 1.25},
-                        v8[3] = {1.1, 1.15, 1.15};
+    static const double v2[3] = {0.6, 0.65, 0.6}, v4[3] = {0.8, 0.85, 0.8},
+                        v8[3] = {0.9, 0.95, 0.95};
     return lpc == 2 ? v2[i] : lpc == 4 ? v4[i] : v8[i];
   }
   static const double w1[3] = {0.45, 0.45, 0.42}, w2[3] = {0.68, 0.75, 0.7},
@@ -111,6 +112,10 @@ double shape_weight(int lpc, int kc, int tt) {
   }
 }
 double warps_weight(int warps) { return warps == 2 ? 0.8 : 1.0; }
+
+// The software-pipelined loop and the five-CTA register cap relative to the
+// plain variant.
+double opt_weight(int opt) { return opt == 0 ? 1.0 : 0.99; }
 
 // Cost of the carry pass per state update it covers, relative to the fused
 // scan's (one exponential and the state update, no readout or gate).
@@ -190,7 +195,7 @@ cudaError_t choose_fwd_shape(int in_dtype, int out_dtype, int64_t batch, int64_t
     const VariantDesc &v = all[vi_];
     if (v.carry || v.ns != ns || v.zoh != zoh || v.conv != conv) continue;
     if ((o.lpc && v.lpc != o.lpc) || (o.warps && v.warps != o.warps) ||
-        (o.tt && v.tt != o.tt) || (o.kc && v.kc != o.kc))
+        (o.tt && v.tt != o.tt) || (o.kc && v.kc != o.kc) || (o.opt && v.opt != o.opt - 1))
       continue;
     const int DT = v.warps * (32 / v.lpc) * v.kc;
     if ((DT * ei) % 16 || (DT * eo) % 16) continue;
@@ -198,6 +203,7 @@ cudaError_t choose_fwd_shape(int in_dtype, int out_dtype, int64_t batch, int64_t
     LaunchShape ls{v.lpc, v.warps, v.tt, kStages, ns, 0, 0, zoh};
     ls.kc = v.kc;
     ls.conv = conv;
+    ls.opt = v.opt;
     VariantInfo info{};
     if (fwd_variant_info(in_dtype, out_dtype, ls, &info) != cudaSuccess || info.occ < 1) {
       cudaGetLastError();
@@ -205,7 +211,8 @@ cudaError_t choose_fwd_shape(int in_dtype, int out_dtype, int64_t batch, int64_t
     }
     const int64_t rows = batch * ((dim + DT - 1) / DT);
     const int64_t S = std::max<int64_t>(1, (seqlen + v.tt - 1) / v.tt);
-    const double w = shape_weight(v.lpc, v.kc, v.tt) * warps_weight(v.warps);
+    const double w = shape_weight(v.lpc, v.kc, v.tt) * warps_weight(v.warps) *
+                     opt_weight(v.opt);
     for (int M : {1, 2, 4, 8}) {
       if (o.segments && M != o.segments) continue;
       if (M > 1 && S < 4 * M) continue;  // each segment keeps a few stages
@@ -291,7 +298,7 @@ cudaError_t choose_map_shape(int in_dtype, int out_dtype, int64_t batch, int64_t
   VariantDesc all[kMaxVariants];
   const int nall = std::min(kMaxVariants, fwd_variants(in_dtype, out_dtype, all, kMaxVariants));
   const VariantDesc main{fs.ls.ns, fs.ls.lpc, fs.ls.kc, fs.ls.warps, fs.ls.tt, fs.ls.zoh, false,
-                         fs.ls.conv};
+                         fs.ls.conv, 0};
   LaunchShape cls{};
   int cDT = 0, cocc = 0;
   if (!pick_carry(in_dtype, out_dtype, main, sms, all, nall, &cls, &cDT, &cocc))

@@ -220,9 +220,11 @@ struct ItemPos {
 // CARRY = false: the fused forward scan.  CARRY = true: the carry pass over
 // sub-chunks of PL stages (items independent, no readout): each item scans
 // its stages from h = 0 and records (sum of Delta, h_end) per channel.
+// OPT bit 0: software-pipelined scan loop (one channel per lane); bit 1:
+// registers capped so that five CTAs fit on an SM (more warps in flight).
 template <typename InT, typename OutT, int NS, int LPC, int KC, int WARPS, int TT, bool ZOH,
-          bool CARRY, bool CONV>
-__global__ void __launch_bounds__((WARPS + 1) * 32)
+          bool CARRY, bool CONV, int OPT>
+__global__ void __launch_bounds__((WARPS + 1) * 32, (OPT & 2) ? 5 : 0)
     fwd_kernel(const __grid_constant__ TmaMaps maps, const FwdParams p) {
   using Cfg = FwdCfg<InT, OutT, NS, LPC, KC, WARPS, TT, CONV>;
   constexpr int NPL = Cfg::NPL, GPW = Cfg::GPW, DT = Cfg::DT, RAW = Cfg::RAW,
@@ -491,6 +493,55 @@ __global__ void __launch_bounds__((WARPS + 1) * 32)
 
         // -- the scan over TT tokens of this lane's channel --
         const float2 *prow = plane + g_loc * Cfg::TTP;
+        if constexpr ((OPT & 1) && !CARRY && !ZOH && NPL % 2 == 0) {
+          // Software-pipelined form: the exponentials, input terms and C of
+          // token t + 1 are formed (loads, ex2) before token t's state update
+          // consumes those of token t, so the special-function latency and
+          // the shared-memory loads overlap the update chain.
+          constexpr int NP = NPL / 2;
+          float2 an[NP], bn[NP], cn[NP];
+          auto prep = [&](int t, float2 (&a)[NP], float2 (&bx)[NP], float2 (&cc)[NP]) {
+            const float4 dp = *reinterpret_cast<const float4 *>(prow + (t & ~1));
+            const float2 dd = (t & 1) ? make_float2(dp.z, dp.w) : make_float2(dp.x, dp.y);
+            float bv[NPL], cv[NPL];
+            load_bc<NPL>(Bs + t * NS + q * NPL, bv);
+            load_bc<NPL>(Cs + t * NS + q * NPL, cv);
+            const float2 dA = make_float2(dd.x, dd.x), dX = make_float2(dd.y, dd.y);
+#pragma unroll
+            for (int k = 0; k < NP; ++k) {
+              const float2 arg = fmul2(dA, make_float2(A2[0][2 * k], A2[0][2 * k + 1]));
+              a[k] = make_float2(ex2_approx(arg.x), ex2_approx(arg.y));
+              bx[k] = fmul2(dX, make_float2(bv[2 * k], bv[2 * k + 1]));
+              cc[k] = make_float2(cv[2 * k], cv[2 * k + 1]);
+            }
+          };
+          prep(0, an, bn, cn);
+#pragma unroll
+          for (int tt = 0; tt < TT; tt += LPC) {
+            float yp[LPC];
+#pragma unroll
+            for (int j = 0; j < LPC; ++j) {
+              const int t = tt + j;
+              float2 ac[NP], bc[NP], ccur[NP];
+#pragma unroll
+              for (int k = 0; k < NP; ++k) { ac[k] = an[k]; bc[k] = bn[k]; ccur[k] = cn[k]; }
+              if (t + 1 < TT) prep(t + 1, an, bn, cn);
+              float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+              for (int k = 0; k < NP; ++k) {
+                const float2 hn = ffma2(ac[k], make_float2(h[0][2 * k], h[0][2 * k + 1]), bc[k]);
+                h[0][2 * k] = hn.x;
+                h[0][2 * k + 1] = hn.y;
+                acc = ffma2(ccur[k], hn, acc);
+              }
+              yp[j] = acc.x + acc.y;
+            }
+            const float ys = reduce_scatter<LPC>(yp, q);
+            const int to = tt + q;
+            if (to < nvalid && valid_ch)
+              yrow[(size_t)to * p.D] = from_f32<OutT>(fmaf(ys, g1[tt / LPC], g2[tt / LPC]));
+          }
+        } else {
         float4 dpair;  // (Delta, Delta*x) of an even token and the next, one 16-byte load
 #pragma unroll
         for (int tt = 0; tt < TT; tt += LPC) {
@@ -538,6 +589,7 @@ __global__ void __launch_bounds__((WARPS + 1) * 32)
             if (to < nvalid && valid_ch)
               yrow[(size_t)to * p.D] = from_f32<OutT>(fmaf(ys, g1[tt / LPC], g2[tt / LPC]));
           }
+        }
         }
       } else {
         // ------------- two channels per lane: ch0 and ch0 + 1 -------------
@@ -677,11 +729,11 @@ __global__ void __launch_bounds__((WARPS + 1) * 32)
 // ---------------------------------------------------------------------------
 
 template <typename InT, typename OutT, int NS, int LPC, int KC, int WARPS, int TT, bool ZOH,
-          bool CARRY, bool CONV>
+          bool CARRY, bool CONV, int OPT>
 static cudaError_t run_variant(const LaunchShape *ls, const TmaMaps *maps, const FwdParams *p,
                                cudaStream_t stream, VariantInfo *vi) {
   using Cfg = FwdCfg<InT, OutT, NS, LPC, KC, WARPS, TT, CONV>;
-  auto kern = fwd_kernel<InT, OutT, NS, LPC, KC, WARPS, TT, ZOH, CARRY, CONV>;
+  auto kern = fwd_kernel<InT, OutT, NS, LPC, KC, WARPS, TT, ZOH, CARRY, CONV, OPT>;
   if (Cfg::SMEM + 8 * Cfg::RAW > 227 * 1024) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
   if (e != cudaSuccess) {
@@ -701,9 +753,9 @@ static cudaError_t run_variant(const LaunchShape *ls, const TmaMaps *maps, const
 
 // Does a launch shape ask for this compiled variant?
 inline bool shape_is(const LaunchShape *ls, int ns, int lpc, int kc, int warps, int tt, bool zoh,
-                     bool carry, bool conv) {
+                     bool carry, bool conv, int opt) {
   return ls->ns == ns && ls->lpc == lpc && ls->kc == kc && ls->warps == warps && ls->tt == tt &&
-         ls->zoh == zoh && ls->carry == carry && ls->conv == conv;
+         ls->zoh == zoh && ls->carry == carry && ls->conv == conv && ls->opt == opt;
 }
 
 }  // namespace ssm

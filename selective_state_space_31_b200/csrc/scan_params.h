@@ -65,6 +65,7 @@ struct LaunchShape {
   int kc = 1;  // channels per lane
   bool carry = false;  // the carry pass of a segmented launch
   bool conv = false;   // the x branch comes through the causal conv front-end
+  int opt = 0;         // bit 0: software-pipelined scan loop; bit 1: five CTAs per SM
 };
 
 // Fused forward kernel (scan_fwd_kernel.cuh, instantiated per dtype pair).
@@ -87,6 +88,7 @@ struct FwdOverrides {
   int lpc, warps, tt, grid;
   int kc = 0;        // channels per lane
   int segments = 0;  // segments per row (1 = none)
+  int opt = 0;       // 1 + the variant's OPT bits (0 = free choice)
 };
 // A launch shape of the fused kernel with its work split.
 struct FwdShape {
@@ -123,6 +125,7 @@ cudaError_t choose_map_shape(int in_dtype, int out_dtype, int64_t batch, int64_t
 struct VariantDesc {
   int ns, lpc, kc, warps, tt;
   bool zoh, carry, conv;
+  int opt;
 };
 // The variants compiled for a dtype pair; returns how many (fills up to max).
 int fwd_variants(int in_dtype, int out_dtype, VariantDesc *out, int max);

@@ -150,6 +150,7 @@ ssm_status plan_tma(ssm_scan_plan *pl) {
                       pl->cfg.grid};
   o.kc = pl->cfg.chans_per_lane;
   o.segments = pl->cfg.segments;
+  o.opt = pl->cfg.scan_loop;
   ssm::FwdShape fs;
   if (ssm::choose_fwd_shape((int)d.in_dtype, (int)d.out_dtype, d.batch, d.seqlen, d.dim, ns,
                             (d.flags & SSM_ZOH) != 0, (d.flags & SSM_CONV_X) != 0, pl->num_sms, o,
@@ -242,7 +243,8 @@ int ssm_scan_list_variants(ssm_dtype in_dtype, ssm_dtype out_dtype, ssm_scan_var
   if (out)
     for (int i = 0; i < n && i < max; ++i)
       out[i] = ssm_scan_variant{v[i].ns, v[i].lpc, v[i].kc, v[i].warps, v[i].tt,
-                                v[i].zoh ? 1 : 0, v[i].carry ? 1 : 0, v[i].conv ? 1 : 0};
+                                v[i].zoh ? 1 : 0, v[i].carry ? 1 : 0, v[i].conv ? 1 : 0,
+                                v[i].opt};
   return n;
 }
 
@@ -323,6 +325,7 @@ ssm_status ssm_scan_get_info(const ssm_scan_plan *pl, ssm_scan_info *info) {
     info->segments = pl->fs.M;
     info->stages_per_segment = pl->fs.SPS;
     info->carry_grid = pl->fs.M > 1 ? pl->fs.cls.grid : 0;
+    info->scan_loop = 1 + pl->ls.opt;
   }
   info->launches_per_call = pl->path == PATH_TMA && pl->fs.M > 1 ? 2 : 1;
   info->workspace_bytes =
@@ -333,7 +336,7 @@ ssm_status ssm_scan_get_info(const ssm_scan_plan *pl, ssm_scan_info *info) {
 ssm_status ssm_scan_set_config(ssm_scan_plan *pl, const ssm_scan_config *cfg) {
   if (!pl || !cfg) return SSM_ERR_INVALID_ARG;
   if (cfg->lanes_per_chan < 0 || cfg->warps_per_cta < 0 || cfg->grid < 0 || cfg->tile_t < 0 ||
-      cfg->chans_per_lane < 0 || cfg->segments < 0)
+      cfg->chans_per_lane < 0 || cfg->segments < 0 || cfg->scan_loop < 0 || cfg->scan_loop > 4)
     return SSM_ERR_INVALID_ARG;
   DeviceGuard guard(pl->device);
   if (!guard.ok) return SSM_ERR_CUDA;

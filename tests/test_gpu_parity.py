@@ -210,8 +210,10 @@ def test_decode_streaming_many_tiles_per_cta():
 @pytest.mark.parametrize("cfg", [None, dict(lanes_per_chan=4, warps_per_cta=4, tile_t=32),
                                  dict(lanes_per_chan=8, warps_per_cta=4, tile_t=64, grid=2),
                                  dict(lanes_per_chan=16, warps_per_cta=4, tile_t=64),
-                                 dict(lanes_per_chan=1, warps_per_cta=2, tile_t=32),
-                                 dict(lanes_per_chan=2, warps_per_cta=8, tile_t=64)])
+                                 dict(lanes_per_chan=4, warps_per_cta=4, tile_t=32,
+                                      chans_per_lane=2),
+                                 dict(lanes_per_chan=8, warps_per_cta=4, tile_t=32,
+                                      chans_per_lane=2, segments=2)])
 @pytest.mark.parametrize("shift", [0.0, 3.0])
 def test_zoh_fused(cfg, shift):
     """Zero-order hold ([P1] "Vi du Python": Bbar = (exp(Delta A) - 1)/A * B)

@@ -44,7 +44,7 @@ def _sweep(inp, in_dt, out_dt, segments_list, grids=(0,)):
             for grid in grids:
                 cfg = dict(lanes_per_chan=v["lanes_per_chan"], warps_per_cta=v["warps_per_cta"],
                            tile_t=v["tile_t"], chans_per_lane=v["chans_per_lane"],
-                           segments=M, grid=grid)
+                           segments=M, grid=grid, scan_loop=1 + v["opt"])
                 try:
                     info, gy, gh, st = _run(inp, dev, cfg)
                 except bnd.SsmError as e:
@@ -54,7 +54,8 @@ def _sweep(inp, in_dt, out_dt, segments_list, grids=(0,)):
                 key = (info["lanes_per_chan"], info["chans_per_lane"], info["warps_per_cta"],
                        info["tile_t"])
                 if key != (v["lanes_per_chan"], v["chans_per_lane"], v["warps_per_cta"],
-                           v["tile_t"]) or info["segments"] != M:
+                           v["tile_t"]) or info["segments"] != M or \
+                        info["scan_loop"] != 1 + v["opt"]:
                     failures.append(f"{cfg}: plan chose {info}")
                 if M > 1:
                     carries.add((v["lanes_per_chan"], v["chans_per_lane"], v["tile_t"]))
