@@ -113,9 +113,20 @@ double shape_weight(int lpc, int kc, int tt) {
 }
 double warps_weight(int warps) { return warps == 2 ? 0.8 : 1.0; }
 
-// The software-pipelined loop and the five-CTA register cap relative to the
-// plain variant.
-double opt_weight(int opt) { return opt == 0 ? 1.0 : 0.99; }
+// The software-pipelined loop (bit 0) and the five-CTA register cap (bit 1)
+// relative to the plain variant, measured on B200: with 8 lanes per channel
+// and 64-token stages the pipelined loop gains 3-5 % on the layer shapes;
+// elsewhere, and with segments, the plain loop was as fast or faster.
+double opt_weight(int opt, int lpc, int tt, int segments) {
+  if (opt == 0) return 1.0;
+  if (segments > 1 || lpc != 8 || tt != 64) return 0.97;
+  return opt == 1 ? 1.05 : opt == 2 ? 1.04 : 1.03;
+}
+// With segments, the 131k-token rows favoured 4 lanes x 32-token stages over
+// 8 lanes x 64-token stages by about 10 % more than the layer shapes do.
+double segmented_weight(int lpc, int tt, int segments) {
+  return segments > 1 && lpc == 8 && tt == 64 ? 0.93 : 1.0;
+}
 
 // Cost of the carry pass per state update it covers, relative to the fused
 // scan's (one exponential and the state update, no readout or gate).
@@ -151,7 +162,11 @@ bool pick_carry(int in_dtype, int out_dtype, const VariantDesc &main, int sms,
     if (!v.carry || v.ns != main.ns || v.zoh != main.zoh || v.tt != main.tt ||
         v.conv != main.conv)
       continue;
-    const double score = (v.lpc == main.lpc && v.kc == main.kc ? 2.0 : 0.0) +
+    // one lane per channel needs no shared plane and no shuffles: the leanest
+    // carry pass (every item is independent, so its fewer lanes still fill
+    // the device); then the main variant's own split
+    const double score = (v.lpc == 1 ? 4.0 + (v.warps == 2 ? 0.1 : 0.0) : 0.0) +
+                         (v.lpc == main.lpc && v.kc == main.kc ? 2.0 : 0.0) +
                          (v.kc == 2 ? 0.5 : 0.0) + (v.lpc == 4 ? 0.25 : 0.0);
     if (score > best_score) { best_score = score; best = i; }
   }
@@ -211,10 +226,10 @@ cudaError_t choose_fwd_shape(int in_dtype, int out_dtype, int64_t batch, int64_t
     }
     const int64_t rows = batch * ((dim + DT - 1) / DT);
     const int64_t S = std::max<int64_t>(1, (seqlen + v.tt - 1) / v.tt);
-    const double w = shape_weight(v.lpc, v.kc, v.tt) * warps_weight(v.warps) *
-                     opt_weight(v.opt);
     for (int M : {1, 2, 4, 8}) {
       if (o.segments && M != o.segments) continue;
+      const double w = shape_weight(v.lpc, v.kc, v.tt) * warps_weight(v.warps) *
+                       opt_weight(v.opt, v.lpc, v.tt, M) * segmented_weight(v.lpc, v.tt, M);
       if (M > 1 && S < 4 * M) continue;  // each segment keeps a few stages
       LaunchShape cls{};
       int cDT = 0, cocc = 0;

@@ -62,7 +62,7 @@ constexpr int align_up(int v, int a) { return (v + a - 1) / a * a; }
 constexpr int clamp_int(int v, int lo, int hi) { return v < lo ? lo : (v > hi ? hi : v); }
 
 template <typename InT, typename OutT, int NS, int LPC, int KC, int WARPS, int TT,
-          bool CONV = false>
+          bool CONV = false, bool CARRY = false>
 struct FwdCfg {
   static constexpr int NPL = NS / LPC;    // states per lane and channel
   static constexpr int GPW = 32 / LPC;    // channel groups per scan warp
@@ -76,9 +76,10 @@ struct FwdCfg {
   static constexpr int XTILE = align_up(TT * DT * (int)sizeof(InT), 128);
   static constexpr int XTILE_X = align_up((TT + XHALO) * DT * (int)sizeof(InT), 128);
   static constexpr int BCTILE = align_up(TT * NS * (int)sizeof(InT), 128);
-  static constexpr int OFF_DT = XTILE_X, OFF_Z = XTILE_X + XTILE, OFF_B = XTILE_X + 2 * XTILE,
-                       OFF_C = OFF_B + BCTILE;
-  static constexpr int SLOT = OFF_C + BCTILE;
+  // (the carry pass reads neither z nor C: its slots hold x, delta and B only)
+  static constexpr int OFF_DT = XTILE_X, OFF_Z = XTILE_X + XTILE,
+                       OFF_B = XTILE_X + (CARRY ? 1 : 2) * XTILE, OFF_C = OFF_B + BCTILE;
+  static constexpr int SLOT = OFF_C + (CARRY ? 0 : BCTILE);
   // ring depth: ~128 tokens of prefetch, within ~64 KB, at least 3 slots
   static constexpr int RAW = clamp_int(65536 / SLOT, 3, 128 / TT > 3 ? 128 / TT : 3);
   // Per warp, channel-group-major plane of per-token values: KC = 1 keeps
@@ -226,7 +227,7 @@ template <typename InT, typename OutT, int NS, int LPC, int KC, int WARPS, int T
           bool CARRY, bool CONV, int OPT>
 __global__ void __launch_bounds__((WARPS + 1) * 32, (OPT & 2) ? 5 : 0)
     fwd_kernel(const __grid_constant__ TmaMaps maps, const FwdParams p) {
-  using Cfg = FwdCfg<InT, OutT, NS, LPC, KC, WARPS, TT, CONV>;
+  using Cfg = FwdCfg<InT, OutT, NS, LPC, KC, WARPS, TT, CONV, CARRY>;
   constexpr int NPL = Cfg::NPL, GPW = Cfg::GPW, DT = Cfg::DT, RAW = Cfg::RAW,
                 TPL = Cfg::TPL;
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -732,7 +733,7 @@ template <typename InT, typename OutT, int NS, int LPC, int KC, int WARPS, int T
           bool CARRY, bool CONV, int OPT>
 static cudaError_t run_variant(const LaunchShape *ls, const TmaMaps *maps, const FwdParams *p,
                                cudaStream_t stream, VariantInfo *vi) {
-  using Cfg = FwdCfg<InT, OutT, NS, LPC, KC, WARPS, TT, CONV>;
+  using Cfg = FwdCfg<InT, OutT, NS, LPC, KC, WARPS, TT, CONV, CARRY>;
   auto kern = fwd_kernel<InT, OutT, NS, LPC, KC, WARPS, TT, ZOH, CARRY, CONV, OPT>;
   if (Cfg::SMEM + 8 * Cfg::RAW > 227 * 1024) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);

@@ -23,6 +23,8 @@
   X(16, 8, 2, 4, 32, false, false, false, 0) X(16, 8, 2, 4, 64, false, false, false, 0)                      \
   X(16, 4, 2, 8, 32, false, false, false, 0) X(16, 8, 2, 8, 32, false, false, false, 0)
 #define SSM_FWD_BF16_N16_ZOH_CARRY(X)                                                    \
+  X(16, 1, 1, 4, 32, false, true, false, 0) X(16, 1, 1, 2, 32, false, true, false, 0)    \
+  X(16, 1, 1, 2, 64, false, true, false, 0)                                              \
   X(16, 4, 1, 4, 32, true, false, false, 0) X(16, 4, 1, 4, 64, true, false, false, 0)                        \
   X(16, 8, 1, 4, 32, true, false, false, 0) X(16, 8, 1, 4, 64, true, false, false, 0)                        \
   X(16, 16, 1, 4, 32, true, false, false, 0) X(16, 16, 1, 4, 64, true, false, false, 0)                      \
