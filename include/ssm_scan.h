@@ -133,7 +133,10 @@ typedef struct {
   int carry_grid;      /* CTAs of the carry pass (segments > 1) */
   int launches_per_call; /* kernels one ssm_scan_fwd launches (2 with segments) */
   int scan_loop;       /* 1 + variant options: bit 0 software-pipelined scan loop,
-                          bit 1 registers capped for five CTAs per SM */
+                          bit 1 registers capped for five CTAs per SM, bit 2 B and C
+                          widened to fp32 once per CTA (bf16 inputs) */
+  int carry_lanes_per_chan; /* lanes per channel of the carry pass (segments > 1) */
+  int carry_loop;      /* 1 + the carry pass's variant options (segments > 1) */
 } ssm_scan_info;
 
 /* Optional overrides of the launch shape (0 = keep the default). */
@@ -147,7 +150,10 @@ typedef struct {
   int scan_loop;      /* 1 + variant options (0 = free choice): option bit 0 =
                          software-pipelined scan loop (the next token's exponentials and
                          loads issued before this token's update), bit 1 = registers
-                         capped so five CTAs fit on an SM */
+                         capped so five CTAs fit on an SM, bit 2 = the load warp widens
+                         each stage's B and C to fp32 once for the CTA (bf16 inputs) */
+  int carry_lanes_per_chan; /* carry pass of a segmented scan: lanes per channel (0 = free) */
+  int carry_loop;     /* carry pass: 1 + its variant options, as scan_loop (0 = free) */
 } ssm_scan_config;
 /* Only the combinations compiled into the library exist; ssm_scan_set_config
  * returns SSM_ERR_UNSUPPORTED for others (ssm_scan_list_variants lists them). */

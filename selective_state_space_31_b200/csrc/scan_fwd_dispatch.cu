@@ -150,23 +150,25 @@ int parts_per_chain(int64_t R, int64_t P, int64_t S) {
   return best_m;
 }
 
-// The carry pass for a main variant: same stage length and zero-order-hold
-// flag; prefer the main variant's own lane split, then fewer lanes per
-// channel.
+// The carry pass for a main variant: same dstate, stage length, zero-order
+// hold and conv flags.  Measured on B200 (131k-token rows, 8 segments): the
+// carry pass in the main variant's own lane split ran its exponentials at
+// ~76 % of the special-function rate, while one lane per channel (few warps
+// per SM) took 45 % longer.  So: the main variant's split and its B/C
+// widening option first, then 4 lanes per channel.  o_lpc / o_opt (1 + the
+// OPT bits) restrict the choice when non-zero.
 bool pick_carry(int in_dtype, int out_dtype, const VariantDesc &main, int sms,
-                const VariantDesc *all, int nall, LaunchShape *cls, int *cDT, int *cocc) {
+                const VariantDesc *all, int nall, int o_lpc, int o_opt, LaunchShape *cls,
+                int *cDT, int *cocc) {
   int best = -1;
   double best_score = -1.0;
   for (int i = 0; i < nall; ++i) {
     const VariantDesc &v = all[i];
     if (!v.carry || v.ns != main.ns || v.zoh != main.zoh || v.tt != main.tt ||
-        v.conv != main.conv)
+        v.conv != main.conv || (o_lpc && v.lpc != o_lpc) || (o_opt && v.opt != o_opt - 1))
       continue;
-    // one lane per channel needs no shared plane and no shuffles: the leanest
-    // carry pass (every item is independent, so its fewer lanes still fill
-    // the device); then the main variant's own split
-    const double score = (v.lpc == 1 ? 4.0 + (v.warps == 2 ? 0.1 : 0.0) : 0.0) +
-                         (v.lpc == main.lpc && v.kc == main.kc ? 2.0 : 0.0) +
+    const double score = (v.lpc == main.lpc && v.kc == main.kc ? 2.0 : 0.0) +
+                         ((v.opt & 4) == (main.opt & 4) ? 1.0 : 0.0) +
                          (v.kc == 2 ? 0.5 : 0.0) + (v.lpc == 4 ? 0.25 : 0.0);
     if (score > best_score) { best_score = score; best = i; }
   }
@@ -176,6 +178,7 @@ bool pick_carry(int in_dtype, int out_dtype, const VariantDesc &main, int sms,
   ls.kc = v.kc;
   ls.carry = true;
   ls.conv = v.conv;
+  ls.opt = v.opt;
   VariantInfo vi{};
   if (fwd_variant_info(in_dtype, out_dtype, ls, &vi) != cudaSuccess || vi.occ < 1) {
     cudaGetLastError();
@@ -233,7 +236,8 @@ cudaError_t choose_fwd_shape(int in_dtype, int out_dtype, int64_t batch, int64_t
       if (M > 1 && S < 4 * M) continue;  // each segment keeps a few stages
       LaunchShape cls{};
       int cDT = 0, cocc = 0;
-      if (M > 1 && !pick_carry(in_dtype, out_dtype, v, sms, all, nall, &cls, &cDT, &cocc))
+      if (M > 1 && !pick_carry(in_dtype, out_dtype, v, sms, all, nall, o.carry_lpc, o.carry_opt,
+                               &cls, &cDT, &cocc))
         continue;
       const int64_t vrows = rows * M;
       const int64_t cap = std::min(vrows, (int64_t)info.occ * sms);
@@ -313,10 +317,10 @@ cudaError_t choose_map_shape(int in_dtype, int out_dtype, int64_t batch, int64_t
   VariantDesc all[kMaxVariants];
   const int nall = std::min(kMaxVariants, fwd_variants(in_dtype, out_dtype, all, kMaxVariants));
   const VariantDesc main{fs.ls.ns, fs.ls.lpc, fs.ls.kc, fs.ls.warps, fs.ls.tt, fs.ls.zoh, false,
-                         fs.ls.conv, 0};
+                         fs.ls.conv, fs.ls.opt};
   LaunchShape cls{};
   int cDT = 0, cocc = 0;
-  if (!pick_carry(in_dtype, out_dtype, main, sms, all, nall, &cls, &cDT, &cocc))
+  if (!pick_carry(in_dtype, out_dtype, main, sms, all, nall, 0, 0, &cls, &cDT, &cocc))
     return cudaErrorInvalidValue;
   const int64_t rows = batch * ((dim + cDT - 1) / cDT);
   const int64_t S = fs.S;

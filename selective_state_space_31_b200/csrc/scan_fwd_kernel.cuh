@@ -53,6 +53,8 @@
 //     ragged tails.
 #pragma once
 
+#include <type_traits>
+
 #include "device_common.cuh"
 #include "scan_params.h"
 
@@ -62,7 +64,7 @@ constexpr int align_up(int v, int a) { return (v + a - 1) / a * a; }
 constexpr int clamp_int(int v, int lo, int hi) { return v < lo ? lo : (v > hi ? hi : v); }
 
 template <typename InT, typename OutT, int NS, int LPC, int KC, int WARPS, int TT,
-          bool CONV = false, bool CARRY = false>
+          bool CONV = false, bool CARRY = false, bool BCF = false>
 struct FwdCfg {
   static constexpr int NPL = NS / LPC;    // states per lane and channel
   static constexpr int GPW = 32 / LPC;    // channel groups per scan warp
@@ -79,9 +81,16 @@ struct FwdCfg {
   // (the carry pass reads neither z nor C: its slots hold x, delta and B only)
   static constexpr int OFF_DT = XTILE_X, OFF_Z = XTILE_X + XTILE,
                        OFF_B = XTILE_X + (CARRY ? 1 : 2) * XTILE, OFF_C = OFF_B + BCTILE;
-  static constexpr int SLOT = OFF_C + (CARRY ? 0 : BCTILE);
-  // ring depth: ~128 tokens of prefetch, within ~64 KB, at least 3 slots
-  static constexpr int RAW = clamp_int(65536 / SLOT, 3, 128 / TT > 3 ? 128 / TT : 3);
+  // BCF: the load warp widens the stage's B (and C) to fp32 beside the bf16
+  // tiles, once per CTA, so the scan warps read fp32 values
+  static constexpr int OFF_BF = OFF_C + (CARRY ? 0 : BCTILE);
+  static constexpr int BFTILE = BCF ? align_up(TT * NS * 4, 128) : 0;
+  static constexpr int OFF_CF = OFF_BF + BFTILE;
+  static constexpr int SLOT = OFF_BF + (CARRY ? 1 : 2) * BFTILE;
+  // ring depth: ~128 tokens of prefetch, within ~64 KB (~40 KB with the
+  // wider BCF slots, so that four CTAs still fit), at least 3 slots
+  static constexpr int RAW =
+      clamp_int((BCF ? 40960 : 65536) / SLOT, 3, 128 / TT > 3 ? 128 / TT : 3);
   // Per warp, channel-group-major plane of per-token values: KC = 1 keeps
   // (Delta, Delta*x) as a float2, KC = 2 (Delta0, Delta1, Delta*x0, Delta*x1)
   // as a float4.  Row g holds tokens 0..TT-1 of group g; the TTP - TT pad
@@ -91,7 +100,7 @@ struct FwdCfg {
   static constexpr int PLANE = align_up(TTP * GPW * ESZ, 128);
   static constexpr int OFF_PLANE = RAW * SLOT;
   static constexpr int OFF_BAR = OFF_PLANE + WARPS * PLANE;
-  static constexpr int SMEM = OFF_BAR + 2 * RAW * 8;
+  static constexpr int SMEM = OFF_BAR + (BCF ? 3 : 2) * RAW * 8;
   static_assert(NS % LPC == 0, "LPC must divide N");
   static_assert(TT % LPC == 0, "LPC must divide the stage length");
   static_assert(KC == 1 || KC == 2, "one or two channels per lane");
@@ -180,6 +189,23 @@ __device__ __forceinline__ void load_bc(const __nv_bfloat16 *src, float (&dst)[N
   }
 }
 
+// Widen a tile of `N` bf16 values (N a multiple of 128) to fp32 with the 32
+// lanes of a warp: per round lane i turns the 4 values at 8-byte word i into
+// one 16-byte store, so both the reads and the writes of a round are
+// consecutive in the banks.
+template <int N>
+__device__ __forceinline__ void widen_tile(const __nv_bfloat16 *src, float *dst, int lane) {
+  static_assert(N % 128 == 0, "whole rounds of 32 lanes x 4 values");
+#pragma unroll
+  for (int i = 0; i < N / 128; ++i) {
+    const uint2 w = reinterpret_cast<const uint2 *>(src)[i * 32 + lane];
+    float4 f;
+    widen_bf16x2(w.x, f.x, f.y);
+    widen_bf16x2(w.y, f.z, f.w);
+    reinterpret_cast<float4 *>(dst)[i * 32 + lane] = f;
+  }
+}
+
 // Two adjacent channels' values of one token (x, delta or z) as fp32.
 __device__ __forceinline__ float2 load_pair(const float *src) {
   return *reinterpret_cast<const float2 *>(src);
@@ -222,12 +248,16 @@ struct ItemPos {
 // sub-chunks of PL stages (items independent, no readout): each item scans
 // its stages from h = 0 and records (sum of Delta, h_end) per channel.
 // OPT bit 0: software-pipelined scan loop (one channel per lane); bit 1:
-// registers capped so that five CTAs fit on an SM (more warps in flight).
+// registers capped so that five CTAs fit on an SM (more warps in flight);
+// bit 2 (bf16 inputs): the load warp widens each stage's B and C to fp32 in
+// shared memory once for the CTA, instead of every lane widening the values
+// it reads at every token.
 template <typename InT, typename OutT, int NS, int LPC, int KC, int WARPS, int TT, bool ZOH,
           bool CARRY, bool CONV, int OPT>
 __global__ void __launch_bounds__((WARPS + 1) * 32, (OPT & 2) ? 5 : 0)
     fwd_kernel(const __grid_constant__ TmaMaps maps, const FwdParams p) {
-  using Cfg = FwdCfg<InT, OutT, NS, LPC, KC, WARPS, TT, CONV, CARRY>;
+  constexpr bool BCF = (OPT & 4) != 0 && std::is_same<InT, __nv_bfloat16>::value;
+  using Cfg = FwdCfg<InT, OutT, NS, LPC, KC, WARPS, TT, CONV, CARRY, BCF>;
   constexpr int NPL = Cfg::NPL, GPW = Cfg::GPW, DT = Cfg::DT, RAW = Cfg::RAW,
                 TPL = Cfg::TPL;
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -235,6 +265,7 @@ __global__ void __launch_bounds__((WARPS + 1) * 32, (OPT & 2) ? 5 : 0)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   uint64_t *rfull = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_BAR);
   uint64_t *rempty = rfull + RAW;  // all scan warps are done with a slot
+  uint64_t *rconv = rempty + RAW;  // BCF: the slot's B and C are widened (32 arrivals)
 
   // item and stage carried by each ring slot (written by the load warp
   // before the slot's full barrier completes; item -1 ends the CTA's work)
@@ -248,62 +279,90 @@ __global__ void __launch_bounds__((WARPS + 1) * 32, (OPT & 2) ? 5 : 0)
     for (int i = 0; i < RAW; ++i) {
       mbar_init(&rfull[i], 1);
       mbar_init(&rempty[i], WARPS);
+      if constexpr (BCF) mbar_init(&rconv[i], 32);
     }
     fence_mbar_init();
   }
   __syncthreads();
 
   if (warp == WARPS) {
-    // =================== load warp (one thread issues) ===================
-    if (lane == 0) {
-      const bool with_z = !CARRY && p.has_z;
-      const uint32_t tx_bytes = (TT + Cfg::XHALO + (with_z ? 2u : 1u) * TT) * DT * sizeof(InT) +
-                                (CARRY ? 1u : 2u) * TT * NS * sizeof(InT);
-      ItemPos iss;
-      int st = 0;
-      bool ok = true;
-      int k = 0;
-      for (;; ++k) {
-        const int r = k % RAW;
+    // ============ load warp (one thread issues; with BCF all 32 widen) ============
+    const bool with_z = !CARRY && p.has_z;
+    const uint32_t tx_bytes = (TT + Cfg::XHALO + (with_z ? 2u : 1u) * TT) * DT * sizeof(InT) +
+                              (CARRY ? 1u : 2u) * TT * NS * sizeof(InT);
+    ItemPos iss;
+    int st = 0;
+    int k = 0, issued = 0;
+    int state = 0;  // 0: stage k issued, 1: no work left, 2: gave up waiting
+    for (;; ++k) {
+      const int r = k % RAW;
+      if (lane == 0) {
+        state = 0;
         if (k >= RAW &&
             !mbar_wait_bounded(&rempty[r], (uint32_t)(((k / RAW) - 1) & 1), p.timeout_ns)) {
-          ok = false;
-          break;
-        }
-        // next item when this one is done (parts past a short segment's end
-        // have no stages and are skipped)
-        bool done = false;
-        while (iss.item < 0 || st == iss.st_end) {
-          const int it = (int)atomicAdd(&p.ctl->ticket, 1u);
-          if (it >= p.items) {
-            done = true;
-            break;
+          state = 2;
+        } else {
+          // next item when this one is done (parts past a short segment's end
+          // have no stages and are skipped)
+          while (iss.item < 0 || st == iss.st_end) {
+            const int it = (int)atomicAdd(&p.ctl->ticket, 1u);
+            if (it >= p.items) {
+              state = 1;
+              break;
+            }
+            iss.set(it, p);
+            st = iss.st_begin;
           }
-          iss.set(it, p);
-          st = iss.st_begin;
+          if (state == 1) {  // no work left: end marker, no data
+            slot_work[r] = make_int2(-1, 0);
+            if constexpr (!BCF) mbar_arrive(&rfull[r]);
+          } else {
+            slot_work[r] = make_int2(iss.item, st);
+            const int d0 = iss.dtile * DT, t0 = st * TT, b = iss.b;
+            unsigned char *sb = smem + r * Cfg::SLOT;
+            mbar_arrive_expect_tx(&rfull[r], tx_bytes);
+            tma_load_3d(sb, &maps.x, &rfull[r], d0, t0 - Cfg::XHALO, b);
+            tma_load_3d(sb + Cfg::OFF_DT, &maps.dt, &rfull[r], d0, t0, b);
+            if (with_z) tma_load_3d(sb + Cfg::OFF_Z, &maps.z, &rfull[r], d0, t0, b);
+            tma_load_3d(sb + Cfg::OFF_B, &maps.B, &rfull[r], 0, t0, b);
+            if (!CARRY) tma_load_3d(sb + Cfg::OFF_C, &maps.C, &rfull[r], 0, t0, b);
+            ++st;
+            issued = k + 1;
+          }
         }
-        if (done) {  // no work left: end marker, no data
-          slot_work[r] = make_int2(-1, 0);
-          mbar_arrive(&rfull[r]);
-          break;
+      }
+      if constexpr (BCF) {
+        // widen the previous stage while this one is in flight, then release
+        // it to the scan warps (which wait on rconv, then on rfull)
+        state = __shfl_sync(FULL_MASK, state, 0);
+        if (state != 2 && k > 0) {
+          const int rp = (k - 1) % RAW;
+          if (!__all_sync(FULL_MASK, mbar_wait_bounded(&rfull[rp], (uint32_t)(((k - 1) / RAW) & 1),
+                                                       p.timeout_ns))) {
+            state = 2;
+          } else {
+            const unsigned char *sb = smem + rp * Cfg::SLOT;
+            widen_tile<TT * NS>(reinterpret_cast<const __nv_bfloat16 *>(sb + Cfg::OFF_B),
+                                reinterpret_cast<float *>(smem + rp * Cfg::SLOT + Cfg::OFF_BF),
+                                lane);
+            if constexpr (!CARRY)
+              widen_tile<TT * NS>(reinterpret_cast<const __nv_bfloat16 *>(sb + Cfg::OFF_C),
+                                  reinterpret_cast<float *>(smem + rp * Cfg::SLOT + Cfg::OFF_CF),
+                                  lane);
+            mbar_arrive(&rconv[rp]);
+          }
         }
-        slot_work[r] = make_int2(iss.item, st);
-        const int d0 = iss.dtile * DT, t0 = st * TT, b = iss.b;
-        unsigned char *sb = smem + r * Cfg::SLOT;
-        mbar_arrive_expect_tx(&rfull[r], tx_bytes);
-        tma_load_3d(sb, &maps.x, &rfull[r], d0, t0 - Cfg::XHALO, b);
-        tma_load_3d(sb + Cfg::OFF_DT, &maps.dt, &rfull[r], d0, t0, b);
-        if (with_z) tma_load_3d(sb + Cfg::OFF_Z, &maps.z, &rfull[r], d0, t0, b);
-        tma_load_3d(sb + Cfg::OFF_B, &maps.B, &rfull[r], 0, t0, b);
-        if (!CARRY) tma_load_3d(sb + Cfg::OFF_C, &maps.C, &rfull[r], 0, t0, b);
-        ++st;
+        if (state == 1) mbar_arrive(&rconv[r]);  // the end marker
+      } else {
+        state = __shfl_sync(FULL_MASK, state, 0);
       }
-      if (!ok) {
-        atomicCAS(&p.ctl->status, 0, kStatusTimeout);
-        // let the loads still in flight land before the CTA exits (bounded)
-        for (int kk = (k > RAW ? k - RAW : 0); kk < k; ++kk)
-          (void)mbar_wait_bounded(&rfull[kk % RAW], (uint32_t)((kk / RAW) & 1), p.timeout_ns);
-      }
+      if (state != 0) break;
+    }
+    if (lane == 0 && state == 2) {
+      atomicCAS(&p.ctl->status, 0, kStatusTimeout);
+      // let the loads still in flight land before the CTA exits (bounded)
+      for (int kk = (issued > RAW ? issued - RAW : 0); kk < issued; ++kk)
+        (void)mbar_wait_bounded(&rfull[kk % RAW], (uint32_t)((kk / RAW) & 1), p.timeout_ns);
     }
   } else {
     // =================== scan warps ===================
@@ -329,13 +388,20 @@ __global__ void __launch_bounds__((WARPS + 1) * 32, (OPT & 2) ? 5 : 0)
     ItemPos cur;
     for (int k = 0;; ++k) {
       const int r = k % RAW;
-      if (!__all_sync(FULL_MASK, mbar_wait_bounded(&rfull[r], (uint32_t)((k / RAW) & 1),
-                                                   p.timeout_ns))) {
+      if (!__all_sync(FULL_MASK, mbar_wait_bounded(BCF ? &rconv[r] : &rfull[r],
+                                                   (uint32_t)((k / RAW) & 1), p.timeout_ns))) {
         if (lane == 0) atomicCAS(&p.ctl->status, 0, kStatusTimeout);
         break;
       }
       const int2 work = slot_work[r];
       if (work.x < 0) break;  // end marker
+      // (BCF: the load warp saw the tiles land before widening; waiting on
+      // the slot's own barrier too makes the bulk copy's data visible here)
+      if (BCF && !__all_sync(FULL_MASK, mbar_wait_bounded(&rfull[r], (uint32_t)((k / RAW) & 1),
+                                                          p.timeout_ns))) {
+        if (lane == 0) atomicCAS(&p.ctl->status, 0, kStatusTimeout);
+        break;
+      }
       if (work.x != cur.item) cur.set(work.x, p);
       const int st = work.y, b = cur.b;
       const int d = cur.dtile * DT + ch0;  // first channel (of KC) in the tensor
@@ -411,8 +477,9 @@ __global__ void __launch_bounds__((WARPS + 1) * 32, (OPT & 2) ? 5 : 0)
       const InT *xs = reinterpret_cast<const InT *>(sb);
       const InT *ds = reinterpret_cast<const InT *>(sb + Cfg::OFF_DT);
       const InT *zs = reinterpret_cast<const InT *>(sb + Cfg::OFF_Z);
-      const InT *Bs = reinterpret_cast<const InT *>(sb + Cfg::OFF_B);
-      const InT *Cs = reinterpret_cast<const InT *>(sb + Cfg::OFF_C);
+      using BCT = typename std::conditional<BCF, float, InT>::type;  // B, C as the lanes read them
+      const BCT *Bs = reinterpret_cast<const BCT *>(sb + (BCF ? Cfg::OFF_BF : Cfg::OFF_B));
+      const BCT *Cs = reinterpret_cast<const BCT *>(sb + (BCF ? Cfg::OFF_CF : Cfg::OFF_C));
       const int t0 = st * TT;
       OutT *xcrow = CONV && p.xconv
                         ? reinterpret_cast<OutT *>(p.xconv) + ((size_t)b * p.L + t0) * p.D + d
@@ -733,7 +800,8 @@ template <typename InT, typename OutT, int NS, int LPC, int KC, int WARPS, int T
           bool CARRY, bool CONV, int OPT>
 static cudaError_t run_variant(const LaunchShape *ls, const TmaMaps *maps, const FwdParams *p,
                                cudaStream_t stream, VariantInfo *vi) {
-  using Cfg = FwdCfg<InT, OutT, NS, LPC, KC, WARPS, TT, CONV, CARRY>;
+  constexpr bool BCF = (OPT & 4) != 0 && std::is_same<InT, __nv_bfloat16>::value;
+  using Cfg = FwdCfg<InT, OutT, NS, LPC, KC, WARPS, TT, CONV, CARRY, BCF>;
   auto kern = fwd_kernel<InT, OutT, NS, LPC, KC, WARPS, TT, ZOH, CARRY, CONV, OPT>;
   if (Cfg::SMEM + 8 * Cfg::RAW > 227 * 1024) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);

@@ -102,6 +102,52 @@ def test_f32_every_variant_and_segments(ns, zoh):
     _sweep(inp, "f32", "f32", (1, 4))
 
 
+@pytest.mark.parametrize("in_dt,out_dt,zoh", [("bf16", "bf16", False), ("bf16", "bf16", True),
+                                               ("bf16", "f32", False), ("f32", "f32", False)])
+def test_every_carry_variant(in_dt, out_dt, zoh):
+    """Each compiled carry-pass variant (lanes per channel and options forced),
+    behind a main variant of the same stage length (and lane split where one
+    exists), with 4 segments on a ragged length: the maps it leaves, folded
+    at each segment's start, give the oracle's result."""
+    for ns in (16, 8):
+        carries = _variants(in_dt, out_dt, ns, zoh, carry=True)
+        if not carries:
+            continue
+        inp = synth.make_fwd(2, 1800, 64, ns, in_dtype=in_dt, out_dtype=out_dt, seed=69,
+                             has_h0=True, zoh=zoh)
+        tol = gu.TOL["f32" if in_dt == "f32" and out_dt == "f32" else "bf16"]
+        dev = gu.upload(inp)
+        ry, rh = gu.run_oracle(inp)
+        mains = _variants(in_dt, out_dt, ns, zoh)
+        failures = []
+        for c in carries:
+            same = [v for v in mains if (v["lanes_per_chan"], v["chans_per_lane"], v["tile_t"]) ==
+                    (c["lanes_per_chan"], c["chans_per_lane"], c["tile_t"])]
+            cands = same or [v for v in mains if v["tile_t"] == c["tile_t"]]
+            if not cands:
+                failures.append(f"carry {c}: no main variant with its stage length")
+                continue
+            v = cands[0]
+            cfg = dict(lanes_per_chan=v["lanes_per_chan"], warps_per_cta=v["warps_per_cta"],
+                       tile_t=v["tile_t"], chans_per_lane=v["chans_per_lane"], segments=4,
+                       scan_loop=1 + v["opt"], carry_lanes_per_chan=c["lanes_per_chan"],
+                       carry_loop=1 + c["opt"])
+            try:
+                info, gy, gh, st = _run(inp, dev, cfg)
+            except bnd.SsmError as e:
+                failures.append(f"{cfg}: refused ({e})")
+                continue
+            if (info["carry_lanes_per_chan"], info["carry_loop"]) != \
+                    (c["lanes_per_chan"], 1 + c["opt"]) or info["segments"] != 4:
+                failures.append(f"{cfg}: plan chose {info}")
+            try:
+                assert st == 0, f"device status {st}"
+                gu.assert_parity(gy, ry, gh, rh, tol, f"carry {c} main {v}")
+            except AssertionError as e:
+                failures.append(str(e))
+        assert not failures, "\n".join(failures)
+
+
 @pytest.mark.parametrize("M", [2, 4, 8])
 @pytest.mark.parametrize("h0", [False, True])
 def test_segments_ragged_lengths(M, h0):
