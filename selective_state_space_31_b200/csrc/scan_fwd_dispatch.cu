@@ -116,9 +116,13 @@ double warps_weight(int warps) { return warps == 2 ? 0.8 : 1.0; }
 // The software-pipelined loop (bit 0) and the five-CTA register cap (bit 1)
 // relative to the plain variant, measured on B200: with 8 lanes per channel
 // and 64-token stages the pipelined loop gains 3-5 % on the layer shapes;
-// elsewhere, and with segments, the plain loop was as fast or faster.
+// elsewhere, and with segments, the plain loop was as fast or faster.  B and
+// C widened by the load warp (bit 2) took 2-10 % longer on every workload
+// (wider slots cost a CTA per SM at 64-token stages; at equal occupancy the
+// removed widening did not shorten the latency-bound loop).
 double opt_weight(int opt, int lpc, int tt, int segments) {
   if (opt == 0) return 1.0;
+  if (opt & 4) return 0.9;
   if (segments > 1 || lpc != 8 || tt != 64) return 0.97;
   return opt == 1 ? 1.05 : opt == 2 ? 1.04 : 1.03;
 }

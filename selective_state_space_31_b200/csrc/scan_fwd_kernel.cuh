@@ -109,103 +109,6 @@ struct FwdCfg {
   static_assert(SLOT % 128 == 0 && OFF_PLANE % 128 == 0, "slot alignment");
 };
 
-// Butterfly reduce-scatter over the LPC lanes of a channel group: on entry
-// lane q holds partial sums v[j] (its NPL states) of the group's LPC tokens;
-// on exit it returns the full sum (all N states) of token q.
-template <int LPC>
-__device__ __forceinline__ float reduce_scatter(float (&v)[LPC], int q) {
-#pragma unroll
-  for (int m = LPC / 2; m >= 1; m >>= 1) {
-    const bool upper = (q & m) != 0;
-#pragma unroll
-    for (int i = 0; i < m; ++i) {
-      const float send = upper ? v[i] : v[i + m];
-      const float keep = upper ? v[i + m] : v[i];
-      v[i] = keep + __shfl_xor_sync(FULL_MASK, send, m);
-    }
-  }
-  return v[0];
-}
-// The same for a lane's two channels at once (.x and .y).
-template <int LPC>
-__device__ __forceinline__ float2 reduce_scatter2(float2 (&v)[LPC], int q) {
-#pragma unroll
-  for (int m = LPC / 2; m >= 1; m >>= 1) {
-    const bool upper = (q & m) != 0;
-#pragma unroll
-    for (int i = 0; i < m; ++i) {
-      const float2 send = upper ? v[i] : v[i + m];
-      const float2 keep = upper ? v[i + m] : v[i];
-      const float2 got = make_float2(__shfl_xor_sync(FULL_MASK, send.x, m),
-                                     __shfl_xor_sync(FULL_MASK, send.y, m));
-      v[i] = fadd2(keep, got);
-    }
-  }
-  return v[0];
-}
-
-// A bf16 is the upper half of the fp32 of equal value.
-__device__ __forceinline__ void widen_bf16x2(uint32_t w, float &lo, float &hi) {
-  lo = __uint_as_float(w << 16);
-  hi = __uint_as_float(w & 0xffff0000u);
-}
-
-// NPL consecutive B or C values of one token as fp32.
-template <int NPL>
-__device__ __forceinline__ void load_bc(const float *src, float (&dst)[NPL]) {
-  if constexpr (NPL % 4 == 0) {
-#pragma unroll
-    for (int i = 0; i < NPL; i += 4) {
-      const float4 v = *reinterpret_cast<const float4 *>(src + i);
-      dst[i] = v.x; dst[i + 1] = v.y; dst[i + 2] = v.z; dst[i + 3] = v.w;
-    }
-  } else if constexpr (NPL == 2) {
-    const float2 v = *reinterpret_cast<const float2 *>(src);
-    dst[0] = v.x; dst[1] = v.y;
-  } else {
-#pragma unroll
-    for (int i = 0; i < NPL; ++i) dst[i] = src[i];
-  }
-}
-template <int NPL>
-__device__ __forceinline__ void load_bc(const __nv_bfloat16 *src, float (&dst)[NPL]) {
-  if constexpr (NPL % 8 == 0) {
-#pragma unroll
-    for (int i = 0; i < NPL; i += 8) {
-      const uint4 w = *reinterpret_cast<const uint4 *>(src + i);
-      widen_bf16x2(w.x, dst[i], dst[i + 1]);
-      widen_bf16x2(w.y, dst[i + 2], dst[i + 3]);
-      widen_bf16x2(w.z, dst[i + 4], dst[i + 5]);
-      widen_bf16x2(w.w, dst[i + 6], dst[i + 7]);
-    }
-  } else if constexpr (NPL == 4) {
-    const uint2 w = *reinterpret_cast<const uint2 *>(src);
-    widen_bf16x2(w.x, dst[0], dst[1]);
-    widen_bf16x2(w.y, dst[2], dst[3]);
-  } else if constexpr (NPL == 2) {
-    widen_bf16x2(*reinterpret_cast<const uint32_t *>(src), dst[0], dst[1]);
-  } else {
-    dst[0] = __bfloat162float(src[0]);
-  }
-}
-
-// Widen a tile of `N` bf16 values (N a multiple of 128) to fp32 with the 32
-// lanes of a warp: per round lane i turns the 4 values at 8-byte word i into
-// one 16-byte store, so both the reads and the writes of a round are
-// consecutive in the banks.
-template <int N>
-__device__ __forceinline__ void widen_tile(const __nv_bfloat16 *src, float *dst, int lane) {
-  static_assert(N % 128 == 0, "whole rounds of 32 lanes x 4 values");
-#pragma unroll
-  for (int i = 0; i < N / 128; ++i) {
-    const uint2 w = reinterpret_cast<const uint2 *>(src)[i * 32 + lane];
-    float4 f;
-    widen_bf16x2(w.x, f.x, f.y);
-    widen_bf16x2(w.y, f.z, f.w);
-    reinterpret_cast<float4 *>(dst)[i * 32 + lane] = f;
-  }
-}
-
 // Two adjacent channels' values of one token (x, delta or z) as fp32.
 __device__ __forceinline__ float2 load_pair(const float *src) {
   return *reinterpret_cast<const float2 *>(src);

@@ -13,10 +13,7 @@
   X(16, 4, 1, 4, 64, false, false, false, 1) X(16, 8, 1, 4, 32, false, false, false, 1)  \
   X(16, 4, 1, 4, 32, false, false, false, 2) X(16, 8, 1, 4, 64, false, false, false, 2)  \
   X(16, 4, 1, 4, 32, false, false, false, 3) X(16, 8, 1, 4, 64, false, false, false, 3)  \
-  X(16, 8, 1, 4, 64, false, false, false, 5) X(16, 8, 1, 4, 32, false, false, false, 5)  \
-  X(16, 4, 1, 4, 32, false, false, false, 5) X(16, 4, 1, 4, 32, false, false, false, 4)  \
-  X(16, 2, 1, 4, 32, false, false, false, 4) X(16, 4, 1, 8, 32, false, false, false, 5)  \
-  X(16, 8, 1, 8, 32, false, false, false, 5) X(16, 8, 2, 4, 32, false, false, false, 4)  \
+  X(16, 8, 1, 4, 64, false, false, false, 5) X(16, 4, 1, 4, 32, false, false, false, 4)  \
   X(16, 1, 1, 4, 32, false, false, false, 0) X(16, 2, 1, 4, 32, false, false, false, 0)                      \
   X(16, 4, 1, 4, 32, false, false, false, 0) X(16, 4, 1, 4, 64, false, false, false, 0)                      \
   X(16, 8, 1, 4, 32, false, false, false, 0) X(16, 8, 1, 4, 64, false, false, false, 0)                      \
@@ -28,8 +25,7 @@
   X(16, 8, 2, 4, 32, false, false, false, 0) X(16, 8, 2, 4, 64, false, false, false, 0)                      \
   X(16, 4, 2, 8, 32, false, false, false, 0) X(16, 8, 2, 8, 32, false, false, false, 0)
 #define SSM_FWD_BF16_N16_ZOH_CARRY(X)                                                    \
-  X(16, 8, 1, 4, 64, false, true, false, 4) X(16, 4, 1, 4, 32, false, true, false, 4)    \
-  X(16, 8, 1, 4, 32, false, true, false, 4)                                              \
+  X(16, 4, 1, 4, 32, false, true, false, 4)                                              \
   X(16, 4, 1, 4, 32, true, false, false, 0) X(16, 4, 1, 4, 64, true, false, false, 0)                        \
   X(16, 8, 1, 4, 32, true, false, false, 0) X(16, 8, 1, 4, 64, true, false, false, 0)                        \
   X(16, 16, 1, 4, 32, true, false, false, 0) X(16, 16, 1, 4, 64, true, false, false, 0)                      \

@@ -309,6 +309,7 @@ ssm_status ssm_scan_destroy(ssm_scan_plan *pl) {
 ssm_status ssm_scan_get_info(const ssm_scan_plan *pl, ssm_scan_info *info) {
   if (!pl || !info) return SSM_ERR_INVALID_ARG;
   std::memset(info, 0, sizeof(*info));
+  const ssm_scan_desc &d = pl->desc;
   info->path = pl->path;
   if (pl->path == PATH_TMA) {
     info->lanes_per_chan = pl->ls.lpc;
@@ -332,6 +333,13 @@ ssm_status ssm_scan_get_info(const ssm_scan_plan *pl, ssm_scan_info *info) {
     info->carry_loop = pl->fs.M > 1 ? 1 + pl->fs.cls.opt : 0;
   }
   info->launches_per_call = pl->path == PATH_TMA && pl->fs.M > 1 ? 2 : 1;
+  ssm::BwdShape bs;
+  info->bwd_warps_per_cta =
+      pl->path == PATH_TMA &&
+              ssm::choose_bwd_shape((int)d.in_dtype, (int)d.out_dtype, d.batch, d.seqlen, d.dim,
+                                    (int)d.dstate, pl->cfg.bwd_warps_per_cta, pl->num_sms, &bs)
+          ? bs.warps
+          : 0;
   info->workspace_bytes =
       pl->ws_state_bytes + pl->ws_flag_bytes + pl->ws_agg_bytes + sizeof(ssm::Control);
   return SSM_OK;
@@ -341,7 +349,8 @@ ssm_status ssm_scan_set_config(ssm_scan_plan *pl, const ssm_scan_config *cfg) {
   if (!pl || !cfg) return SSM_ERR_INVALID_ARG;
   if (cfg->lanes_per_chan < 0 || cfg->warps_per_cta < 0 || cfg->grid < 0 || cfg->tile_t < 0 ||
       cfg->chans_per_lane < 0 || cfg->segments < 0 || cfg->scan_loop < 0 || cfg->scan_loop > 8 ||
-      cfg->carry_lanes_per_chan < 0 || cfg->carry_loop < 0 || cfg->carry_loop > 8)
+      cfg->carry_lanes_per_chan < 0 || cfg->carry_loop < 0 || cfg->carry_loop > 8 ||
+      (cfg->bwd_warps_per_cta != 0 && cfg->bwd_warps_per_cta != 2 && cfg->bwd_warps_per_cta != 4))
     return SSM_ERR_INVALID_ARG;
   DeviceGuard guard(pl->device);
   if (!guard.ok) return SSM_ERR_CUDA;
@@ -654,6 +663,54 @@ ssm_status ssm_scan_bwd(ssm_scan_plan *pl, const void *x, const void *delta,
   if (d.dim == 0) return SSM_OK;
   DeviceGuard guard(pl->device);
   if (!guard.ok) return SSM_ERR_CUDA;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  ssm::BwdShape bs;
+  const bool fused = has_tokens && pl->path == PATH_TMA &&
+                     ssm::choose_bwd_shape((int)d.in_dtype, (int)d.out_dtype, d.batch, d.seqlen,
+                                           d.dim, (int)d.dstate, pl->cfg.bwd_warps_per_cta,
+                                           pl->num_sms, &bs) &&
+                     aligned16(x) && aligned16(delta) && aligned16(z) && aligned16(B) &&
+                     aligned16(C) && aligned16(dy) && aligned16(dB) && aligned16(dC) &&
+                     aligned16(dh0);
+  if (fused) {
+    const size_t need = (bs.ws_ck_floats + bs.ws_bc_floats) * sizeof(float);
+    if (need > pl->ws_ck_bytes) {
+      if (pl->ws_ck) cudaFree(pl->ws_ck);
+      pl->ws_ck = nullptr;
+      pl->ws_ck_bytes = 0;
+      if (cudaMalloc(&pl->ws_ck, need) != cudaSuccess) {
+        cudaGetLastError();
+        return SSM_ERR_OOM;
+      }
+      pl->ws_ck_bytes = need;
+    }
+    ssm::BwdMaps maps;
+    const uint64_t Bn = d.batch, L = d.seqlen, Dm = d.dim, N = d.dstate;
+    const uint32_t DT = (uint32_t)bs.DT, TT = (uint32_t)ssm::kBwdStage;
+    if (!encode3d(&maps.x, d.in_dtype, x, Dm, L, Bn, DT, TT) ||
+        !encode3d(&maps.dt, d.in_dtype, delta, Dm, L, Bn, DT, TT) ||
+        !encode3d(&maps.z, d.in_dtype, z ? z : x, Dm, L, Bn, DT, TT) ||
+        !encode3d(&maps.dy, d.out_dtype, dy, Dm, L, Bn, DT, TT) ||
+        !encode3d(&maps.B, d.in_dtype, B, N, L, Bn, (uint32_t)N, TT) ||
+        !encode3d(&maps.C, d.in_dtype, C, N, L, Bn, (uint32_t)N, TT))
+      return SSM_ERR_CUDA;
+    ssm::BwdTmaParams p{};
+    p.Bsz = (int)d.batch; p.L = (int)d.seqlen; p.D = (int)d.dim; p.N = (int)d.dstate;
+    p.DT = bs.DT; p.nDT = bs.nDT; p.S = bs.S; p.rows = (int)bs.rows;
+    p.softplus = f & SSM_DELTA_SOFTPLUS;
+    p.has_z = f & SSM_HAS_Z;
+    p.has_D = f & SSM_HAS_D;
+    p.has_bias = f & SSM_HAS_DELTA_BIAS;
+    p.has_h0 = f & SSM_HAS_H0;
+    p.A = A; p.Dv = D; p.bias = delta_bias; p.h0 = h0; p.dh_last = dh_last;
+    p.dx = dx; p.ddelta = ddelta; p.dz = dz; p.dB = dB; p.dC = dC; p.dA = dA; p.dD = dD;
+    p.dbias = ddelta_bias; p.dh0 = dh0;
+    p.ws_ck = pl->ws_ck;
+    p.ws_bc = pl->ws_ck + bs.ws_ck_floats;
+    p.ctl = pl->ctl;
+    p.timeout_ns = pl->timeout_ns;
+    return map_cuda(ssm::launch_bwd_tma((int)d.in_dtype, (int)d.out_dtype, bs, maps, p, stream));
+  }
   const int64_t nck = (d.seqlen + ssm::kBwdChunk - 1) / ssm::kBwdChunk;
   const size_t need = (size_t)(d.batch * d.dim * nck * d.dstate) * sizeof(float);
   if (need > pl->ws_ck_bytes) {
@@ -679,7 +736,7 @@ ssm_status ssm_scan_bwd(ssm_scan_plan *pl, const void *x, const void *delta,
   p.A = A; p.Dv = D; p.bias = delta_bias; p.h0 = h0; p.dh_last = dh_last;
   p.dx = dx; p.ddelta = ddelta; p.dz = dz; p.dB = dB; p.dC = dC; p.dA = dA; p.dD = dD;
   p.dbias = ddelta_bias; p.dh0 = dh0; p.ws_ck = pl->ws_ck;
-  return map_cuda(ssm::launch_bwd(p, reinterpret_cast<cudaStream_t>(stream_)));
+  return map_cuda(ssm::launch_bwd(p, stream));
 }
 
 ssm_status ssm_scan_step(ssm_scan_plan *pl, const void *x, const void *delta,

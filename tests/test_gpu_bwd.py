@@ -26,13 +26,15 @@ def _round_bf16(a):
     return torch.from_numpy(np.asarray(a, np.float32)).to(torch.bfloat16).float().numpy()
 
 
-def _check(inp, dh_last=True, want_dh0=True, seed=0):
+def _check(inp, dh_last=True, want_dh0=True, seed=0, cfg=None):
     rng = np.random.default_rng(seed)
     dy = rng.standard_normal((inp.Bsz, inp.L, inp.D)).astype(np.float32)
     if inp.out_dtype == "bf16":
         dy = _round_bf16(dy)
     dhl = rng.standard_normal((inp.Bsz, inp.D, inp.N)).astype(np.float32) if dh_last else None
     plan = gu.make_plan(inp)
+    if cfg:
+        plan.set_config(**cfg)
     dev = gu.upload(inp)
     g = plan.bwd(dev["x"], dev["delta"], dev["A"], dev["B"], dev["C"],
                  gu.dev_tensor(dy, inp.out_dtype), D=dev["D"], z=dev["z"],
@@ -118,3 +120,65 @@ def test_bwd_130m_layer_sampled():
     assert gu.normwise(g["delta"].cpu().numpy()[:, :, chans], ref["delta"]) <= 2e-2
     assert gu.normwise(g["A"].cpu().numpy()[chans], ref["A"]) <= 2e-2
     assert gu.normwise(g["D"].cpu().numpy()[chans], ref["D"]) <= 2e-2
+
+
+# ---------------------------------------------------------------------------
+# the fused backward kernel (TMA-fed row tiles; two or four scan warps)
+# ---------------------------------------------------------------------------
+
+def _check_fused(inp, warps, dh_last=True, want_dh0=True, seed=0):
+    """_check with the fused kernel's scan warps forced, after checking that
+    the plan takes the fused kernel with that shape."""
+    plan = gu.make_plan(inp)
+    plan.set_config(bwd_warps_per_cta=warps)
+    assert plan.info()["bwd_warps_per_cta"] == warps
+    plan.close()
+    _check(inp, dh_last=dh_last, want_dh0=want_dh0, seed=seed,
+           cfg=dict(bwd_warps_per_cta=warps))
+
+
+@pytest.mark.parametrize("warps", [2, 4])
+@pytest.mark.parametrize("ns", [16, 8])
+def test_bwd_fused_fp32_ragged(warps, ns):
+    """fp32, every option, L = 77 (the last 16-token stage holds 13 tokens)
+    and D = 72 (the last row tile is partly past the channels)."""
+    _check_fused(synth.make_fwd(2, 77, 72, ns, in_dtype="f32", seed=59 + ns, has_h0=True),
+                 warps, seed=8)
+
+
+@pytest.mark.parametrize("warps", [2, 4])
+def test_bwd_fused_bf16_in_bf16_and_f32_dy(warps):
+    _check_fused(synth.make_fwd(3, 150, 64, 16, seed=61, has_h0=True), warps, seed=9)
+    _check_fused(synth.make_fwd(2, 96, 48, 16, out_dtype="f32", seed=62, has_h0=True), warps,
+                 seed=10)
+
+
+def test_bwd_fused_no_gate_no_softplus():
+    inp = synth.make_fwd(2, 45, 32, 16, in_dtype="f32", seed=63, has_z=False, has_D=False,
+                         has_bias=False, delta_softplus=False)
+    inp.delta = np.abs(inp.delta) * np.float32(0.3) + np.float32(0.05)
+    _check_fused(inp, 2, dh_last=False, want_dh0=False, seed=11)
+
+
+def test_bwd_fused_single_token_and_one_stage():
+    _check_fused(synth.make_fwd(1, 1, 32, 16, in_dtype="f32", seed=64, has_h0=True), 2, seed=12)
+    _check_fused(synth.make_fwd(2, 16, 32, 16, in_dtype="f32", seed=65, has_h0=True), 4, seed=13)
+
+
+def test_bwd_fused_deterministic():
+    """Every gradient but the batch sums (dA, dD, delta bias: atomics over
+    the batch) is bitwise reproducible: dB and dC add the row tiles' sums
+    in a fixed order."""
+    inp = synth.make_fwd(2, 300, 128, 16, seed=66, has_h0=True)
+    rng = np.random.default_rng(14)
+    dy = gu.dev_tensor(_round_bf16(rng.standard_normal((2, 300, 128)).astype(np.float32)), "bf16")
+    plan = gu.make_plan(inp)
+    assert plan.info()["bwd_warps_per_cta"] in (2, 4)
+    dev = gu.upload(inp)
+    run = lambda: plan.bwd(dev["x"], dev["delta"], dev["A"], dev["B"], dev["C"], dy, D=dev["D"],
+                           z=dev["z"], delta_bias=dev["delta_bias"], h0=dev["h0"])
+    g1, g2 = run(), run()
+    torch.cuda.synchronize()
+    for name in ("x", "delta", "B", "C", "z", "h0"):
+        assert torch.equal(g1[name], g2[name]), name
+    assert plan.status() == 0
