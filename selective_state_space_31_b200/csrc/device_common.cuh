@@ -230,20 +230,24 @@ __device__ __forceinline__ void load_bc(const __nv_bfloat16 *src, float (&dst)[N
   }
 }
 
-// Widen a tile of `N` bf16 values (N a multiple of 128) to fp32 with the 32
+// Widen a tile of `N` bf16 values (N a multiple of 4) to fp32 with the 32
 // lanes of a warp: per round lane i turns the 4 values at 8-byte word i into
 // one 16-byte store, so both the reads and the writes of a round are
 // consecutive in the banks.
 template <int N>
 __device__ __forceinline__ void widen_tile(const __nv_bfloat16 *src, float *dst, int lane) {
-  static_assert(N % 128 == 0, "whole rounds of 32 lanes x 4 values");
+  static_assert(N % 4 == 0, "whole 8-byte words");
+  constexpr int WORDS = N / 4;
 #pragma unroll
-  for (int i = 0; i < N / 128; ++i) {
-    const uint2 w = reinterpret_cast<const uint2 *>(src)[i * 32 + lane];
-    float4 f;
-    widen_bf16x2(w.x, f.x, f.y);
-    widen_bf16x2(w.y, f.z, f.w);
-    reinterpret_cast<float4 *>(dst)[i * 32 + lane] = f;
+  for (int i = 0; i < (WORDS + 31) / 32; ++i) {
+    const int w = i * 32 + lane;
+    if (WORDS % 32 == 0 || w < WORDS) {
+      const uint2 u = reinterpret_cast<const uint2 *>(src)[w];
+      float4 f;
+      widen_bf16x2(u.x, f.x, f.y);
+      widen_bf16x2(u.y, f.z, f.w);
+      reinterpret_cast<float4 *>(dst)[w] = f;
+    }
   }
 }
 

@@ -22,7 +22,7 @@ cudaError_t launch_bwd(const BwdParams &p, cudaStream_t stream);
 
 // Fused backward kernel (scan_bwd_tma.cu): TMA-fed tiles of DT channels x
 // kBwdStage tokens, a load warp and W scan warps of 32 / LPC channels each.
-constexpr int kBwdStage = 16;
+constexpr int kBwdStage = 8;
 struct BwdMaps {
   CUtensorMap x, dt, z, dy, B, C;  // boxes (DT, kBwdStage) and (N, kBwdStage)
 };
@@ -32,6 +32,7 @@ struct BwdShape {
   int64_t rows = 0;        // B * nDT: one CTA each
   int S = 0;               // stages of kBwdStage tokens
   size_t smem = 0;
+  int occ = 0;              // resident CTAs per SM
   size_t ws_ck_floats = 0;  // (rows, S, DT, N): the state at the start of each stage
   size_t ws_bc_floats = 0;  // (B, nDT, L, 2N): each row tile's sums of dC and dB
 };

@@ -58,7 +58,10 @@ struct BwdCfg {
   static constexpr int TTP = TT + 1;
   static constexpr int PLANE = rup(GPW * TTP * 16, 128);
   // per warp: the lanes' dC / dB shares of LPC tokens, (token, block of 4
-  // values, group) with a padded block row
+  // values, group) with a padded block row; a lane stores its group at
+  // position (group + block) mod GPW of the row, so that the lanes' stores
+  // as well as the per-block sums (which read whole rows) spread over the
+  // banks
   static constexpr int VB = 2 * NS / 4;
   static constexpr int BSTR = GPW * 4 + 4;
   static constexpr int XPOSE = rup(LPC * VB * BSTR * 4, 128);
@@ -102,7 +105,7 @@ __device__ __forceinline__ float sigmoid_f(float v) {
 }
 
 template <typename InT, typename GT, int NS, int LPC, int W>
-__global__ void __launch_bounds__((W + 1) * 32)
+__global__ void __launch_bounds__((W + 1) * 32, W == 4 ? 3 : 5)
     bwd_tma_kernel(const __grid_constant__ BwdMaps maps, const BwdTmaParams p) {
   using Cfg = BwdCfg<InT, GT, NS, LPC, W>;
   constexpr int TT = Cfg::TT, NPL = Cfg::NPL, GPW = Cfg::GPW, DT = Cfg::DT, RAW = Cfg::RAW,
@@ -204,6 +207,11 @@ __global__ void __launch_bounds__((W + 1) * 32)
   float4 *plane = reinterpret_cast<float4 *>(smem + Cfg::OFF_PLANE + warp * Cfg::PLANE) +
                   g_loc * TTP;
   float *xp = reinterpret_cast<float *>(smem + Cfg::OFF_XP + warp * Cfg::XPOSE);
+  // this lane's dC block q and dB block LPC + q of the first token, at its
+  // rotated position (a rotation only permutes the groups within a row, and
+  // the per-block sum reads the whole row)
+  float *xp_c = xp + q * BSTR + ((g_loc + q) % GPW) * 4;
+  float *xp_b = xp + (LPC + q) * BSTR + ((g_loc + LPC + q) % GPW) * 4;
   using BCT = typename std::conditional<WIDEN, float, InT>::type;
   bool ok = true;
   int k = 0;
@@ -389,9 +397,9 @@ __global__ void __launch_bounds__((W + 1) * 32)
               dCv[i] = dc.x; dCv[i + 1] = dc.y;
               dBv[i] = db.x; dBv[i + 1] = db.y;
             }
-            *reinterpret_cast<float4 *>(xp + (jj * VB + q) * BSTR + g_loc * 4) =
+            *reinterpret_cast<float4 *>(xp_c + jj * VB * BSTR) =
                 make_float4(dCv[0], dCv[1], dCv[2], dCv[3]);
-            *reinterpret_cast<float4 *>(xp + (jj * VB + LPC + q) * BSTR + g_loc * 4) =
+            *reinterpret_cast<float4 *>(xp_b + jj * VB * BSTR) =
                 make_float4(dBv[0], dBv[1], dBv[2], dBv[3]);
             yc[jj] = sc.x + sc.y;
             yg[jj] = sg.x + sg.y;
@@ -418,12 +426,15 @@ __global__ void __launch_bounds__((W + 1) * 32)
             const int jl = lane / VB, vb = lane - jl * VB;
             const float *src = xp + (jl * VB + vb) * BSTR;
             float4 s = *reinterpret_cast<const float4 *>(src);
+            float2 lo = make_float2(s.x, s.y), hi = make_float2(s.z, s.w);
 #pragma unroll
             for (int gg = 1; gg < GPW; ++gg) {
               const float4 u = *reinterpret_cast<const float4 *>(src + gg * 4);
-              s.x += u.x; s.y += u.y; s.z += u.z; s.w += u.w;
+              lo = fadd2(lo, make_float2(u.x, u.y));
+              hi = fadd2(hi, make_float2(u.z, u.w));
             }
-            *reinterpret_cast<float4 *>(slice + (tt + jl) * 2 * NS + vb * 4) = s;
+            *reinterpret_cast<float4 *>(slice + (tt + jl) * 2 * NS + vb * 4) =
+                make_float4(lo.x, lo.y, hi.x, hi.y);
           }
           __syncwarp();
         }
@@ -437,13 +448,15 @@ __global__ void __launch_bounds__((W + 1) * 32)
         for (int i = warp * 32 + lane; i < TT * VB; i += W * 32) {
           const int t = i / VB;
           if (t >= nvalid) continue;
-          float4 s = *reinterpret_cast<const float4 *>(sl + i * 4);
+          const float4 s = *reinterpret_cast<const float4 *>(sl + i * 4);
+          float2 lo = make_float2(s.x, s.y), hi = make_float2(s.z, s.w);
 #pragma unroll
           for (int w = 1; w < W; ++w) {
             const float4 u = *reinterpret_cast<const float4 *>(sl + w * TT * 2 * NS + i * 4);
-            s.x += u.x; s.y += u.y; s.z += u.z; s.w += u.w;
+            lo = fadd2(lo, make_float2(u.x, u.y));
+            hi = fadd2(hi, make_float2(u.z, u.w));
           }
-          *reinterpret_cast<float4 *>(dst + (size_t)i * 4) = s;
+          *reinterpret_cast<float4 *>(dst + (size_t)i * 4) = make_float4(lo.x, lo.y, hi.x, hi.y);
         }
       }
     }
@@ -493,15 +506,16 @@ __global__ void __launch_bounds__(256) bwd_bc_sum_kernel(const BwdTmaParams p) {
 
 template <typename InT, typename GT, int NS, int LPC, int W>
 cudaError_t run_bwd(const BwdShape &s, const BwdMaps &maps, const BwdTmaParams &p,
-                    cudaStream_t stream, size_t *smem_out) {
+                    cudaStream_t stream, BwdShape *query) {
   using Cfg = BwdCfg<InT, GT, NS, LPC, W>;
   auto kern = bwd_tma_kernel<InT, GT, NS, LPC, W>;
-  if (smem_out) {
-    *smem_out = Cfg::SMEM;
-    return cudaSuccess;
-  }
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
   if (e != cudaSuccess) return e;
+  if (query) {  // what the variant needs and gets on the device
+    query->smem = Cfg::SMEM;
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(&query->occ, kern, Cfg::THREADS,
+                                                         Cfg::SMEM);
+  }
   kern<<<(unsigned)s.rows, Cfg::THREADS, Cfg::SMEM, stream>>>(maps, p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const long long total = (long long)p.Bsz * p.L * (2 * NS / 4);
@@ -514,34 +528,36 @@ cudaError_t run_bwd(const BwdShape &s, const BwdMaps &maps, const BwdTmaParams &
 // states per lane either way), 2 or 4 scan warps.
 template <typename InT, typename GT>
 cudaError_t bwd_by_shape(const BwdShape &s, const BwdMaps *maps, const BwdTmaParams *p,
-                         cudaStream_t stream, size_t *smem_out) {
+                         cudaStream_t stream, BwdShape *query) {
   static const BwdMaps kNoMaps{};
   static const BwdTmaParams kNoParams{};
   const BwdMaps &m = maps ? *maps : kNoMaps;
   const BwdTmaParams &pp = p ? *p : kNoParams;
-  if (s.lpc == 4 && s.warps == 4) return run_bwd<InT, GT, 16, 4, 4>(s, m, pp, stream, smem_out);
-  if (s.lpc == 4 && s.warps == 2) return run_bwd<InT, GT, 16, 4, 2>(s, m, pp, stream, smem_out);
-  if (s.lpc == 2 && s.warps == 4) return run_bwd<InT, GT, 8, 2, 4>(s, m, pp, stream, smem_out);
-  if (s.lpc == 2 && s.warps == 2) return run_bwd<InT, GT, 8, 2, 2>(s, m, pp, stream, smem_out);
+  if (s.lpc == 4 && s.warps == 4) return run_bwd<InT, GT, 16, 4, 4>(s, m, pp, stream, query);
+  if (s.lpc == 4 && s.warps == 2) return run_bwd<InT, GT, 16, 4, 2>(s, m, pp, stream, query);
+  if (s.lpc == 2 && s.warps == 4) return run_bwd<InT, GT, 8, 2, 4>(s, m, pp, stream, query);
+  if (s.lpc == 2 && s.warps == 2) return run_bwd<InT, GT, 8, 2, 2>(s, m, pp, stream, query);
   return cudaErrorInvalidValue;
 }
 
 cudaError_t bwd_dispatch(int in_dtype, int out_dtype, const BwdShape &s, const BwdMaps *maps,
-                         const BwdTmaParams *p, cudaStream_t stream, size_t *smem_out) {
+                         const BwdTmaParams *p, cudaStream_t stream, BwdShape *query) {
   constexpr int kF32 = 0, kBF16 = 1;  // ssm_dtype values
   if (in_dtype == kBF16 && out_dtype == kBF16)
-    return bwd_by_shape<__nv_bfloat16, __nv_bfloat16>(s, maps, p, stream, smem_out);
+    return bwd_by_shape<__nv_bfloat16, __nv_bfloat16>(s, maps, p, stream, query);
   if (in_dtype == kBF16 && out_dtype == kF32)
-    return bwd_by_shape<__nv_bfloat16, float>(s, maps, p, stream, smem_out);
+    return bwd_by_shape<__nv_bfloat16, float>(s, maps, p, stream, query);
   if (in_dtype == kF32 && out_dtype == kF32)
-    return bwd_by_shape<float, float>(s, maps, p, stream, smem_out);
+    return bwd_by_shape<float, float>(s, maps, p, stream, query);
   return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
-// Four scan warps when the row tiles still give every SM three CTAs, else
-// two (twice the row tiles).
+// Two or four scan warps: whichever fills the resident CTA slots of the
+// device best over its whole number of waves (every CTA runs one row tile
+// over the whole sequence, so a last partial wave leaves SMs idle); ties go
+// to four (fewer load warps).
 bool choose_bwd_shape(int in_dtype, int out_dtype, int64_t batch, int64_t seqlen, int64_t dim,
                       int ns, int warps, int sms, BwdShape *out) {
   if (ns != 16 && ns != 8) return false;
@@ -550,22 +566,36 @@ bool choose_bwd_shape(int in_dtype, int out_dtype, int64_t batch, int64_t seqlen
   const int es = in_dtype == 1 ? 2 : 4, gs = out_dtype == 1 ? 2 : 4;
   if (in_dtype == 0 && out_dtype == 1) return false;  // no such variant
   if ((dim * es) % 16 != 0 || (dim * gs) % 16 != 0 || (ns * es) % 16 != 0) return false;
-  BwdShape s;
-  s.lpc = ns / 4;
-  const int gpw = 32 / s.lpc;
-  auto rows_for = [&](int w) { return batch * ((dim + w * gpw - 1) / (w * gpw)); };
-  s.warps = warps ? warps : (rows_for(4) >= 3LL * sms ? 4 : 2);
-  s.DT = s.warps * gpw;
-  s.nDT = (int)((dim + s.DT - 1) / s.DT);
-  s.rows = batch * s.nDT;
-  s.S = (int)((seqlen + kBwdStage - 1) / kBwdStage);
-  if (s.rows > INT32_MAX || s.rows * (int64_t)s.S > INT32_MAX / 2) return false;
-  s.ws_ck_floats = (size_t)s.rows * s.S * s.DT * ns;
-  s.ws_bc_floats = (size_t)s.rows * seqlen * 2 * ns;
-  if (bwd_dispatch(in_dtype, out_dtype, s, nullptr, nullptr, nullptr, &s.smem) != cudaSuccess)
-    return false;
-  *out = s;
-  return true;
+  bool found = false;
+  double best_fill = -1.0;
+  BwdShape best;
+  for (int w : {4, 2}) {
+    if (warps && w != warps) continue;
+    BwdShape s;
+    s.lpc = ns / 4;
+    s.warps = w;
+    s.DT = w * (32 / s.lpc);
+    s.nDT = (int)((dim + s.DT - 1) / s.DT);
+    s.rows = batch * s.nDT;
+    s.S = (int)((seqlen + kBwdStage - 1) / kBwdStage);
+    if (s.rows > INT32_MAX || s.rows * (int64_t)s.S > INT32_MAX / 2) continue;
+    s.ws_ck_floats = (size_t)s.rows * s.S * s.DT * ns;
+    s.ws_bc_floats = (size_t)s.rows * seqlen * 2 * ns;
+    if (bwd_dispatch(in_dtype, out_dtype, s, nullptr, nullptr, nullptr, &s) != cudaSuccess ||
+        s.occ < 1) {
+      cudaGetLastError();
+      continue;
+    }
+    const int64_t slots = (int64_t)s.occ * sms;
+    const double fill = (double)s.rows / (double)(((s.rows + slots - 1) / slots) * slots);
+    if (!found || fill > best_fill + 1e-9) {
+      found = true;
+      best_fill = fill;
+      best = s;
+    }
+  }
+  if (found) *out = best;
+  return found;
 }
 
 cudaError_t launch_bwd_tma(int in_dtype, int out_dtype, const BwdShape &s, const BwdMaps &maps,
