@@ -90,8 +90,8 @@ def algorithmic_counts(inp, backward=False):
     exp+log for softplus and exp+reciprocal for the silu gate.
 
     Backward bytes: the forward inputs and dy read once, the fp32 gradients
-    dx, ddelta, dz (B,L,D) and dB, dC (B,L,N) written once, the per-16-token
-    state checkpoints (B,D,L/16,N) fp32 written and read once, dA/dD/dbias
+    dx, ddelta, dz (B,L,D) and dB, dC (B,L,N) written once, the per-8-token
+    stage-start states (B,D,L/8,N) fp32 written and read once, dA/dD/dbias
     and h0/dh_last/dh0 once.  mufu: the state's exp is evaluated three times
     (checkpoint pass, recomputation, reverse walk), the per-token ones twice."""
     B, L, D, N = inp.Bsz, inp.L, inp.D, inp.N
@@ -108,7 +108,7 @@ def algorithmic_counts(inp, backward=False):
     else:
         byt = es_in * n_bld + es_out * B * L * D + es_in * 2 * B * L * N   # inputs + dy
         byt += 4 * n_bld + 4 * 2 * B * L * N                             # dx, ddelta, dz, dB, dC
-        byt += 2 * 4 * B * D * ((L + 15) // 16) * N                     # checkpoints out + in
+        byt += 2 * 4 * B * D * ((L + 7) // 8) * N                       # stage starts out + in
         byt += 2 * params + 4 * B * D * N * (1 + 2 * (inp.h0 is not None))
         mufu = 3 * B * L * D * N + 2 * per_tok
     return {"updates": B * L * D * N, "bytes": byt, "mufu": mufu}

@@ -331,6 +331,15 @@ SSM_API ssm_status ssm_scan_set_debug(ssm_scan_plan *plan, uint64_t wait_timeout
 SSM_API ssm_status ssm_probe_peak(int kind, int64_t iters, int blocks, float *sink,
                                   int64_t *ops, ssm_stream_t stream);
 
+/* The kernels' two implementations of 2^x on n device floats x (a check of
+ * the FMA-pipe one, no counterpart in the pages): y_fma receives the
+ * range-reduced polynomial that kernel option bit 3 uses for a quarter of the
+ * state exponentials, y_sfu the special-function unit's ex2.approx.  All three
+ * are device pointers of n floats; enqueued on `stream`.  Returns
+ * SSM_ERR_INVALID_ARG for a negative n or a null pointer with n > 0. */
+SSM_API ssm_status ssm_probe_exp2(const float *x, float *y_fma, float *y_sfu, int64_t n,
+                                  ssm_stream_t stream);
+
 /* One compiled variant of the fused kernel. */
 typedef struct {
   int dstate, lanes_per_chan, chans_per_lane, warps_per_cta, tile_t;

@@ -130,6 +130,8 @@ def load_library(path: str | None = None):
         lib.ssm_probe_peak.argtypes = [ctypes.c_int, ctypes.c_int64, ctypes.c_int, _vp,
                                        ctypes.POINTER(ctypes.c_int64), _vp]
         lib.ssm_probe_peak.restype = st
+        lib.ssm_probe_exp2.argtypes = [_vp, _vp, _vp, ctypes.c_int64, _vp]
+        lib.ssm_probe_exp2.restype = st
         lib.ssm_scan_list_variants.argtypes = [ctypes.c_int, ctypes.c_int,
                                                ctypes.POINTER(Variant), ctypes.c_int]
         lib.ssm_scan_list_variants.restype = ctypes.c_int
@@ -410,6 +412,17 @@ def probe_peak(kind: int, iters: int, blocks: int, sink, stream=None) -> int:
     _check(load_library().ssm_probe_peak(int(kind), int(iters), int(blocks), _ptr(sink),
                                          ctypes.byref(ops), st), "ssm_probe_peak")
     return ops.value
+
+
+def probe_exp2(x):
+    """The kernels' two 2^x implementations on the fp32 device tensor x:
+    returns (FMA-pipe polynomial, ex2.approx) as tensors shaped like x."""
+    _need(x, "x", tuple(x.shape), torch.float32, x.device)
+    y_fma, y_sfu = torch.empty_like(x), torch.empty_like(x)
+    st = ctypes.c_void_p(torch.cuda.current_stream(x.device).cuda_stream)
+    _check(load_library().ssm_probe_exp2(_ptr(x), _ptr(y_fma), _ptr(y_sfu), x.numel(), st),
+           "ssm_probe_exp2")
+    return y_fma, y_sfu
 
 
 def flags_for(*, z=None, D=None, delta_bias=None, h0=None, delta_softplus=True,

@@ -135,6 +135,30 @@ __device__ __forceinline__ float2 zoh_coef2(float2 u, float2 e, float2 dlt, floa
   return make_float2(fabsf(u.x) < 0.25f ? small.x : large.x,
                      fabsf(u.y) < 0.25f ? small.y : large.y);
 }
+// 2^x for a pair on the FMA pipe instead of the special-function unit
+// (Cody-Waite range reduction): x = n + f with n the nearest integer (adding
+// 1.5 * 2^23 rounds x to an integer in the low mantissa bits) and f in
+// [-1/2, 1/2]; 2^f = 1 + f * Q(f), Q of degree 4 fitted to (2^f - 1) / f for
+// relative error (csrc/fit_exp2.py derives and checks the coefficients: max
+// relative error 1.8e-7 in float32), so f = 0 gives exactly 1; 2^n is added
+// to the exponent field.  x is first clamped to [-125, 127] so the exponent
+// never wraps (below, the result is a number under 2^-124 where ex2.approx
+// flushes to 0; above, it stays finite).
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+  x = make_float2(fminf(fmaxf(x.x, -125.f), 127.f), fminf(fmaxf(x.y, -125.f), 127.f));
+  const float2 t = fadd2(x, make_float2(12582912.f, 12582912.f));
+  const float2 n = fadd2(t, make_float2(-12582912.f, -12582912.f));
+  const float2 f = ffma2(n, make_float2(-1.f, -1.f), x);
+  float2 q = ffma2(make_float2(0.00132186722f, 0.00132186722f), f,
+                   make_float2(0.00967169832f, 0.00967169832f));
+  q = ffma2(q, f, make_float2(0.0555089302f, 0.0555089302f));
+  q = ffma2(q, f, make_float2(0.24022238f, 0.24022238f));
+  q = ffma2(q, f, make_float2(0.693146884f, 0.693146884f));
+  const float2 p = ffma2(q, f, make_float2(1.f, 1.f));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
 constexpr float kLn2 = 0.6931471805599453f;
 
 template <typename T> __device__ __forceinline__ float to_f32(T v);

@@ -50,7 +50,33 @@ __global__ void __launch_bounds__(kThreads) ffma_probe(int64_t iters, float *sin
   if (s == 12345.f) sink[blockIdx.x] = s;
 }
 
+// Both 2^x implementations of the kernels on the same inputs.
+__global__ void __launch_bounds__(256) exp2_pair_kernel(const float *x, float *y_fma,
+                                                        float *y_sfu, int64_t n) {
+  const int64_t i = 2 * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float2 v = make_float2(x[i], i + 1 < n ? x[i + 1] : 0.f);
+  const float2 f = ssm::exp2_fma2(v);
+  y_fma[i] = f.x;
+  y_sfu[i] = ssm::ex2_approx(v.x);
+  if (i + 1 < n) {
+    y_fma[i + 1] = f.y;
+    y_sfu[i + 1] = ssm::ex2_approx(v.y);
+  }
+}
+
 }  // namespace
+
+extern "C" SSM_API ssm_status ssm_probe_exp2(const float *x, float *y_fma, float *y_sfu,
+                                             int64_t n, ssm_stream_t stream) {
+  if (n < 0 || (n > 0 && (!x || !y_fma || !y_sfu))) return SSM_ERR_INVALID_ARG;
+  if (n == 0) return SSM_OK;
+  const int64_t pairs = (n + 1) / 2;
+  if ((pairs + 255) / 256 > INT32_MAX) return SSM_ERR_UNSUPPORTED;
+  exp2_pair_kernel<<<(unsigned)((pairs + 255) / 256), 256, 0,
+                     reinterpret_cast<cudaStream_t>(stream)>>>(x, y_fma, y_sfu, n);
+  return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
 
 extern "C" SSM_API ssm_status ssm_probe_peak(int kind, int64_t iters, int blocks,
                                              float *sink, int64_t *ops, ssm_stream_t stream) {

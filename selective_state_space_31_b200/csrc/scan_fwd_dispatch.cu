@@ -123,6 +123,7 @@ double warps_weight(int warps) { return warps == 2 ? 0.8 : 1.0; }
 double opt_weight(int opt, int lpc, int tt, int segments) {
   if (opt == 0) return 1.0;
   if (opt & 4) return 0.9;
+  if (opt & 8) return 0.9;
   if (segments > 1 || lpc != 8 || tt != 64) return 0.97;
   return opt == 1 ? 1.05 : opt == 2 ? 1.04 : 1.03;
 }

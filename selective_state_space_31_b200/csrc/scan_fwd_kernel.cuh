@@ -154,12 +154,17 @@ struct ItemPos {
 // registers capped so that five CTAs fit on an SM (more warps in flight);
 // bit 2 (bf16 inputs): the load warp widens each stage's B and C to fp32 in
 // shared memory once for the CTA, instead of every lane widening the values
-// it reads at every token.
+// it reads at every token; bit 3: a quarter of the state exponentials on the
+// FMA pipe (one channel per lane, even states per lane).
 template <typename InT, typename OutT, int NS, int LPC, int KC, int WARPS, int TT, bool ZOH,
           bool CARRY, bool CONV, int OPT>
 __global__ void __launch_bounds__((WARPS + 1) * 32, (OPT & 2) ? 5 : 0)
     fwd_kernel(const __grid_constant__ TmaMaps maps, const FwdParams p) {
   constexpr bool BCF = (OPT & 4) != 0 && std::is_same<InT, __nv_bfloat16>::value;
+  // OPT bit 3: one state pair in four (by token and pair index) takes its
+  // exponentials on the FMA pipe (exp2_fma2) instead of the special-function
+  // unit; the choice is fixed at compile time in the unrolled loops
+  auto fma_exp = [](int pair_index) { return (OPT & 8) != 0 && pair_index % 4 == 0; };
   using Cfg = FwdCfg<InT, OutT, NS, LPC, KC, WARPS, TT, CONV, CARRY, BCF>;
   constexpr int NPL = Cfg::NPL, GPW = Cfg::GPW, DT = Cfg::DT, RAW = Cfg::RAW,
                 TPL = Cfg::TPL;
@@ -481,7 +486,8 @@ __global__ void __launch_bounds__((WARPS + 1) * 32, (OPT & 2) ? 5 : 0)
 #pragma unroll
             for (int k = 0; k < NP; ++k) {
               const float2 arg = fmul2(dA, make_float2(A2[0][2 * k], A2[0][2 * k + 1]));
-              a[k] = make_float2(ex2_approx(arg.x), ex2_approx(arg.y));
+              a[k] = fma_exp(t * NP + k) ? exp2_fma2(arg)
+                                         : make_float2(ex2_approx(arg.x), ex2_approx(arg.y));
               bx[k] = fmul2(dX, make_float2(bv[2 * k], bv[2 * k + 1]));
               cc[k] = make_float2(cv[2 * k], cv[2 * k + 1]);
             }
@@ -533,7 +539,9 @@ __global__ void __launch_bounds__((WARPS + 1) * 32, (OPT & 2) ? 5 : 0)
 #pragma unroll
               for (int i = 0; i < NPL; i += 2) {
                 const float2 arg = fmul2(dA, make_float2(A2[0][i], A2[0][i + 1]));
-                const float2 a = make_float2(ex2_approx(arg.x), ex2_approx(arg.y));
+                const float2 a = fma_exp(t * (NPL / 2) + i / 2)
+                                     ? exp2_fma2(arg)
+                                     : make_float2(ex2_approx(arg.x), ex2_approx(arg.y));
                 float2 bx = fmul2(dX, make_float2(bv[i], bv[i + 1]));
                 if constexpr (ZOH)  // dX holds x: Bbar x = ((e^u - 1) / A) * (B x)
                   bx = fmul2(zoh_coef2(fmul2(arg, make_float2(kLn2, kLn2)), a, dA,

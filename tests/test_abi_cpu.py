@@ -105,3 +105,9 @@ def test_binding_refuses_missing_library(tmp_path):
             bnd.load_library(str(tmp_path / "nope.so"))
         finally:
             bnd._lib = saved
+
+
+def test_probe_exp2_validates_before_touching_cuda(lib):
+    assert lib.ssm_probe_exp2(None, None, None, -1, None) == bnd.ERR_INVALID_ARG
+    assert lib.ssm_probe_exp2(None, None, None, 4, None) == bnd.ERR_INVALID_ARG
+    assert lib.ssm_probe_exp2(None, None, None, 0, None) == bnd.OK
