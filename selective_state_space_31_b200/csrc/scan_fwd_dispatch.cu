@@ -119,7 +119,11 @@ double warps_weight(int warps) { return warps == 2 ? 0.8 : 1.0; }
 // elsewhere, and with segments, the plain loop was as fast or faster.  B and
 // C widened by the load warp (bit 2) took 2-10 % longer on every workload
 // (wider slots cost a CTA per SM at 64-token stages; at equal occupancy the
-// removed widening did not shorten the latency-bound loop).
+// removed widening did not shorten the latency-bound loop).  A quarter of
+// the exponentials on the FMA pipe (bit 3) took 4-27 % longer, in the carry
+// pass too although its special-function pipe is the busiest (82 %): the
+// polynomial's eight instructions per exponential cost more issue than the
+// relief is worth.
 double opt_weight(int opt, int lpc, int tt, int segments) {
   if (opt == 0) return 1.0;
   if (opt & 4) return 0.9;

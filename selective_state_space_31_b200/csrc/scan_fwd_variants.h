@@ -15,7 +15,7 @@
   X(16, 4, 1, 4, 32, false, false, false, 2) X(16, 8, 1, 4, 64, false, false, false, 2)  \
   X(16, 4, 1, 4, 32, false, false, false, 3) X(16, 8, 1, 4, 64, false, false, false, 3)  \
   X(16, 8, 1, 4, 64, false, false, false, 5) X(16, 4, 1, 4, 32, false, false, false, 4)  \
-  X(16, 8, 1, 4, 64, false, false, false, 9) X(16, 4, 1, 4, 32, false, false, false, 8)  \
+  X(16, 4, 1, 4, 32, false, false, false, 8)                                              \
   X(16, 1, 1, 4, 32, false, false, false, 0) X(16, 2, 1, 4, 32, false, false, false, 0)                      \
   X(16, 4, 1, 4, 32, false, false, false, 0) X(16, 4, 1, 4, 64, false, false, false, 0)                      \
   X(16, 8, 1, 4, 32, false, false, false, 0) X(16, 8, 1, 4, 64, false, false, false, 0)                      \
