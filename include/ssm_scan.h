@@ -149,7 +149,7 @@ typedef struct {
   int grid;           /* CTAs (any number: work items go out by ticket; capped by the items) */
   int tile_t;         /* tokens per pipeline stage: 32 or 64 */
   int chans_per_lane; /* 1 or 2 */
-  int segments;       /* segments per row: 1, 2, 4 or 8 (1 = none) */
+  int segments;       /* segments per row: 1, 2, 4, 8 or 16 (1 = none) */
   int scan_loop;      /* 1 + variant options (0 = free choice): option bit 0 =
                          software-pipelined scan loop (the next token's exponentials and
                          loads issued before this token's update), bit 1 = registers

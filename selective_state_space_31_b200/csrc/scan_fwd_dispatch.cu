@@ -238,7 +238,7 @@ cudaError_t choose_fwd_shape(int in_dtype, int out_dtype, int64_t batch, int64_t
     }
     const int64_t rows = batch * ((dim + DT - 1) / DT);
     const int64_t S = std::max<int64_t>(1, (seqlen + v.tt - 1) / v.tt);
-    for (int M : {1, 2, 4, 8}) {
+    for (int M : {1, 2, 4, 8, 16}) {
       if (o.segments && M != o.segments) continue;
       const double w = shape_weight(v.lpc, v.kc, v.tt) * warps_weight(v.warps) *
                        opt_weight(v.opt, v.lpc, v.tt, M) * segmented_weight(v.lpc, v.tt, M);

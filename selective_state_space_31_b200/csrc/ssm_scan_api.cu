@@ -144,7 +144,8 @@ ssm_status plan_tma(ssm_scan_plan *pl) {
   if (pl->cfg.chans_per_lane && pl->cfg.chans_per_lane != 1 && pl->cfg.chans_per_lane != 2)
     return SSM_ERR_INVALID_ARG;
   if (pl->cfg.segments && pl->cfg.segments != 1 && pl->cfg.segments != 2 &&
-      pl->cfg.segments != 4 && pl->cfg.segments != 8)
+      pl->cfg.segments != 4 && pl->cfg.segments != 8 &&
+      pl->cfg.segments != 16)
     return SSM_ERR_INVALID_ARG;
   ssm::FwdOverrides o{pl->cfg.lanes_per_chan, pl->cfg.warps_per_cta, pl->cfg.tile_t,
                       pl->cfg.grid};

@@ -215,3 +215,17 @@ def test_progress_without_co_residency():
     assert plan.status() == 0
     ry, rh = gu.run_oracle(inp)
     gu.assert_parity(gy, ry, gh, rh, gu.TOL["bf16"], str(info))
+
+
+def test_sixteen_segments():
+    """Sixteen segments: the last segments fold sixty-odd sub-chunk maps
+    before their first token; ragged length, h0 on."""
+    inp = synth.make_fwd(1, 8190, 256, 16, seed=70, has_h0=True)
+    plan = gu.make_plan(inp)
+    plan.set_config(segments=16, tile_t=32)
+    info = plan.info()
+    assert info["segments"] == 16, info
+    gy, gh = gu.run_gpu(inp, plan)
+    assert plan.status() == 0
+    ry, rh = gu.run_oracle(inp)
+    gu.assert_parity(gy, ry, gh, rh, gu.TOL["bf16"], str(info))
