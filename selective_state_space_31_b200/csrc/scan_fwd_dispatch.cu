@@ -165,16 +165,17 @@ int parts_per_chain(int64_t R, int64_t P, int64_t S) {
 // ~76 % of the special-function rate, while one lane per channel (few warps
 // per SM) took 45 % longer.  So: the main variant's split and its B/C
 // widening option first, then 4 lanes per channel.  o_lpc / o_opt (1 + the
-// OPT bits) restrict the choice when non-zero.
+// OPT bits) / o_kc restrict the choice when non-zero.
 bool pick_carry(int in_dtype, int out_dtype, const VariantDesc &main, int sms,
-                const VariantDesc *all, int nall, int o_lpc, int o_opt, LaunchShape *cls,
-                int *cDT, int *cocc) {
+                const VariantDesc *all, int nall, int o_lpc, int o_opt, int o_kc,
+                LaunchShape *cls, int *cDT, int *cocc) {
   int best = -1;
   double best_score = -1.0;
   for (int i = 0; i < nall; ++i) {
     const VariantDesc &v = all[i];
     if (!v.carry || v.ns != main.ns || v.zoh != main.zoh || v.tt != main.tt ||
-        v.conv != main.conv || (o_lpc && v.lpc != o_lpc) || (o_opt && v.opt != o_opt - 1))
+        v.conv != main.conv || (o_lpc && v.lpc != o_lpc) || (o_opt && v.opt != o_opt - 1) ||
+        (o_kc && v.kc != o_kc))
       continue;
     const double score = (v.lpc == main.lpc && v.kc == main.kc ? 2.0 : 0.0) +
                          ((v.opt & 4) == (main.opt & 4) ? 1.0 : 0.0) +
@@ -246,7 +247,7 @@ cudaError_t choose_fwd_shape(int in_dtype, int out_dtype, int64_t batch, int64_t
       LaunchShape cls{};
       int cDT = 0, cocc = 0;
       if (M > 1 && !pick_carry(in_dtype, out_dtype, v, sms, all, nall, o.carry_lpc, o.carry_opt,
-                               &cls, &cDT, &cocc))
+                               o.carry_kc, &cls, &cDT, &cocc))
         continue;
       const int64_t vrows = rows * M;
       const int64_t cap = std::min(vrows, (int64_t)info.occ * sms);
@@ -329,7 +330,7 @@ cudaError_t choose_map_shape(int in_dtype, int out_dtype, int64_t batch, int64_t
                          fs.ls.conv, fs.ls.opt};
   LaunchShape cls{};
   int cDT = 0, cocc = 0;
-  if (!pick_carry(in_dtype, out_dtype, main, sms, all, nall, 0, 0, &cls, &cDT, &cocc))
+  if (!pick_carry(in_dtype, out_dtype, main, sms, all, nall, 0, 0, 0, &cls, &cDT, &cocc))
     return cudaErrorInvalidValue;
   const int64_t rows = batch * ((dim + cDT - 1) / cDT);
   const int64_t S = fs.S;

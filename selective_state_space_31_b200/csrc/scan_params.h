@@ -91,6 +91,7 @@ struct FwdOverrides {
   int opt = 0;       // 1 + the variant's OPT bits (0 = free choice)
   int carry_lpc = 0;  // carry pass: lanes per channel (0 = free choice)
   int carry_opt = 0;  // carry pass: 1 + its OPT bits (0 = free choice)
+  int carry_kc = 0;   // carry pass: channels per lane (0 = free choice)
 };
 // A launch shape of the fused kernel with its work split.
 struct FwdShape {

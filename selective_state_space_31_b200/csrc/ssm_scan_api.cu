@@ -154,6 +154,7 @@ ssm_status plan_tma(ssm_scan_plan *pl) {
   o.opt = pl->cfg.scan_loop;
   o.carry_lpc = pl->cfg.carry_lanes_per_chan;
   o.carry_opt = pl->cfg.carry_loop;
+  o.carry_kc = pl->cfg.carry_chans_per_lane;
   ssm::FwdShape fs;
   if (ssm::choose_fwd_shape((int)d.in_dtype, (int)d.out_dtype, d.batch, d.seqlen, d.dim, ns,
                             (d.flags & SSM_ZOH) != 0, (d.flags & SSM_CONV_X) != 0, pl->num_sms, o,
@@ -332,6 +333,7 @@ ssm_status ssm_scan_get_info(const ssm_scan_plan *pl, ssm_scan_info *info) {
     info->scan_loop = 1 + pl->ls.opt;
     info->carry_lanes_per_chan = pl->fs.M > 1 ? pl->fs.cls.lpc : 0;
     info->carry_loop = pl->fs.M > 1 ? 1 + pl->fs.cls.opt : 0;
+    info->carry_chans_per_lane = pl->fs.M > 1 ? pl->fs.cls.kc : 0;
   }
   info->launches_per_call = pl->path == PATH_TMA && pl->fs.M > 1 ? 2 : 1;
   ssm::BwdShape bs;
@@ -351,7 +353,8 @@ ssm_status ssm_scan_set_config(ssm_scan_plan *pl, const ssm_scan_config *cfg) {
   if (cfg->lanes_per_chan < 0 || cfg->warps_per_cta < 0 || cfg->grid < 0 || cfg->tile_t < 0 ||
       cfg->chans_per_lane < 0 || cfg->segments < 0 || cfg->scan_loop < 0 || cfg->scan_loop > 16 ||
       cfg->carry_lanes_per_chan < 0 || cfg->carry_loop < 0 || cfg->carry_loop > 16 ||
-      (cfg->bwd_warps_per_cta != 0 && cfg->bwd_warps_per_cta != 2 && cfg->bwd_warps_per_cta != 4))
+      (cfg->bwd_warps_per_cta != 0 && cfg->bwd_warps_per_cta != 2 && cfg->bwd_warps_per_cta != 4) ||
+      cfg->carry_chans_per_lane < 0 || cfg->carry_chans_per_lane > 2)
     return SSM_ERR_INVALID_ARG;
   DeviceGuard guard(pl->device);
   if (!guard.ok) return SSM_ERR_CUDA;

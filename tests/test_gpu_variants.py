@@ -131,14 +131,14 @@ def test_every_carry_variant(in_dt, out_dt, zoh):
             cfg = dict(lanes_per_chan=v["lanes_per_chan"], warps_per_cta=v["warps_per_cta"],
                        tile_t=v["tile_t"], chans_per_lane=v["chans_per_lane"], segments=4,
                        scan_loop=1 + v["opt"], carry_lanes_per_chan=c["lanes_per_chan"],
-                       carry_loop=1 + c["opt"])
+                       carry_loop=1 + c["opt"], carry_chans_per_lane=c["chans_per_lane"])
             try:
                 info, gy, gh, st = _run(inp, dev, cfg)
             except bnd.SsmError as e:
                 failures.append(f"{cfg}: refused ({e})")
                 continue
-            if (info["carry_lanes_per_chan"], info["carry_loop"]) != \
-                    (c["lanes_per_chan"], 1 + c["opt"]) or info["segments"] != 4:
+            if (info["carry_lanes_per_chan"], info["carry_loop"], info["carry_chans_per_lane"]) != \
+                    (c["lanes_per_chan"], 1 + c["opt"], c["chans_per_lane"]) or info["segments"] != 4:
                 failures.append(f"{cfg}: plan chose {info}")
             try:
                 assert st == 0, f"device status {st}"
