@@ -491,23 +491,18 @@ def run_fwd(name, steps, warmup, args, rank, world, device, peaks, e2e_steps,
             return None if a is None else torch.from_numpy(np.ascontiguousarray(a)).to(dt).pin_memory()
         host = dict(x=pinned(inp.x, tdt[inp.in_dtype]), delta=pinned(inp.delta, tdt[inp.in_dtype]),
                     z=pinned(inp.z, tdt[inp.in_dtype]), B=pinned(inp.B, tdt[inp.in_dtype]),
-                    C=pinned(inp.C, tdt[inp.in_dtype]), h0=pinned(inp.h0, torch.float32))
-        dev_in = sets[0]
+                    C=pinned(inp.C, tdt[inp.in_dtype]), h0=pinned(inp.h0, torch.float32),
+                    A=pinned(inp.A, torch.float32), D=pinned(inp.Dskip, torch.float32),
+                    delta_bias=pinned(inp.delta_bias, torch.float32))
         y_h = torch.empty((inp.Bsz, inp.L, inp.D), dtype=tdt[inp.out_dtype]).pin_memory()
         hl_h = torch.empty((inp.Bsz, inp.D, inp.N), dtype=torch.float32).pin_memory()
-        y_d, hl_d = outs[0]
         h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
         d2h = y_h.numel() * y_h.element_size() + hl_h.numel() * 4
 
-        def e2e_step():
-            for k, v in host.items():
-                if v is not None:
-                    dev_in[k].copy_(v, non_blocking=True)
-            plan.fwd(dev_in["x"], dev_in["delta"], dev_in["A"], dev_in["B"], dev_in["C"],
-                     D=dev_in["D"], z=dev_in["z"], delta_bias=dev_in["delta_bias"],
-                     h0=dev_in["h0"], y=y_d, h_last=hl_d)
-            y_h.copy_(y_d, non_blocking=True)
-            hl_h.copy_(hl_d, non_blocking=True)
+        def e2e_step():  # the C-ABI call on host buffers: chunked copy-in / scan / copy-out
+            plan.fwd_host(host["x"], host["delta"], host["A"], host["B"], host["C"],
+                          D=host["D"], z=host["z"], delta_bias=host["delta_bias"],
+                          h0=host["h0"], y=y_h, h_last=hl_h, stream=stream)
 
         for _ in range(2):
             e2e_step()
@@ -525,7 +520,8 @@ def run_fwd(name, steps, warmup, args, rank, world, device, peaks, e2e_steps,
         e2e = {"value": replica_throughput(counts["updates"], world, e_ms),
                "unit": "state-updates/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": e_ms, "steps": e2e_steps,
-               "note": "host->device inputs and device->host y/h_last over PCIe each step"}
+               "note": "ssm_scan_fwd_host on pinned host buffers: inputs in and y/h_last out "
+                       "over PCIe each step, overlapped with the scan chunk by chunk"}
         del host, y_h, hl_h
 
     info = plan.info()

@@ -186,6 +186,33 @@ SSM_API ssm_status ssm_scan_fwd(ssm_scan_plan *plan, const void *x, const void *
                         const void *C, const float *D, const void *z,
                         const float *h0, void *y, float *h_last, ssm_stream_t stream);
 
+/* Forward pass with every tensor in HOST memory: x, delta, z, B, C, y, h0,
+ * h_last and the parameters A, D, delta_bias (shapes, layouts and flags as
+ * for ssm_scan_fwd).  For a caller whose data is not on the device: the
+ * library streams the sequence through the GPU in chunks of tokens, with the
+ * copy-in of chunk c+1, the scan of chunk c (its state carried on from chunk
+ * c-1 on the device) and the copy-out of chunk c-1's y overlapping on three
+ * streams, so the host<->device transfers rather than the scan set the time.
+ * The host buffers should be page-locked (cudaHostAlloc / cudaHostRegister,
+ * torch's pin_memory) for the copies to overlap; pageable memory works but
+ * serialises.  Stream-ordered: the work starts behind `stream`'s earlier
+ * work and `stream` waits for all of it, so synchronising `stream` (or an
+ * event recorded on it after the call) covers the copy-out of y and h_last;
+ * the host buffers must stay valid and unmodified until then.  Calls on one
+ * plan share its staging memory: issue them on one stream (or synchronise
+ * between them).
+ * `chunk_tokens` is the number of tokens per chunk (0 = the library's
+ * choice, about L/12 rounded up to a multiple of 64).  The first call (and a
+ * call with another chunk length) allocates three chunk slots of device
+ * staging memory and the plans for the chunk lengths; later calls reuse
+ * them.  SSM_A_DIRECT and SSM_CONV_X plans are refused with
+ * SSM_ERR_UNSUPPORTED; SSM_ERR_OOM if the staging memory cannot be had. */
+SSM_API ssm_status ssm_scan_fwd_host(ssm_scan_plan *plan, const void *x, const void *delta,
+                                     const float *delta_bias, const float *A, const void *B,
+                                     const void *C, const float *D, const void *z,
+                                     const float *h0, void *y, float *h_last,
+                                     int64_t chunk_tokens, ssm_stream_t stream);
+
 /* Forward pass fed by the causal conv front-end of the x branch, fused into
  * the scan kernel so the conv output never goes through HBM unless asked
  * for.  "Tong quan ..." (vietitpro.vn), section 5.3 "Toi uu hoa Kernel

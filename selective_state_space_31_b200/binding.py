@@ -100,6 +100,8 @@ def load_library(path: str | None = None):
         lib.ssm_scan_destroy.restype = st
         lib.ssm_scan_fwd.argtypes = [_vp] * 13
         lib.ssm_scan_fwd.restype = st
+        lib.ssm_scan_fwd_host.argtypes = [_vp] * 12 + [ctypes.c_int64, _vp]
+        lib.ssm_scan_fwd_host.restype = st
         lib.ssm_scan_fwd_conv.argtypes = [_vp] * 16
         lib.ssm_scan_fwd_conv.restype = st
         lib.ssm_scan_seq_map.argtypes = [_vp] * 9
@@ -254,6 +256,42 @@ class Plan:
                                     _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(h0), _ptr(y),
                                     _ptr(h_last), _stream(dev))
         _check(rc, "ssm_scan_fwd")
+        return y, h_last
+
+    def fwd_host(self, x, delta, A, B, C, D=None, z=None, delta_bias=None, h0=None, y=None,
+                 h_last=None, chunk_tokens=0, stream=None):
+        """Forward pass on CPU tensors (pinned for overlapped copies): the
+        library streams the sequence through the plan's device in chunks of
+        tokens (ssm_scan_fwd_host).  Returns (y, h_last) as CPU tensors; they
+        are complete once `stream` (default: the device's current stream)
+        has been synchronised."""
+        d, f = self.desc, self.flags
+        if f & (A_DIRECT | CONV_X):
+            raise ValueError("fwd_host takes neither A_DIRECT nor CONV_X plans")
+        Bz, L, Dm, N = d.batch, d.seqlen, d.dim, d.dstate
+        cpu = torch.device("cpu")
+        for name, t, shape, dt in (("x", x, (Bz, L, Dm), self.in_dtype),
+                                   ("delta", delta, (Bz, L, Dm), self.in_dtype),
+                                   ("z", z, (Bz, L, Dm), self.in_dtype),
+                                   ("B", B, (Bz, L, N), self.in_dtype),
+                                   ("C", C, (Bz, L, N), self.in_dtype),
+                                   ("A", A, (Dm, N), torch.float32),
+                                   ("D", D, (Dm,), torch.float32),
+                                   ("delta_bias", delta_bias, (Dm,), torch.float32),
+                                   ("h0", h0, (Bz, Dm, N), torch.float32)):
+            _need(t, name, shape, dt, cpu)
+        if y is None:
+            y = torch.empty((Bz, L, Dm), dtype=self.out_dtype).pin_memory()
+        _need(y, "y", (Bz, L, Dm), self.out_dtype, cpu)
+        if f & WANT_HLAST and h_last is None:
+            h_last = torch.empty((Bz, Dm, N), dtype=torch.float32).pin_memory()
+        _need(h_last, "h_last", (Bz, Dm, N), torch.float32, cpu)
+        st = ctypes.c_void_p(stream.cuda_stream if stream is not None
+                             else torch.cuda.current_stream(self.device).cuda_stream)
+        rc = self._lib.ssm_scan_fwd_host(self._h, _ptr(x), _ptr(delta), _ptr(delta_bias),
+                                         _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(h0),
+                                         _ptr(y), _ptr(h_last), int(chunk_tokens), st)
+        _check(rc, "ssm_scan_fwd_host")
         return y, h_last
 
     def fwd_conv(self, x_in, conv_w, delta, A, B, C, conv_b=None, D=None, z=None,

@@ -76,6 +76,11 @@ bool aligned16(const void *p) { return p == nullptr || (reinterpret_cast<uintptr
 
 }  // namespace
 
+namespace {
+struct HostPipe;
+void host_pipe_free(HostPipe *hp);
+}  // namespace
+
 struct ssm_scan_plan {
   ssm_scan_desc desc{};
   int device = 0;
@@ -99,6 +104,7 @@ struct ssm_scan_plan {
   size_t ws_state_bytes = 0, ws_flag_bytes = 0;
   uint64_t timeout_ns = kDefaultTimeoutNs;
   int64_t drop_unit = -1;
+  HostPipe *pipe = nullptr;  // staging of ssm_scan_fwd_host (allocated by its first call)
 };
 
 namespace {
@@ -303,6 +309,7 @@ ssm_status ssm_scan_destroy(ssm_scan_plan *pl) {
     if (pl->ws_flags) cudaFree(pl->ws_flags);
     if (pl->ws_agg) cudaFree(pl->ws_agg);
     if (pl->ws_map) cudaFree(pl->ws_map);
+    host_pipe_free(pl->pipe);
   }
   delete pl;
   return SSM_OK;
@@ -772,6 +779,217 @@ ssm_status ssm_scan_step(ssm_scan_plan *pl, const void *x, const void *delta,
   p.x = x; p.dt = delta; p.z = z; p.B = B; p.C = C;
   p.A = A; p.Dv = D; p.bias = delta_bias; p.state = state; p.y = y;
   return map_cuda(ssm::launch_step(p, reinterpret_cast<cudaStream_t>(stream_)));
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// ssm_scan_fwd_host: the sequence streamed through the device in chunks of
+// tokens, copies and scans overlapping on three streams
+// ---------------------------------------------------------------------------
+
+namespace {
+
+constexpr int kPipeSlots = 3;  // chunks in flight: copy-in, scan, copy-out
+
+struct HostPipe {
+  int64_t Lc = 0;                                  // tokens per chunk
+  ssm_scan_plan *body = nullptr, *tail = nullptr;  // plans for Lc and the last chunk's length
+  cudaStream_t s_in = nullptr, s_out = nullptr;
+  cudaEvent_t ev_start = nullptr, ev_done = nullptr;
+  cudaEvent_t ev_in[kPipeSlots] = {}, ev_comp[kPipeSlots] = {}, ev_out[kPipeSlots] = {};
+  unsigned char *slots = nullptr;  // kPipeSlots x [x | delta | z | B | C | y] of one chunk
+  size_t off_dt = 0, off_z = 0, off_B = 0, off_C = 0, off_y = 0, slot_bytes = 0;
+  float *params = nullptr;  // A (D x N), D (D), delta_bias (D)
+  float *hbuf = nullptr;    // 2 x (B, D, N): the state handed from chunk to chunk
+};
+
+void host_pipe_free(HostPipe *hp) {
+  if (!hp) return;
+  if (hp->body) ssm_scan_destroy(hp->body);
+  if (hp->tail) ssm_scan_destroy(hp->tail);
+  for (cudaEvent_t e : {hp->ev_start, hp->ev_done})
+    if (e) cudaEventDestroy(e);
+  for (int i = 0; i < kPipeSlots; ++i)
+    for (cudaEvent_t e : {hp->ev_in[i], hp->ev_comp[i], hp->ev_out[i]})
+      if (e) cudaEventDestroy(e);
+  if (hp->s_in) cudaStreamDestroy(hp->s_in);
+  if (hp->s_out) cudaStreamDestroy(hp->s_out);
+  if (hp->slots) cudaFree(hp->slots);
+  if (hp->params) cudaFree(hp->params);
+  if (hp->hbuf) cudaFree(hp->hbuf);
+  delete hp;
+}
+
+size_t align256(size_t v) { return (v + 255) / 256 * 256; }
+
+// A chunk plan: the parent's problem over `len` tokens, always with a
+// starting state and a final state (they carry the sequence across chunks).
+ssm_status make_chunk_plan(const ssm_scan_plan *pl, int64_t len, ssm_scan_plan **out) {
+  ssm_scan_desc d = pl->desc;
+  d.seqlen = len;
+  d.flags |= SSM_HAS_H0 | SSM_WANT_HLAST;
+  ssm_status st = ssm_scan_create(out, &d, pl->device);
+  if (st == SSM_OK) (*out)->timeout_ns = pl->timeout_ns;
+  return st;
+}
+
+ssm_status host_pipe_build(ssm_scan_plan *pl, int64_t Lc, HostPipe **out) {
+  const ssm_scan_desc &d = pl->desc;
+  HostPipe *hp = new (std::nothrow) HostPipe;
+  if (!hp) return SSM_ERR_OOM;
+  hp->Lc = Lc;
+  auto fail = [&](ssm_status st) {
+    cudaGetLastError();
+    host_pipe_free(hp);
+    return st;
+  };
+  const int64_t L = d.seqlen, nch = (L + Lc - 1) / Lc, tail = L - (nch - 1) * Lc;
+  ssm_status st = make_chunk_plan(pl, Lc, &hp->body);
+  if (st != SSM_OK) return fail(st);
+  if (tail != Lc && (st = make_chunk_plan(pl, tail, &hp->tail)) != SSM_OK) return fail(st);
+  const size_t ei = dtype_size(d.in_dtype), eo = dtype_size(d.out_dtype);
+  const size_t tok = (size_t)(d.batch * Lc);
+  const size_t xb = align256(tok * d.dim * ei), bb = align256(tok * d.dstate * ei);
+  hp->off_dt = xb;
+  hp->off_z = 2 * xb;
+  hp->off_B = 3 * xb;
+  hp->off_C = 3 * xb + bb;
+  hp->off_y = 3 * xb + 2 * bb;
+  hp->slot_bytes = hp->off_y + align256(tok * d.dim * eo);
+  const size_t nparam = (size_t)(d.dim * d.dstate + 2 * d.dim);
+  const size_t nstate = (size_t)(d.batch * d.dim * d.dstate);
+  if (cudaMalloc(&hp->slots, kPipeSlots * hp->slot_bytes) != cudaSuccess ||
+      cudaMalloc(&hp->params, nparam * sizeof(float)) != cudaSuccess ||
+      cudaMalloc(&hp->hbuf, 2 * std::max<size_t>(nstate, 1) * sizeof(float)) != cudaSuccess)
+    return fail(SSM_ERR_OOM);
+  if (cudaStreamCreateWithFlags(&hp->s_in, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaStreamCreateWithFlags(&hp->s_out, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaEventCreateWithFlags(&hp->ev_start, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&hp->ev_done, cudaEventDisableTiming) != cudaSuccess)
+    return fail(SSM_ERR_CUDA);
+  for (int i = 0; i < kPipeSlots; ++i)
+    if (cudaEventCreateWithFlags(&hp->ev_in[i], cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&hp->ev_comp[i], cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&hp->ev_out[i], cudaEventDisableTiming) != cudaSuccess)
+      return fail(SSM_ERR_CUDA);
+  *out = hp;
+  return SSM_OK;
+}
+
+// Tokens [l0, l0 + len) of every batch element of a (B, L, W) host tensor
+// into a contiguous (B, len, W) device buffer, or back.
+cudaError_t copy_tokens_in(void *dst, const void *src, const ssm_scan_desc &d, int64_t W,
+                           size_t es, int64_t l0, int64_t len, cudaStream_t s) {
+  const size_t row = (size_t)(len * W) * es;
+  return cudaMemcpy2DAsync(dst, row, static_cast<const unsigned char *>(src) + (size_t)(l0 * W) * es,
+                           (size_t)(d.seqlen * W) * es, row, (size_t)d.batch,
+                           cudaMemcpyHostToDevice, s);
+}
+cudaError_t copy_tokens_out(void *dst, const void *src, const ssm_scan_desc &d, int64_t W,
+                            size_t es, int64_t l0, int64_t len, cudaStream_t s) {
+  const size_t row = (size_t)(len * W) * es;
+  return cudaMemcpy2DAsync(static_cast<unsigned char *>(dst) + (size_t)(l0 * W) * es,
+                           (size_t)(d.seqlen * W) * es, src, row, row, (size_t)d.batch,
+                           cudaMemcpyDeviceToHost, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+ssm_status ssm_scan_fwd_host(ssm_scan_plan *pl, const void *x, const void *delta,
+                             const float *delta_bias, const float *A, const void *B,
+                             const void *C, const float *D, const void *z, const float *h0,
+                             void *y, float *h_last, int64_t chunk_tokens, ssm_stream_t stream_) {
+  if (!pl || chunk_tokens < 0) return SSM_ERR_INVALID_ARG;
+  const ssm_scan_desc &d = pl->desc;
+  const uint32_t f = d.flags;
+  if (f & (SSM_A_DIRECT | SSM_CONV_X)) return SSM_ERR_UNSUPPORTED;
+  const bool has_tokens = d.batch * d.seqlen * d.dim != 0;
+  if (has_tokens && (!x || !delta || !B || !C || !y)) return SSM_ERR_INVALID_ARG;
+  if (d.dim != 0 && !A) return SSM_ERR_INVALID_ARG;
+  if (((f & SSM_HAS_Z) != 0) != (z != nullptr) || ((f & SSM_HAS_D) != 0) != (D != nullptr) ||
+      ((f & SSM_HAS_DELTA_BIAS) != 0) != (delta_bias != nullptr) ||
+      ((f & SSM_HAS_H0) != 0) != (h0 != nullptr) ||
+      ((f & SSM_WANT_HLAST) != 0) != (h_last != nullptr))
+    return SSM_ERR_INVALID_ARG;
+  if (d.batch * d.dim == 0) return SSM_OK;
+  DeviceGuard guard(pl->device);
+  if (!guard.ok) return SSM_ERR_CUDA;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  const int64_t L = d.seqlen;
+  const size_t ei = dtype_size(d.in_dtype), eo = dtype_size(d.out_dtype);
+  const size_t nstate = (size_t)(d.batch * d.dim * d.dstate);
+  if (L == 0) {  // no tokens: h_last = h0 (or 0)
+    if (!h_last) return SSM_OK;
+    if (h0) return map_cuda(cudaMemcpyAsync(h_last, h0, nstate * 4, cudaMemcpyHostToHost, stream));
+    return map_cuda(cudaMemsetAsync(h_last, 0, nstate * 4, stream));
+  }
+  int64_t Lc = chunk_tokens ? chunk_tokens : ((L + 11) / 12 + 63) / 64 * 64;
+  Lc = std::min(Lc, L);
+  if (!pl->pipe || pl->pipe->Lc != Lc) {
+    host_pipe_free(pl->pipe);
+    pl->pipe = nullptr;
+    const ssm_status st = host_pipe_build(pl, Lc, &pl->pipe);
+    if (st != SSM_OK) return st;
+  }
+  HostPipe &hp = *pl->pipe;
+  const int64_t nch = (L + Lc - 1) / Lc;
+  float *dA = hp.params, *dD = hp.params + d.dim * d.dstate, *dbias = dD + d.dim;
+  auto ck = [](cudaError_t e) { return e == cudaSuccess; };
+  // the copies start behind the caller's earlier work on `stream`
+  if (!ck(cudaEventRecord(hp.ev_start, stream)) || !ck(cudaStreamWaitEvent(hp.s_in, hp.ev_start, 0)) ||
+      !ck(cudaStreamWaitEvent(hp.s_out, hp.ev_start, 0)))
+    return SSM_ERR_CUDA;
+  // parameters once; the state before the first chunk into hbuf[1]
+  if (!ck(cudaMemcpyAsync(dA, A, (size_t)(d.dim * d.dstate) * 4, cudaMemcpyHostToDevice, hp.s_in)) ||
+      (D && !ck(cudaMemcpyAsync(dD, D, (size_t)d.dim * 4, cudaMemcpyHostToDevice, hp.s_in))) ||
+      (delta_bias &&
+       !ck(cudaMemcpyAsync(dbias, delta_bias, (size_t)d.dim * 4, cudaMemcpyHostToDevice, hp.s_in))))
+    return SSM_ERR_CUDA;
+  float *hprev0 = hp.hbuf + nstate;
+  if (!ck(h0 ? cudaMemcpyAsync(hprev0, h0, nstate * 4, cudaMemcpyHostToDevice, hp.s_in)
+             : cudaMemsetAsync(hprev0, 0, nstate * 4, hp.s_in)))
+    return SSM_ERR_CUDA;
+  for (int64_t c = 0; c < nch; ++c) {
+    const int s = (int)(c % kPipeSlots);
+    const int64_t l0 = c * Lc, len = std::min(Lc, L - l0);
+    unsigned char *sb = hp.slots + s * hp.slot_bytes;
+    // copy-in of chunk c once the scan of chunk c - kPipeSlots has left the slot
+    if (c >= kPipeSlots && !ck(cudaStreamWaitEvent(hp.s_in, hp.ev_comp[s], 0))) return SSM_ERR_CUDA;
+    if (!ck(copy_tokens_in(sb, x, d, d.dim, ei, l0, len, hp.s_in)) ||
+        !ck(copy_tokens_in(sb + hp.off_dt, delta, d, d.dim, ei, l0, len, hp.s_in)) ||
+        (z && !ck(copy_tokens_in(sb + hp.off_z, z, d, d.dim, ei, l0, len, hp.s_in))) ||
+        !ck(copy_tokens_in(sb + hp.off_B, B, d, d.dstate, ei, l0, len, hp.s_in)) ||
+        !ck(copy_tokens_in(sb + hp.off_C, C, d, d.dstate, ei, l0, len, hp.s_in)) ||
+        !ck(cudaEventRecord(hp.ev_in[s], hp.s_in)))
+      return SSM_ERR_CUDA;
+    // the scan of chunk c on the caller's stream, from the state chunk c - 1 left
+    if (!ck(cudaStreamWaitEvent(stream, hp.ev_in[s], 0)) ||
+        (c >= kPipeSlots && !ck(cudaStreamWaitEvent(stream, hp.ev_out[s], 0))))
+      return SSM_ERR_CUDA;
+    float *hprev = hp.hbuf + ((c + 1) % 2) * nstate, *hnext = hp.hbuf + (c % 2) * nstate;
+    ssm_scan_plan *cp = len == Lc ? hp.body : hp.tail;
+    const ssm_status st =
+        ssm_scan_fwd(cp, sb, sb + hp.off_dt, delta_bias ? dbias : nullptr, dA, sb + hp.off_B,
+                     sb + hp.off_C, D ? dD : nullptr, z ? sb + hp.off_z : nullptr, hprev,
+                     sb + hp.off_y, hnext, stream_);
+    if (st != SSM_OK) return st;
+    if (!ck(cudaEventRecord(hp.ev_comp[s], stream))) return SSM_ERR_CUDA;
+    // copy-out of chunk c's y
+    if (!ck(cudaStreamWaitEvent(hp.s_out, hp.ev_comp[s], 0)) ||
+        !ck(copy_tokens_out(y, sb + hp.off_y, d, d.dim, eo, l0, len, hp.s_out)) ||
+        !ck(cudaEventRecord(hp.ev_out[s], hp.s_out)))
+      return SSM_ERR_CUDA;
+  }
+  if (h_last && !ck(cudaMemcpyAsync(h_last, hp.hbuf + ((nch - 1) % 2) * nstate, nstate * 4,
+                                    cudaMemcpyDeviceToHost, hp.s_out)))
+    return SSM_ERR_CUDA;
+  // the caller's stream waits for the last copies
+  if (!ck(cudaEventRecord(hp.ev_done, hp.s_out)) || !ck(cudaStreamWaitEvent(stream, hp.ev_done, 0)))
+    return SSM_ERR_CUDA;
+  return SSM_OK;
 }
 
 }  // extern "C"
