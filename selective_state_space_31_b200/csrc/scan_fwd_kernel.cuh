@@ -140,7 +140,9 @@ struct ItemPos {
     seg = vrow - row * p.M;
     seg_begin = seg * p.SPS;
     seg_end = min(p.S, seg_begin + p.SPS);
-    st_begin = seg_begin + part * p.PL;
+    // a segment shorter than the others (the last) can end before some of
+    // its parts begin: those parts are empty (st_begin == st_end)
+    st_begin = min(seg_end, seg_begin + part * p.PL);
     st_end = min(seg_end, st_begin + p.PL);
     b = row / p.nDT;
     dtile = row - b * p.nDT;
@@ -212,7 +214,7 @@ __global__ void __launch_bounds__((WARPS + 1) * 32, (OPT & 2) ? 5 : 0)
         } else {
           // next item when this one is done (parts past a short segment's end
           // have no stages and are skipped)
-          while (iss.item < 0 || st == iss.st_end) {
+          while (iss.item < 0 || st >= iss.st_end) {
             const int it = (int)atomicAdd(&p.ctl->ticket, 1u);
             if (it >= p.items) {
               state = 1;

@@ -229,3 +229,24 @@ def test_sixteen_segments():
     assert plan.status() == 0
     ry, rh = gu.run_oracle(inp)
     gu.assert_parity(gy, ry, gh, rh, gu.TOL["bf16"], str(info))
+
+
+@pytest.mark.parametrize("shape,segments", [((3, 2100, 512), 0), ((1, 4100, 128), 16),
+                                            ((2, 1100, 256), 4)])
+def test_parts_past_a_short_last_segment(shape, segments):
+    """Plans whose last segment is shorter than the others, so that some of
+    its parts begin past its end (14 segments of 5 one-stage parts over 66
+    stages: the last segment holds one stage): those parts are empty and
+    every stage is scanned once."""
+    inp = synth.make_fwd(*shape, 16, seed=76, has_h0=True)
+    plan = gu.make_plan(inp)
+    if segments:
+        plan.set_config(segments=segments, tile_t=32)
+    info = plan.info()
+    M, SPS, S = info["segments"], info["stages_per_segment"], info["stages_per_row"]
+    assert M >= 2 and S - (M - 1) * SPS < SPS, info
+    plan.set_debug(wait_timeout_ns=200_000_000)
+    gy, gh = gu.run_gpu(inp, plan)
+    assert plan.status() == 0
+    ry, rh = gu.run_oracle(inp)
+    gu.assert_parity(gy, ry, gh, rh, gu.TOL["bf16"], str(info))
