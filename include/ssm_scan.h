@@ -202,7 +202,8 @@ SSM_API ssm_status ssm_scan_fwd(ssm_scan_plan *plan, const void *x, const void *
  * plan share its staging memory: issue them on one stream (or synchronise
  * between them).
  * `chunk_tokens` is the number of tokens per chunk (0 = the library's
- * choice, about L/12 rounded up to a multiple of 64).  The first call (and a
+ * choice: about L/12, at least ~8 MB of copies per chunk, rounded up to a
+ * multiple of 64).  The first call (and a
  * call with another chunk length) allocates three chunk slots of device
  * staging memory and the plans for the chunk lengths; later calls reuse
  * them.  SSM_A_DIRECT and SSM_CONV_X plans are refused with

@@ -926,7 +926,12 @@ ssm_status ssm_scan_fwd_host(ssm_scan_plan *pl, const void *x, const void *delta
     if (h0) return map_cuda(cudaMemcpyAsync(h_last, h0, nstate * 4, cudaMemcpyHostToHost, stream));
     return map_cuda(cudaMemsetAsync(h_last, 0, nstate * 4, stream));
   }
-  int64_t Lc = chunk_tokens ? chunk_tokens : ((L + 11) / 12 + 63) / 64 * 64;
+  int64_t Lc = chunk_tokens;
+  if (!Lc) {  // about twelve chunks, none under ~8 MB of copies (below that, per-copy overheads rule)
+    const int64_t per_token = d.batch * (d.dim * (3 * (int64_t)ei + (int64_t)eo) + 2 * d.dstate * (int64_t)ei);
+    const int64_t min_tokens = ((int64_t)8 << 20) / std::max<int64_t>(per_token, 1) + 1;
+    Lc = (std::max((L + 11) / 12, min_tokens) + 63) / 64 * 64;
+  }
   Lc = std::min(Lc, L);
   if (!pl->pipe || pl->pipe->Lc != Lc) {
     host_pipe_free(pl->pipe);
