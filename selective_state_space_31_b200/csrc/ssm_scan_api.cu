@@ -943,58 +943,67 @@ ssm_status ssm_scan_fwd_host(ssm_scan_plan *pl, const void *x, const void *delta
   const int64_t nch = (L + Lc - 1) / Lc;
   float *dA = hp.params, *dD = hp.params + d.dim * d.dstate, *dbias = dD + d.dim;
   auto ck = [](cudaError_t e) { return e == cudaSuccess; };
-  // the copies start behind the caller's earlier work on `stream`
-  if (!ck(cudaEventRecord(hp.ev_start, stream)) || !ck(cudaStreamWaitEvent(hp.s_in, hp.ev_start, 0)) ||
-      !ck(cudaStreamWaitEvent(hp.s_out, hp.ev_start, 0)))
-    return SSM_ERR_CUDA;
-  // parameters once; the state before the first chunk into hbuf[1]
-  if (!ck(cudaMemcpyAsync(dA, A, (size_t)(d.dim * d.dstate) * 4, cudaMemcpyHostToDevice, hp.s_in)) ||
-      (D && !ck(cudaMemcpyAsync(dD, D, (size_t)d.dim * 4, cudaMemcpyHostToDevice, hp.s_in))) ||
-      (delta_bias &&
-       !ck(cudaMemcpyAsync(dbias, delta_bias, (size_t)d.dim * 4, cudaMemcpyHostToDevice, hp.s_in))))
-    return SSM_ERR_CUDA;
-  float *hprev0 = hp.hbuf + nstate;
-  if (!ck(h0 ? cudaMemcpyAsync(hprev0, h0, nstate * 4, cudaMemcpyHostToDevice, hp.s_in)
-             : cudaMemsetAsync(hprev0, 0, nstate * 4, hp.s_in)))
-    return SSM_ERR_CUDA;
-  for (int64_t c = 0; c < nch; ++c) {
-    const int s = (int)(c % kPipeSlots);
-    const int64_t l0 = c * Lc, len = std::min(Lc, L - l0);
-    unsigned char *sb = hp.slots + s * hp.slot_bytes;
-    // copy-in of chunk c once the scan of chunk c - kPipeSlots has left the slot
-    if (c >= kPipeSlots && !ck(cudaStreamWaitEvent(hp.s_in, hp.ev_comp[s], 0))) return SSM_ERR_CUDA;
-    if (!ck(copy_tokens_in(sb, x, d, d.dim, ei, l0, len, hp.s_in)) ||
-        !ck(copy_tokens_in(sb + hp.off_dt, delta, d, d.dim, ei, l0, len, hp.s_in)) ||
-        (z && !ck(copy_tokens_in(sb + hp.off_z, z, d, d.dim, ei, l0, len, hp.s_in))) ||
-        !ck(copy_tokens_in(sb + hp.off_B, B, d, d.dstate, ei, l0, len, hp.s_in)) ||
-        !ck(copy_tokens_in(sb + hp.off_C, C, d, d.dstate, ei, l0, len, hp.s_in)) ||
-        !ck(cudaEventRecord(hp.ev_in[s], hp.s_in)))
+  // everything is enqueued by `run`; whatever it returns, the caller's stream
+  // then waits for both copy streams, so no copy outlives the call's stream
+  // order (the host buffers may be released after a synchronisation)
+  auto run = [&]() -> ssm_status {
+    // the copies start behind the caller's earlier work on `stream`
+    if (!ck(cudaEventRecord(hp.ev_start, stream)) || !ck(cudaStreamWaitEvent(hp.s_in, hp.ev_start, 0)) ||
+        !ck(cudaStreamWaitEvent(hp.s_out, hp.ev_start, 0)))
       return SSM_ERR_CUDA;
-    // the scan of chunk c on the caller's stream, from the state chunk c - 1 left
-    if (!ck(cudaStreamWaitEvent(stream, hp.ev_in[s], 0)) ||
-        (c >= kPipeSlots && !ck(cudaStreamWaitEvent(stream, hp.ev_out[s], 0))))
+    // parameters once; the state before the first chunk into hbuf[1]
+    if (!ck(cudaMemcpyAsync(dA, A, (size_t)(d.dim * d.dstate) * 4, cudaMemcpyHostToDevice, hp.s_in)) ||
+        (D && !ck(cudaMemcpyAsync(dD, D, (size_t)d.dim * 4, cudaMemcpyHostToDevice, hp.s_in))) ||
+        (delta_bias &&
+         !ck(cudaMemcpyAsync(dbias, delta_bias, (size_t)d.dim * 4, cudaMemcpyHostToDevice, hp.s_in))))
       return SSM_ERR_CUDA;
-    float *hprev = hp.hbuf + ((c + 1) % 2) * nstate, *hnext = hp.hbuf + (c % 2) * nstate;
-    ssm_scan_plan *cp = len == Lc ? hp.body : hp.tail;
-    const ssm_status st =
-        ssm_scan_fwd(cp, sb, sb + hp.off_dt, delta_bias ? dbias : nullptr, dA, sb + hp.off_B,
-                     sb + hp.off_C, D ? dD : nullptr, z ? sb + hp.off_z : nullptr, hprev,
-                     sb + hp.off_y, hnext, stream_);
-    if (st != SSM_OK) return st;
-    if (!ck(cudaEventRecord(hp.ev_comp[s], stream))) return SSM_ERR_CUDA;
-    // copy-out of chunk c's y
-    if (!ck(cudaStreamWaitEvent(hp.s_out, hp.ev_comp[s], 0)) ||
-        !ck(copy_tokens_out(y, sb + hp.off_y, d, d.dim, eo, l0, len, hp.s_out)) ||
-        !ck(cudaEventRecord(hp.ev_out[s], hp.s_out)))
+    float *hprev0 = hp.hbuf + nstate;
+    if (!ck(h0 ? cudaMemcpyAsync(hprev0, h0, nstate * 4, cudaMemcpyHostToDevice, hp.s_in)
+               : cudaMemsetAsync(hprev0, 0, nstate * 4, hp.s_in)))
       return SSM_ERR_CUDA;
-  }
-  if (h_last && !ck(cudaMemcpyAsync(h_last, hp.hbuf + ((nch - 1) % 2) * nstate, nstate * 4,
-                                    cudaMemcpyDeviceToHost, hp.s_out)))
-    return SSM_ERR_CUDA;
-  // the caller's stream waits for the last copies
-  if (!ck(cudaEventRecord(hp.ev_done, hp.s_out)) || !ck(cudaStreamWaitEvent(stream, hp.ev_done, 0)))
-    return SSM_ERR_CUDA;
-  return SSM_OK;
+    for (int64_t c = 0; c < nch; ++c) {
+      const int s = (int)(c % kPipeSlots);
+      const int64_t l0 = c * Lc, len = std::min(Lc, L - l0);
+      unsigned char *sb = hp.slots + s * hp.slot_bytes;
+      // copy-in of chunk c once the scan of chunk c - kPipeSlots has left the slot
+      if (c >= kPipeSlots && !ck(cudaStreamWaitEvent(hp.s_in, hp.ev_comp[s], 0))) return SSM_ERR_CUDA;
+      if (!ck(copy_tokens_in(sb, x, d, d.dim, ei, l0, len, hp.s_in)) ||
+          !ck(copy_tokens_in(sb + hp.off_dt, delta, d, d.dim, ei, l0, len, hp.s_in)) ||
+          (z && !ck(copy_tokens_in(sb + hp.off_z, z, d, d.dim, ei, l0, len, hp.s_in))) ||
+          !ck(copy_tokens_in(sb + hp.off_B, B, d, d.dstate, ei, l0, len, hp.s_in)) ||
+          !ck(copy_tokens_in(sb + hp.off_C, C, d, d.dstate, ei, l0, len, hp.s_in)) ||
+          !ck(cudaEventRecord(hp.ev_in[s], hp.s_in)))
+        return SSM_ERR_CUDA;
+      // the scan of chunk c on the caller's stream, from the state chunk c - 1 left
+      if (!ck(cudaStreamWaitEvent(stream, hp.ev_in[s], 0)) ||
+          (c >= kPipeSlots && !ck(cudaStreamWaitEvent(stream, hp.ev_out[s], 0))))
+        return SSM_ERR_CUDA;
+      float *hprev = hp.hbuf + ((c + 1) % 2) * nstate, *hnext = hp.hbuf + (c % 2) * nstate;
+      ssm_scan_plan *cp = len == Lc ? hp.body : hp.tail;
+      const ssm_status st =
+          ssm_scan_fwd(cp, sb, sb + hp.off_dt, delta_bias ? dbias : nullptr, dA, sb + hp.off_B,
+                       sb + hp.off_C, D ? dD : nullptr, z ? sb + hp.off_z : nullptr, hprev,
+                       sb + hp.off_y, hnext, stream_);
+      if (st != SSM_OK) return st;
+      if (!ck(cudaEventRecord(hp.ev_comp[s], stream))) return SSM_ERR_CUDA;
+      // copy-out of chunk c's y
+      if (!ck(cudaStreamWaitEvent(hp.s_out, hp.ev_comp[s], 0)) ||
+          !ck(copy_tokens_out(y, sb + hp.off_y, d, d.dim, eo, l0, len, hp.s_out)) ||
+          !ck(cudaEventRecord(hp.ev_out[s], hp.s_out)))
+        return SSM_ERR_CUDA;
+    }
+    if (h_last && !ck(cudaMemcpyAsync(h_last, hp.hbuf + ((nch - 1) % 2) * nstate, nstate * 4,
+                                      cudaMemcpyDeviceToHost, hp.s_out)))
+      return SSM_ERR_CUDA;
+    return SSM_OK;
+  };
+  const ssm_status st = run();
+  const bool joined = ck(cudaEventRecord(hp.ev_done, hp.s_out)) &&
+                      ck(cudaStreamWaitEvent(stream, hp.ev_done, 0)) &&
+                      ck(cudaEventRecord(hp.ev_start, hp.s_in)) &&
+                      ck(cudaStreamWaitEvent(stream, hp.ev_start, 0));
+  if (st != SSM_OK) return st;
+  return joined ? SSM_OK : SSM_ERR_CUDA;
 }
 
 }  // extern "C"
