@@ -141,6 +141,7 @@ typedef struct {
   int bwd_warps_per_cta; /* scan warps of the fused backward kernel (0: ssm_scan_bwd
                             uses the general kernel for this problem) */
   int carry_chans_per_lane; /* channels per lane of the carry pass (segments > 1) */
+  int bwd_segments;    /* segments per row tile of the fused backward kernel (1 = none) */
 } ssm_scan_info;
 
 /* Optional overrides of the launch shape (0 = keep the default). */
@@ -162,6 +163,9 @@ typedef struct {
   int carry_loop;     /* carry pass: 1 + its variant options, as scan_loop (0 = free) */
   int bwd_warps_per_cta; /* fused backward kernel: 2 or 4 scan warps (0 = free) */
   int carry_chans_per_lane; /* carry pass: 1 or 2 channels per lane (0 = free) */
+  int bwd_segments;   /* fused backward kernel: segments per row tile, 1, 2, 4, 8 or 16
+                         (0 = free); with more than one, a map pass first computes each
+                         segment's forward and adjoint maps */
 } ssm_scan_config;
 /* Only the combinations compiled into the library exist; ssm_scan_set_config
  * returns SSM_ERR_UNSUPPORTED for others (ssm_scan_list_variants lists them). */

@@ -52,7 +52,8 @@ class Info(ctypes.Structure):
                 ("stages_per_segment", ctypes.c_int), ("carry_grid", ctypes.c_int),
                 ("launches_per_call", ctypes.c_int), ("scan_loop", ctypes.c_int),
                 ("carry_lanes_per_chan", ctypes.c_int), ("carry_loop", ctypes.c_int),
-                ("bwd_warps_per_cta", ctypes.c_int), ("carry_chans_per_lane", ctypes.c_int)]
+                ("bwd_warps_per_cta", ctypes.c_int), ("carry_chans_per_lane", ctypes.c_int),
+                ("bwd_segments", ctypes.c_int)]
 
     def as_dict(self):
         return {k: getattr(self, k) for k, _ in self._fields_}
@@ -64,7 +65,7 @@ class Config(ctypes.Structure):
                 ("chans_per_lane", ctypes.c_int), ("segments", ctypes.c_int),
                 ("scan_loop", ctypes.c_int), ("carry_lanes_per_chan", ctypes.c_int),
                 ("carry_loop", ctypes.c_int), ("bwd_warps_per_cta", ctypes.c_int),
-                ("carry_chans_per_lane", ctypes.c_int)]
+                ("carry_chans_per_lane", ctypes.c_int), ("bwd_segments", ctypes.c_int)]
 
 
 class Variant(ctypes.Structure):
@@ -211,10 +212,10 @@ class Plan:
 
     def set_config(self, lanes_per_chan=0, warps_per_cta=0, grid=0, tile_t=0,
                    chans_per_lane=0, segments=0, scan_loop=0, carry_lanes_per_chan=0,
-                   carry_loop=0, bwd_warps_per_cta=0, carry_chans_per_lane=0):
+                   carry_loop=0, bwd_warps_per_cta=0, carry_chans_per_lane=0, bwd_segments=0):
         c = Config(lanes_per_chan, warps_per_cta, grid, tile_t, chans_per_lane, segments,
                    scan_loop, carry_lanes_per_chan, carry_loop, bwd_warps_per_cta,
-                   carry_chans_per_lane)
+                   carry_chans_per_lane, bwd_segments)
         _check(self._lib.ssm_scan_set_config(self._h, ctypes.byref(c)), "ssm_scan_set_config")
 
     def set_debug(self, wait_timeout_ns=0, drop_unit=-1):

@@ -104,7 +104,29 @@ __device__ __forceinline__ float sigmoid_f(float v) {
   return rcp_approx(1.f + ex2_approx(-v * kLog2e));
 }
 
-template <typename InT, typename GT, int NS, int LPC, int W>
+// Work item i: row tile i / M, segment i % M over stages [st_lo, st_hi);
+// n1 forward steps (phase 1), then n2 reverse steps (phase 2).  The map pass
+// walks a segment forward only if a later segment needs its forward map and
+// backwards only if an earlier one needs its adjoint map.
+struct BwdItem {
+  int row, seg, st_lo, st_hi, n1, n2;
+  __device__ __forceinline__ void set(int i, const BwdTmaParams &p, bool maps) {
+    row = i / p.M;
+    seg = i - row * p.M;
+    st_lo = min(p.S, seg * p.SPS);
+    st_hi = min(p.S, st_lo + p.SPS);
+    const int n = st_hi - st_lo;
+    n1 = maps ? (seg < p.M - 1 ? n : 0) : n;
+    n2 = maps ? (seg > 0 ? n : 0) : n;
+  }
+};
+
+// MAPS = false: the backward pass over each item (phase 1 from the segment's
+// start state, phase 2 from the gradient flowing in from the later
+// segments).  MAPS = true (segmented plans, launched first): per item the
+// forward map (state reached from 0, sum of Delta) and the adjoint map
+// (dL/dh carried from 0 backwards across the segment, sum of Delta).
+template <typename InT, typename GT, int NS, int LPC, int W, bool MAPS>
 __global__ void __launch_bounds__((W + 1) * 32, W == 4 ? 3 : 5)
     bwd_tma_kernel(const __grid_constant__ BwdMaps maps, const BwdTmaParams p) {
   using Cfg = BwdCfg<InT, GT, NS, LPC, W>;
@@ -130,8 +152,7 @@ __global__ void __launch_bounds__((W + 1) * 32, W == 4 ? 3 : 5)
   __syncthreads();
 
   const int S = p.S;
-  const int my_rows = blockIdx.x < p.rows ? (p.rows - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-  const int nsteps = my_rows * 2 * S;  // per row: phase 1 stages 0..S-1, phase 2 S-1..0
+  const int items = p.rows * p.M;
 
   if (warp == W) {
     // ===================== load warp =====================
@@ -150,45 +171,48 @@ __global__ void __launch_bounds__((W + 1) * 32, W == 4 ? 3 : 5)
       mbar_arrive(&rconv[r]);
       return true;
     };
-    int issued = 0;
+    int issued = 0, k = 0;
     bool ok = true;
-    for (int k = 0; k < nsteps; ++k) {
-      const int r = k % RAW;
-      if (lane == 0) {
-        const int row = blockIdx.x + (k / (2 * S)) * gridDim.x;
-        const int step = k % (2 * S);
-        const bool ph2 = step >= S;
-        const int st = ph2 ? 2 * S - 1 - step : step;
-        if (k >= RAW &&
-            !wait_or_abort(&rempty[r], (uint32_t)(((k / RAW) - 1) & 1), abort, p.timeout_ns)) {
-          ok = false;
-        } else {
-          const int b = row / p.nDT, d0 = (row - b * p.nDT) * DT, t0 = st * TT;
-          const uint32_t tx = 2u * XB + BB + (ph2 ? (p.has_z ? XB : 0u) + YB + BB : 0u);
-          unsigned char *sb = smem + r * Cfg::SLOT;
-          mbar_arrive_expect_tx(&rfull[r], tx);
-          tma_load_3d(sb, &maps.x, &rfull[r], d0, t0, b);
-          tma_load_3d(sb + Cfg::OFF_DT, &maps.dt, &rfull[r], d0, t0, b);
-          tma_load_3d(sb + Cfg::OFF_B, &maps.B, &rfull[r], 0, t0, b);
-          if (ph2) {
-            if (p.has_z) tma_load_3d(sb + Cfg::OFF_Z, &maps.z, &rfull[r], d0, t0, b);
-            tma_load_3d(sb + Cfg::OFF_DY, &maps.dy, &rfull[r], d0, t0, b);
-            tma_load_3d(sb + Cfg::OFF_C, &maps.C, &rfull[r], 0, t0, b);
+    for (int it = blockIdx.x; it < items && ok; it += gridDim.x) {
+      BwdItem I;
+      I.set(it, p, MAPS);
+      const int b = I.row / p.nDT, d0 = (I.row - b * p.nDT) * DT;
+      for (int j = 0; j < I.n1 + I.n2; ++j, ++k) {
+        const int r = k % RAW;
+        const bool ph2 = j >= I.n1;
+        const int st = ph2 ? I.st_hi - 1 - (j - I.n1) : I.st_lo + j;
+        if (lane == 0) {
+          if (k >= RAW &&
+              !wait_or_abort(&rempty[r], (uint32_t)(((k / RAW) - 1) & 1), abort, p.timeout_ns)) {
+            ok = false;
+          } else {
+            const int t0 = st * TT;
+            const uint32_t tx = 2u * XB + BB + (ph2 ? (p.has_z ? XB : 0u) + YB + BB : 0u);
+            unsigned char *sb = smem + r * Cfg::SLOT;
+            mbar_arrive_expect_tx(&rfull[r], tx);
+            tma_load_3d(sb, &maps.x, &rfull[r], d0, t0, b);
+            tma_load_3d(sb + Cfg::OFF_DT, &maps.dt, &rfull[r], d0, t0, b);
+            tma_load_3d(sb + Cfg::OFF_B, &maps.B, &rfull[r], 0, t0, b);
+            if (ph2) {
+              if (p.has_z) tma_load_3d(sb + Cfg::OFF_Z, &maps.z, &rfull[r], d0, t0, b);
+              tma_load_3d(sb + Cfg::OFF_DY, &maps.dy, &rfull[r], d0, t0, b);
+              tma_load_3d(sb + Cfg::OFF_C, &maps.C, &rfull[r], 0, t0, b);
+            }
+            issued = k + 1;
           }
-          issued = k + 1;
         }
-      }
-      ok = __shfl_sync(FULL_MASK, ok, 0);
-      if (!ok) break;
-      if constexpr (WIDEN) {  // the previous step's slot, while this one is in flight
-        if (k > 0 && !widen(k - 1)) {
-          ok = false;
-          break;
+        ok = __shfl_sync(FULL_MASK, ok, 0);
+        if (!ok) break;
+        if constexpr (WIDEN) {  // the previous step's slot, while this one is in flight
+          if (k > 0 && !widen(k - 1)) {
+            ok = false;
+            break;
+          }
         }
       }
     }
     if constexpr (WIDEN) {
-      if (ok && nsteps > 0) ok = widen(nsteps - 1);
+      if (ok && k > 0) ok = widen(k - 1);
     }
     if (!ok && lane == 0) {
       *abort = 1;
@@ -225,7 +249,10 @@ __global__ void __launch_bounds__((W + 1) * 32, W == 4 ? 3 : 5)
     return __all_sync(FULL_MASK, got);
   };
 
-  for (int row = blockIdx.x; row < p.rows; row += gridDim.x) {
+  for (int it = blockIdx.x; it < items; it += gridDim.x) {
+    BwdItem I;
+    I.set(it, p, MAPS);
+    const int row = I.row;
     const int b = row / p.nDT, dtile = row - b * p.nDT;
     const int d = dtile * DT + grp;
     const bool valid = d < p.D;
@@ -234,14 +261,35 @@ __global__ void __launch_bounds__((W + 1) * 32, W == 4 ? 3 : 5)
     for (int i = 0; i < NPL; ++i) {
       An[i] = valid ? __ldg(p.A + (size_t)d * NS + q * NPL + i) : 0.f;
       A2[i] = An[i] * kLog2e;
-      h[i] = (valid && p.has_h0) ? __ldg(p.h0 + ((size_t)b * p.D + d) * NS + q * NPL + i) : 0.f;
+      h[i] = (!MAPS && valid && p.has_h0)
+                 ? __ldg(p.h0 + ((size_t)b * p.D + d) * NS + q * NPL + i) : 0.f;
     }
     const float bias = (valid && p.has_bias) ? __ldg(p.bias + d) : 0.f;
     const float Dd = (valid && p.has_D) ? __ldg(p.Dv + d) : 0.f;
     float *ckrow = p.ws_ck + (size_t)row * S * DT * NS + (size_t)grp * NS + q * NPL;
+    // this channel's maps of (row, segment j): N states, then the sum of Delta
+    // (a stride of N + 4 floats keeps every map 16-byte aligned)
+    auto map_at = [&](float *base, int j) {
+      return base + ((size_t)(row * p.M + j) * DT + grp) * (NS + 4);
+    };
+    if constexpr (!MAPS) {
+      // the segment's start state: h0 carried through the forward maps of the
+      // segments before it, h <- exp(A sum Delta) h + h_from_0
+      for (int j = 0; j < I.seg; ++j) {
+        const float *m = map_at(p.ws_fmap, j);
+        const float sj = __ldcg(m + NS);
+#pragma unroll
+        for (int i = 0; i < NPL; ++i)
+          h[i] = fmaf(ex2_approx(A2[i] * sj), h[i], __ldcg(m + q * NPL + i));
+      }
+    }
+    float hstart[NPL];
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) hstart[i] = h[i];
+    float dsum = 0.f;  // sum of Delta over the segment (map pass)
 
     // ---------------- phase 1: forward, stage-start states ----------------
-    for (int st = 0; st < S; ++st, ++k) {
+    for (int st = I.st_lo; st < I.st_lo + I.n1; ++st, ++k) {
       ok = ok && wait_slot(k);
       if (ok) {
         const unsigned char *sb = smem + (k % RAW) * Cfg::SLOT;
@@ -261,6 +309,7 @@ __global__ void __launch_bounds__((W + 1) * 32, W == 4 ? 3 : 5)
 #pragma unroll
         for (int t = 0; t < TT; ++t) {
           const float2 pl = *reinterpret_cast<const float2 *>(plane + t);
+          if constexpr (MAPS) dsum += pl.x;
           float bv[NPL];
           load_bc<NPL>(Bs + t * NS + q * NPL, bv);
 #pragma unroll
@@ -275,9 +324,16 @@ __global__ void __launch_bounds__((W + 1) * 32, W == 4 ? 3 : 5)
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&rempty[k % RAW]);
-        if (st + 1 < S)
+        if (!MAPS && st + 1 < I.st_hi)
           *reinterpret_cast<float4 *>(ckrow + (size_t)(st + 1) * DT * NS) =
               make_float4(h[0], h[1], h[2], h[3]);
+      }
+    }
+    if constexpr (MAPS) {
+      if (ok && I.n1 > 0) {  // forward map of this segment
+        float *m = map_at(p.ws_fmap, I.seg);
+        *reinterpret_cast<float4 *>(m + q * NPL) = make_float4(h[0], h[1], h[2], h[3]);
+        if (q == 0) m[NS] = dsum;
       }
     }
 
@@ -285,23 +341,88 @@ __global__ void __launch_bounds__((W + 1) * 32, W == 4 ? 3 : 5)
     float lam[NPL], dA[NPL];
 #pragma unroll
     for (int i = 0; i < NPL; ++i) {
-      lam[i] = (valid && p.dh_last)
+      lam[i] = (!MAPS && valid && p.dh_last)
                    ? __ldg(p.dh_last + ((size_t)b * p.D + d) * NS + q * NPL + i) : 0.f;
       dA[i] = 0.f;
     }
+    if constexpr (MAPS) {
+      // adjoint map: dL/dh from 0 at the segment's end, carried back across
+      // it (lam += ds C_t; lam <- lam Abar_t), and the sum of Delta
+      dsum = 0.f;
+      for (int st = I.st_hi - 1; st >= I.st_hi - I.n2; --st, ++k) {
+        ok = ok && wait_slot(k);
+        if (!ok) continue;
+        const unsigned char *sb = smem + (k % RAW) * Cfg::SLOT;
+        const InT *ds = reinterpret_cast<const InT *>(sb + Cfg::OFF_DT);
+        const InT *zs = reinterpret_cast<const InT *>(sb + Cfg::OFF_Z);
+        const GT *dys = reinterpret_cast<const GT *>(sb + Cfg::OFF_DY);
+        const BCT *Cs = reinterpret_cast<const BCT *>(sb + (WIDEN ? Cfg::OFF_CF : Cfg::OFF_C));
+        const int nvalid = min(TT, p.L - st * TT);
+#pragma unroll
+        for (int j = 0; j < TPL; ++j) {
+          const int ta = j * LPC + q;
+          const float v = to_f32(ds[ta * DT + grp]) + bias;
+          float dl = p.softplus ? softplus_f(v) : v;
+          float dsv = to_f32(dys[ta * DT + grp]);
+          if (p.has_z) {
+            const float zv = to_f32(zs[ta * DT + grp]);
+            dsv *= zv * sigmoid_f(zv);
+          }
+          if (ta >= nvalid) {
+            dl = 0.f;
+            dsv = 0.f;
+          }
+          *reinterpret_cast<float2 *>(plane + ta) = make_float2(dl, dsv);
+        }
+        __syncwarp();
+#pragma unroll
+        for (int t = TT - 1; t >= 0; --t) {
+          const float2 pl = *reinterpret_cast<const float2 *>(plane + t);  // (Delta, ds)
+          dsum += pl.x;
+          float cv[NPL];
+          load_bc<NPL>(Cs + t * NS + q * NPL, cv);
+#pragma unroll
+          for (int i = 0; i < NPL; i += 2) {
+            const float2 arg = fmul2(make_float2(pl.x, pl.x), make_float2(A2[i], A2[i + 1]));
+            float2 lm = ffma2(make_float2(pl.y, pl.y), make_float2(cv[i], cv[i + 1]),
+                              make_float2(lam[i], lam[i + 1]));
+            lm = fmul2(lm, make_float2(ex2_approx(arg.x), ex2_approx(arg.y)));
+            lam[i] = lm.x;
+            lam[i + 1] = lm.y;
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&rempty[k % RAW]);
+      }
+      if (ok && I.n2 > 0) {
+        float *m = map_at(p.ws_amap, I.seg);
+        *reinterpret_cast<float4 *>(m + q * NPL) = make_float4(lam[0], lam[1], lam[2], lam[3]);
+        if (q == 0) m[NS] = dsum;
+      }
+      continue;
+    } else {
+      // the gradient flowing in from the later segments: dL/dh_last carried
+      // back through their adjoint maps, lam <- exp(A sum Delta) lam + e
+      for (int j = p.M - 1; j > I.seg; --j) {
+        const float *m = map_at(p.ws_amap, j);
+        const float sj = __ldcg(m + NS);
+#pragma unroll
+        for (int i = 0; i < NPL; ++i)
+          lam[i] = fmaf(ex2_approx(A2[i] * sj), lam[i], __ldcg(m + q * NPL + i));
+      }
+    }
     float dD_acc = 0.f, dbias_acc = 0.f;
-    for (int st = S - 1; st >= 0; --st, ++k) {
+    for (int st = I.st_hi - 1; st >= I.st_hi - I.n2; --st, ++k) {
       const int par = st & 1;
       float *slice = reinterpret_cast<float *>(smem + Cfg::OFF_SL) + (par * W + warp) * TT * 2 * NS;
       const int t0 = st * TT;
       const int nvalid = min(TT, p.L - t0);
-      // the stage's start state (this lane wrote it in phase 1)
+      // the stage's start state (the segment's start, or what this lane wrote
+      // in phase 1)
       float hs[TT + 1][NPL];
-      if (st == 0) {
+      if (st == I.st_lo) {
 #pragma unroll
-        for (int i = 0; i < NPL; ++i)
-          hs[0][i] = (valid && p.has_h0)
-                         ? __ldg(p.h0 + ((size_t)b * p.D + d) * NS + q * NPL + i) : 0.f;
+        for (int i = 0; i < NPL; ++i) hs[0][i] = hstart[i];
       } else {
         const float4 c = *reinterpret_cast<const float4 *>(ckrow + (size_t)st * DT * NS);
         hs[0][0] = c.x; hs[0][1] = c.y; hs[0][2] = c.z; hs[0][3] = c.w;
@@ -463,7 +584,7 @@ __global__ void __launch_bounds__((W + 1) * 32, W == 4 ? 3 : 5)
     if (!ok) continue;  // (every remaining step gives up at once: the CTA's abort flag)
     // ---------------- per-row results ----------------
     if (valid) {
-      if (p.dh0) {
+      if (p.dh0 && I.seg == 0) {
         *reinterpret_cast<float4 *>(p.dh0 + ((size_t)b * p.D + d) * NS + q * NPL) =
             make_float4(lam[0], lam[1], lam[2], lam[3]);
       }
@@ -508,15 +629,23 @@ template <typename InT, typename GT, int NS, int LPC, int W>
 cudaError_t run_bwd(const BwdShape &s, const BwdMaps &maps, const BwdTmaParams &p,
                     cudaStream_t stream, BwdShape *query) {
   using Cfg = BwdCfg<InT, GT, NS, LPC, W>;
-  auto kern = bwd_tma_kernel<InT, GT, NS, LPC, W>;
+  auto kern = bwd_tma_kernel<InT, GT, NS, LPC, W, false>;
+  auto kmap = bwd_tma_kernel<InT, GT, NS, LPC, W, true>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(kmap, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
   if (e != cudaSuccess) return e;
   if (query) {  // what the variant needs and gets on the device
     query->smem = Cfg::SMEM;
     return cudaOccupancyMaxActiveBlocksPerMultiprocessor(&query->occ, kern, Cfg::THREADS,
                                                          Cfg::SMEM);
   }
-  kern<<<(unsigned)s.rows, Cfg::THREADS, Cfg::SMEM, stream>>>(maps, p);
+  const unsigned grid = (unsigned)(s.rows * s.M);  // one CTA per (row tile, segment)
+  if (s.M > 1) {  // the segments' maps first
+    kmap<<<grid, Cfg::THREADS, Cfg::SMEM, stream>>>(maps, p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  kern<<<grid, Cfg::THREADS, Cfg::SMEM, stream>>>(maps, p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const long long total = (long long)p.Bsz * p.L * (2 * NS / 4);
   if (total > 0)
@@ -554,20 +683,27 @@ cudaError_t bwd_dispatch(int in_dtype, int out_dtype, const BwdShape &s, const B
 
 }  // namespace
 
-// Two or four scan warps: whichever fills the resident CTA slots of the
-// device best over its whole number of waves (every CTA runs one row tile
-// over the whole sequence, so a last partial wave leaves SMs idle); ties go
-// to four (fewer load warps).
+// Scan warps (2 or 4) and segments per row tile (1, 2, 4, 8, 16): each
+// CTA walks one (row tile, segment) item, so the score is how well the items
+// fill whole waves of resident CTAs, divided by the map pass's extra work
+// for segments (about two more exponentials per update on (M-1)/M of the
+// tokens, against the backward's 3.5: weight kBwdSegCost); ties go to fewer
+// segments and then to four warps.
+constexpr double kBwdSegCost = 0.8;
+
 bool choose_bwd_shape(int in_dtype, int out_dtype, int64_t batch, int64_t seqlen, int64_t dim,
-                      int ns, int warps, int sms, BwdShape *out) {
+                      int ns, int warps, int segments, int sms, BwdShape *out) {
   if (ns != 16 && ns != 8) return false;
   if (warps != 0 && warps != 2 && warps != 4) return false;
+  if (segments != 0 && segments != 1 && segments != 2 && segments != 4 && segments != 8 &&
+      segments != 16)
+    return false;
   if (batch <= 0 || seqlen <= 0 || dim <= 0) return false;
   const int es = in_dtype == 1 ? 2 : 4, gs = out_dtype == 1 ? 2 : 4;
   if (in_dtype == 0 && out_dtype == 1) return false;  // no such variant
   if ((dim * es) % 16 != 0 || (dim * gs) % 16 != 0 || (ns * es) % 16 != 0) return false;
   bool found = false;
-  double best_fill = -1.0;
+  double best_score = -1.0;
   BwdShape best;
   for (int w : {4, 2}) {
     if (warps && w != warps) continue;
@@ -578,24 +714,35 @@ bool choose_bwd_shape(int in_dtype, int out_dtype, int64_t batch, int64_t seqlen
     s.nDT = (int)((dim + s.DT - 1) / s.DT);
     s.rows = batch * s.nDT;
     s.S = (int)((seqlen + kBwdStage - 1) / kBwdStage);
-    if (s.rows > INT32_MAX || s.rows * (int64_t)s.S > INT32_MAX / 2) continue;
-    s.ws_ck_floats = (size_t)s.rows * s.S * s.DT * ns;
-    s.ws_bc_floats = (size_t)s.rows * seqlen * 2 * ns;
     if (bwd_dispatch(in_dtype, out_dtype, s, nullptr, nullptr, nullptr, &s) != cudaSuccess ||
         s.occ < 1) {
       cudaGetLastError();
       continue;
     }
     const int64_t slots = (int64_t)s.occ * sms;
-    const double fill = (double)s.rows / (double)(((s.rows + slots - 1) / slots) * slots);
-    if (!found || fill > best_fill + 1e-9) {
-      found = true;
-      best_fill = fill;
-      best = s;
+    for (int M : {1, 2, 4, 8, 16}) {
+      if (segments && M != segments) continue;
+      if (M > 1 && s.S < 4 * M) continue;  // each segment keeps a few stages
+      BwdShape c = s;
+      c.SPS = (s.S + M - 1) / M;
+      c.M = (s.S + c.SPS - 1) / c.SPS;
+      const int64_t units = c.rows * c.M;
+      if (units > INT32_MAX || c.rows * (int64_t)c.S > INT32_MAX / 2) continue;
+      const double fill = (double)units / (double)(((units + slots - 1) / slots) * slots);
+      const double score = fill / (1.0 + kBwdSegCost * (c.M - 1) / c.M) - 1e-4 * c.M;
+      if (!found || score > best_score + 1e-9) {
+        found = true;
+        best_score = score;
+        best = c;
+      }
     }
   }
-  if (found) *out = best;
-  return found;
+  if (!found) return false;
+  best.ws_ck_floats = (size_t)best.rows * best.S * best.DT * ns;
+  best.ws_bc_floats = (size_t)best.rows * seqlen * 2 * ns;
+  best.ws_map_floats = best.M > 1 ? (size_t)best.rows * best.M * best.DT * (ns + 4) : 0;
+  *out = best;
+  return true;
 }
 
 cudaError_t launch_bwd_tma(int in_dtype, int out_dtype, const BwdShape &s, const BwdMaps &maps,

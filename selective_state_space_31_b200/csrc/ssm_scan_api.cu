@@ -347,9 +347,11 @@ ssm_status ssm_scan_get_info(const ssm_scan_plan *pl, ssm_scan_info *info) {
   info->bwd_warps_per_cta =
       pl->path == PATH_TMA &&
               ssm::choose_bwd_shape((int)d.in_dtype, (int)d.out_dtype, d.batch, d.seqlen, d.dim,
-                                    (int)d.dstate, pl->cfg.bwd_warps_per_cta, pl->num_sms, &bs)
+                                    (int)d.dstate, pl->cfg.bwd_warps_per_cta,
+                                    pl->cfg.bwd_segments, pl->num_sms, &bs)
           ? bs.warps
           : 0;
+  info->bwd_segments = info->bwd_warps_per_cta ? bs.M : 0;
   info->workspace_bytes =
       pl->ws_state_bytes + pl->ws_flag_bytes + pl->ws_agg_bytes + sizeof(ssm::Control);
   return SSM_OK;
@@ -361,6 +363,8 @@ ssm_status ssm_scan_set_config(ssm_scan_plan *pl, const ssm_scan_config *cfg) {
       cfg->chans_per_lane < 0 || cfg->segments < 0 || cfg->scan_loop < 0 || cfg->scan_loop > 16 ||
       cfg->carry_lanes_per_chan < 0 || cfg->carry_loop < 0 || cfg->carry_loop > 16 ||
       (cfg->bwd_warps_per_cta != 0 && cfg->bwd_warps_per_cta != 2 && cfg->bwd_warps_per_cta != 4) ||
+      (cfg->bwd_segments != 0 && cfg->bwd_segments != 1 && cfg->bwd_segments != 2 &&
+       cfg->bwd_segments != 4 && cfg->bwd_segments != 8 && cfg->bwd_segments != 16) ||
       cfg->carry_chans_per_lane < 0 || cfg->carry_chans_per_lane > 2)
     return SSM_ERR_INVALID_ARG;
   DeviceGuard guard(pl->device);
@@ -679,12 +683,12 @@ ssm_status ssm_scan_bwd(ssm_scan_plan *pl, const void *x, const void *delta,
   const bool fused = has_tokens && pl->path == PATH_TMA &&
                      ssm::choose_bwd_shape((int)d.in_dtype, (int)d.out_dtype, d.batch, d.seqlen,
                                            d.dim, (int)d.dstate, pl->cfg.bwd_warps_per_cta,
-                                           pl->num_sms, &bs) &&
+                                           pl->cfg.bwd_segments, pl->num_sms, &bs) &&
                      aligned16(x) && aligned16(delta) && aligned16(z) && aligned16(B) &&
                      aligned16(C) && aligned16(dy) && aligned16(dB) && aligned16(dC) &&
                      aligned16(dh0);
   if (fused) {
-    const size_t need = (bs.ws_ck_floats + bs.ws_bc_floats) * sizeof(float);
+    const size_t need = (bs.ws_ck_floats + bs.ws_bc_floats + 2 * bs.ws_map_floats) * sizeof(float);
     if (need > pl->ws_ck_bytes) {
       if (pl->ws_ck) cudaFree(pl->ws_ck);
       pl->ws_ck = nullptr;
@@ -708,6 +712,7 @@ ssm_status ssm_scan_bwd(ssm_scan_plan *pl, const void *x, const void *delta,
     ssm::BwdTmaParams p{};
     p.Bsz = (int)d.batch; p.L = (int)d.seqlen; p.D = (int)d.dim; p.N = (int)d.dstate;
     p.DT = bs.DT; p.nDT = bs.nDT; p.S = bs.S; p.rows = (int)bs.rows;
+    p.M = bs.M; p.SPS = bs.SPS;
     p.softplus = f & SSM_DELTA_SOFTPLUS;
     p.has_z = f & SSM_HAS_Z;
     p.has_D = f & SSM_HAS_D;
@@ -718,6 +723,8 @@ ssm_status ssm_scan_bwd(ssm_scan_plan *pl, const void *x, const void *delta,
     p.dbias = ddelta_bias; p.dh0 = dh0;
     p.ws_ck = pl->ws_ck;
     p.ws_bc = pl->ws_ck + bs.ws_ck_floats;
+    p.ws_fmap = bs.M > 1 ? p.ws_bc + bs.ws_bc_floats : nullptr;
+    p.ws_amap = bs.M > 1 ? p.ws_fmap + bs.ws_map_floats : nullptr;
     p.ctl = pl->ctl;
     p.timeout_ns = pl->timeout_ns;
     return map_cuda(ssm::launch_bwd_tma((int)d.in_dtype, (int)d.out_dtype, bs, maps, p, stream));

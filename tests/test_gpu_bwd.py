@@ -244,3 +244,28 @@ def test_bwd_130m_layer_every_channel():
     for k, ref in acc.items():
         e = gu.normwise(got[k], ref)
         assert e <= 1e-3, f"d/d{k}: normwise {e:.2e}"
+
+
+@pytest.mark.parametrize("segments", [2, 4, 16])
+@pytest.mark.parametrize("in_dt", ["f32", "bf16"])
+def test_bwd_fused_segments(segments, in_dt):
+    """Segments of a row tile walked at the same time: the map pass's
+    forward maps give each segment its start state, its adjoint maps the
+    gradient flowing in from the later segments; ragged L (the last 8-token
+    stage holds 3 tokens, the last segment is short), every option."""
+    inp = synth.make_fwd(2, 603, 64, 16, in_dtype=in_dt, seed=67 + segments, has_h0=True)
+    plan = gu.make_plan(inp)
+    plan.set_config(bwd_segments=segments)
+    info = plan.info()
+    assert info["bwd_segments"] >= 2, info
+    plan.close()
+    _check(inp, seed=16 + segments, cfg=dict(bwd_segments=segments))
+
+
+def test_bwd_long_row_picks_segments():
+    """One long row (few row tiles): the planner splits it into segments."""
+    inp = synth.make_fwd(1, 4000, 64, 16, in_dtype="f32", seed=69, has_h0=True)
+    plan = gu.make_plan(inp)
+    assert plan.info()["bwd_segments"] > 1, plan.info()
+    plan.close()
+    _check(inp, seed=17)
