@@ -541,8 +541,9 @@ def run_fwd(name, steps, warmup, args, rank, world, device, peaks, e2e_steps,
         peak_mufu, basis = nominal_mufu, "16 MUFU results/clk/SM x 148 SMs x 1965 MHz (nominal)"
     traffic = None if args.bwd else profiled_traffic(name)
     launches_per_call = int(info.get("launches_per_call", 1) or 1)
-    if args.bwd:  # fused backward: the kernel and the row-tile sum of dB / dC
-        launches_per_call = 2 if info.get("bwd_warps_per_cta") else 1
+    if args.bwd:  # fused backward: (the map pass,) the kernel and the row-tile sum of dB / dC
+        launches_per_call = ((3 if info.get("bwd_segments", 1) > 1 else 2)
+                             if info.get("bwd_warps_per_cta") else 1)
 
     result = {
         "metric": METRIC,
@@ -563,7 +564,7 @@ def run_fwd(name, steps, warmup, args, rank, world, device, peaks, e2e_steps,
                                         "parts_per_row", "segments", "stages_per_segment",
                                         "carry_grid", "launches_per_call", "scan_loop",
                                         "carry_lanes_per_chan", "carry_loop",
-                                        "bwd_warps_per_cta") if k in info},
+                                        "bwd_warps_per_cta", "bwd_segments") if k in info},
         "roofline": {"bound": "alu", "achieved": achieved_mufu / 1e9, "peak": peak_mufu / 1e9,
                      "unit": "G MUFU-op/s (ex2, lg2, rcp)", "frac": achieved_mufu / peak_mufu,
                      "traffic": traffic, "peak_basis": basis,
