@@ -142,3 +142,21 @@ def test_decode_1024_steps_every_channel():
     gs = state.cpu().numpy()
     assert np.all(np.isfinite(gs))
     assert gu.normwise(gs, ostate) <= 1e-5, gu.normwise(gs, ostate)
+
+
+@pytest.mark.parametrize("name", ["mamba130m_layer", "long_seq"])
+def test_host_buffer_path_every_row(name):
+    """The workload through ssm_scan_fwd_host (pinned host buffers, the
+    library's chunking) at full size, every (b, d) row against the oracle."""
+    inp = synth.FWD_WORKLOADS[name]()
+    plan = gu.make_plan(inp)
+    idt = gu.TDT[inp.in_dtype]
+    pin = lambda a, dt: None if a is None else torch.from_numpy(np.ascontiguousarray(a)).to(dt).pin_memory()
+    y, hl = plan.fwd_host(pin(inp.x, idt), pin(inp.delta, idt), pin(inp.A, torch.float32),
+                          pin(inp.B, idt), pin(inp.C, idt), D=pin(inp.Dskip, torch.float32),
+                          z=pin(inp.z, idt), delta_bias=pin(inp.delta_bias, torch.float32),
+                          h0=pin(inp.h0, torch.float32))
+    torch.cuda.synchronize()
+    assert plan.status() == 0
+    plan.close()
+    check_every_row(inp, y.float().numpy(), hl.numpy(), gu.TOL["bf16"], f"{name} host path")
