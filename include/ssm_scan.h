@@ -275,11 +275,18 @@ SSM_API ssm_status ssm_scan_fold_maps(ssm_scan_plan *plan, int count, const floa
  * (batch, dim, dstate).  dz, dD, ddelta_bias must be non-NULL exactly when
  * SSM_HAS_Z, SSM_HAS_D, SSM_HAS_DELTA_BIAS are set; dh0 may be NULL.  The
  * accumulated gradients (dB, dC, dA, dD, ddelta_bias) are overwritten, not
- * added to.  States are recomputed from per-chunk checkpoints rather than
- * stored ("Tai sao chi parallel scan van chua du nhanh?"); the first call on
- * a plan allocates the checkpoint workspace (batch*dim*ceil(seqlen/16)*dstate
- * floats) and may return SSM_ERR_OOM.  Summation order of dB, dC, dA, dD and
- * ddelta_bias follows atomics, so those are reproducible to rounding only. */
+ * added to.  States are recomputed from per-stage checkpoints rather than
+ * stored ("Tai sao chi parallel scan van chua du nhanh?").  The first call on
+ * a plan allocates the workspace — for the fused kernel (dstate 8 or 16,
+ * TMA-aligned shapes) the stage-start states (about batch*dim*seqlen*dstate/8
+ * floats), per-row-tile dB/dC sums (about batch*seqlen*2*dstate floats per 32
+ * channels) and, for a segmented plan, the segments' maps; for the general
+ * kernel batch*dim*ceil(seqlen/16)*dstate floats — and may return
+ * SSM_ERR_OOM; later calls reuse it.  dB and dC are added in a fixed order
+ * (reproducible bit for bit) on the fused path; dA, dD and ddelta_bias (and
+ * dB, dC on the general path) follow atomics, reproducible to rounding only.
+ * ssm_scan_set_config's bwd_warps_per_cta and bwd_segments choose the fused
+ * kernel's shape; ssm_scan_get_info reports it. */
 SSM_API ssm_status ssm_scan_bwd(ssm_scan_plan *plan, const void *x, const void *delta,
                         const float *delta_bias, const float *A, const void *B,
                         const void *C, const float *D, const void *z, const float *h0,
