@@ -652,20 +652,27 @@ def run_decode(steps, warmup, args, rank, world, device, e2e_steps, want_cpu=Tru
     byt = 8 * Bz * Dm * N + 3 * 2 * Bz * Dm + 2 * 2 * Bz * N + 2 * Bz * Dm + 4 * Dm * N + 8 * Dm
     hbm_peak, hbm_basis = measured_hbm_peak()
     gbs = byt / (ms_per_step * 1e-3) / 1e9
-    # e2e: a token's inputs come from pinned host memory, y goes back
+    # e2e through the C-ABI host-buffer step: a token's inputs come from
+    # pinned host memory and y goes back, the state stays on the device
     host = [{k: v.to(bf).cpu().pin_memory() for k, v in t.items()} for t in tin[:4]]
     y_h = torch.empty((Bz, Dm), dtype=bf).pin_memory()
     h2d = sum(v.numel() * v.element_size() for v in host[0].values())
     d2h = y_h.numel() * y_h.element_size()
     s0 = torch.cuda.current_stream(device)
+
+    def e2e_step(i):
+        t = host[i % 4]
+        plan.step_host(states[0], t["x"], t["delta"], A, t["B"], t["C"], D=D, z=t["z"],
+                       delta_bias=bias, y=y_h, stream=s0)
+
+    for i in range(3):
+        e2e_step(i)
+    torch.cuda.synchronize(device)
     e1, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     E = max(8, min(e2e_steps * 10, 200))
     e1.record(s0)
     for i in range(E):
-        for k, v in host[i % 4].items():
-            tin[0][k].copy_(v, non_blocking=True)
-        step(0)
-        y_h.copy_(ys[0], non_blocking=True)
+        e2e_step(i)
     e2.record(s0)
     torch.cuda.synchronize(device)
     e_ms = max_over_ranks([e1.elapsed_time(e2) / E], device)[0]
@@ -686,7 +693,9 @@ def run_decode(steps, warmup, args, rank, world, device, e2e_steps, want_cpu=Tru
         "gpu_launches": nsteps,
         "clocks": sampler.summary(),
         "e2e": {"value": replica_throughput(upd, world, e_ms), "unit": "state-updates/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms,
+                "note": "ssm_scan_step_host: token inputs in and y out over PCIe each step, "
+                        "overlapped with the step by batch chunks; the state stays on the device"},
     }
     if rank == 0 and world == 1 and want_cpu and not args.no_cpu_baseline:
         res["cpu_baseline"] = decode_cpu_baselines(synth.make_decode(steps=1), args.cpu_budget_s)

@@ -218,6 +218,26 @@ SSM_API ssm_status ssm_scan_fwd_host(ssm_scan_plan *plan, const void *x, const v
                                      const float *h0, void *y, float *h_last,
                                      int64_t chunk_tokens, ssm_stream_t stream);
 
+/* One decode step (as ssm_scan_step) with the token's inputs x, delta, z, B,
+ * C and the output y in HOST memory, while the state and the parameters A,
+ * D, delta_bias stay on the device (a server whose tokens arrive on the host
+ * and whose state is resident).  The batch is streamed through the device in
+ * chunks of `chunk_rows` rows (0 = the library's choice: about four chunks,
+ * at least ~1 MB of copies each): the copy-in of chunk c+1, the step of chunk
+ * c and the copy-out of chunk c-1's y overlap on three streams.  Host buffers
+ * should be page-locked for the copies to overlap.  Stream-ordered like
+ * ssm_scan_fwd_host (the work starts behind `stream`'s earlier work and
+ * `stream` waits for all of it; calls on one plan share its staging, so
+ * issue them on one stream).  The first call (and one with another chunk
+ * size) allocates three chunk slots of staging memory (SSM_ERR_OOM if it
+ * cannot).  SSM_A_DIRECT plans get SSM_ERR_INVALID_ARG, SSM_CONV_X plans
+ * SSM_ERR_UNSUPPORTED, as for ssm_scan_step. */
+SSM_API ssm_status ssm_scan_step_host(ssm_scan_plan *plan, const void *x, const void *delta,
+                                      const float *delta_bias, const float *A, const void *B,
+                                      const void *C, const float *D, const void *z,
+                                      float *state, void *y, int64_t chunk_rows,
+                                      ssm_stream_t stream);
+
 /* Forward pass fed by the causal conv front-end of the x branch, fused into
  * the scan kernel so the conv output never goes through HBM unless asked
  * for.  "Tong quan ..." (vietitpro.vn), section 5.3 "Toi uu hoa Kernel

@@ -101,6 +101,8 @@ def load_library(path: str | None = None):
         lib.ssm_scan_destroy.restype = st
         lib.ssm_scan_fwd.argtypes = [_vp] * 13
         lib.ssm_scan_fwd.restype = st
+        lib.ssm_scan_step_host.argtypes = [_vp] * 11 + [ctypes.c_int64, _vp]
+        lib.ssm_scan_step_host.restype = st
         lib.ssm_scan_fwd_host.argtypes = [_vp] * 12 + [ctypes.c_int64, _vp]
         lib.ssm_scan_fwd_host.restype = st
         lib.ssm_scan_fwd_conv.argtypes = [_vp] * 16
@@ -430,6 +432,34 @@ class Plan:
                                      _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(state), _ptr(y),
                                      _stream(dev))
         _check(rc, "ssm_scan_step")
+        return y
+
+    def step_host(self, state, x, delta, A, B, C, D=None, z=None, delta_bias=None, y=None,
+                  chunk_rows=0, stream=None):
+        """One decode step with the token's inputs and y on the host (CPU
+        tensors, pinned for overlapped copies) and the state, A, D,
+        delta_bias on the device (ssm_scan_step_host).  Returns y (CPU),
+        complete once `stream` (default: the current stream) is synchronised."""
+        d, dev = self.desc, self.device
+        Bz, Dm, N = d.batch, d.dim, d.dstate
+        cpu = torch.device("cpu")
+        _need(state, "state", (Bz, Dm, N), torch.float32, dev)
+        for name, t in (("x", x), ("delta", delta), ("z", z)):
+            _need(t, name, (Bz, Dm), self.in_dtype, cpu)
+        _need(B, "B", (Bz, N), self.in_dtype, cpu)
+        _need(C, "C", (Bz, N), self.in_dtype, cpu)
+        _need(A, "A", (Dm, N), torch.float32, dev)
+        _need(D, "D", (Dm,), torch.float32, dev)
+        _need(delta_bias, "delta_bias", (Dm,), torch.float32, dev)
+        if y is None:
+            y = torch.empty((Bz, Dm), dtype=self.out_dtype).pin_memory()
+        _need(y, "y", (Bz, Dm), self.out_dtype, cpu)
+        st = ctypes.c_void_p(stream.cuda_stream if stream is not None
+                             else torch.cuda.current_stream(dev).cuda_stream)
+        rc = self._lib.ssm_scan_step_host(self._h, _ptr(x), _ptr(delta), _ptr(delta_bias),
+                                          _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+                                          _ptr(state), _ptr(y), int(chunk_rows), st)
+        _check(rc, "ssm_scan_step_host")
         return y
 
 

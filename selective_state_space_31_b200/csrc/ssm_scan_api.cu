@@ -104,7 +104,8 @@ struct ssm_scan_plan {
   size_t ws_state_bytes = 0, ws_flag_bytes = 0;
   uint64_t timeout_ns = kDefaultTimeoutNs;
   int64_t drop_unit = -1;
-  HostPipe *pipe = nullptr;  // staging of ssm_scan_fwd_host (allocated by its first call)
+  HostPipe *pipe = nullptr;       // staging of ssm_scan_fwd_host (allocated by its first call)
+  HostPipe *step_pipe = nullptr;  // staging of ssm_scan_step_host (allocated by its first call)
 };
 
 namespace {
@@ -310,6 +311,7 @@ ssm_status ssm_scan_destroy(ssm_scan_plan *pl) {
     if (pl->ws_agg) cudaFree(pl->ws_agg);
     if (pl->ws_map) cudaFree(pl->ws_map);
     host_pipe_free(pl->pipe);
+    host_pipe_free(pl->step_pipe);
   }
   delete pl;
   return SSM_OK;
@@ -1002,6 +1004,143 @@ ssm_status ssm_scan_fwd_host(ssm_scan_plan *pl, const void *x, const void *delta
     if (h_last && !ck(cudaMemcpyAsync(h_last, hp.hbuf + ((nch - 1) % 2) * nstate, nstate * 4,
                                       cudaMemcpyDeviceToHost, hp.s_out)))
       return SSM_ERR_CUDA;
+    return SSM_OK;
+  };
+  const ssm_status st = run();
+  const bool joined = ck(cudaEventRecord(hp.ev_done, hp.s_out)) &&
+                      ck(cudaStreamWaitEvent(stream, hp.ev_done, 0)) &&
+                      ck(cudaEventRecord(hp.ev_start, hp.s_in)) &&
+                      ck(cudaStreamWaitEvent(stream, hp.ev_start, 0));
+  if (st != SSM_OK) return st;
+  return joined ? SSM_OK : SSM_ERR_CUDA;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// ssm_scan_step_host: one decode step with the token's inputs and y in host
+// memory, the batch streamed through the device in chunks of rows
+// ---------------------------------------------------------------------------
+
+namespace {
+
+ssm_status step_pipe_build(ssm_scan_plan *pl, int64_t R, HostPipe **out) {
+  const ssm_scan_desc &d = pl->desc;
+  HostPipe *hp = new (std::nothrow) HostPipe;
+  if (!hp) return SSM_ERR_OOM;
+  hp->Lc = R;  // rows per chunk
+  auto fail = [&](ssm_status st) {
+    cudaGetLastError();
+    host_pipe_free(hp);
+    return st;
+  };
+  const size_t ei = dtype_size(d.in_dtype), eo = dtype_size(d.out_dtype);
+  const size_t xb = align256((size_t)(R * d.dim) * ei), bb = align256((size_t)(R * d.dstate) * ei);
+  hp->off_dt = xb;
+  hp->off_z = 2 * xb;
+  hp->off_B = 3 * xb;
+  hp->off_C = 3 * xb + bb;
+  hp->off_y = 3 * xb + 2 * bb;
+  hp->slot_bytes = hp->off_y + align256((size_t)(R * d.dim) * eo);
+  if (cudaMalloc(&hp->slots, kPipeSlots * hp->slot_bytes) != cudaSuccess) return fail(SSM_ERR_OOM);
+  if (cudaStreamCreateWithFlags(&hp->s_in, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaStreamCreateWithFlags(&hp->s_out, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaEventCreateWithFlags(&hp->ev_start, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&hp->ev_done, cudaEventDisableTiming) != cudaSuccess)
+    return fail(SSM_ERR_CUDA);
+  for (int i = 0; i < kPipeSlots; ++i)
+    if (cudaEventCreateWithFlags(&hp->ev_in[i], cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&hp->ev_comp[i], cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&hp->ev_out[i], cudaEventDisableTiming) != cudaSuccess)
+      return fail(SSM_ERR_CUDA);
+  *out = hp;
+  return SSM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+ssm_status ssm_scan_step_host(ssm_scan_plan *pl, const void *x, const void *delta,
+                              const float *delta_bias, const float *A, const void *B,
+                              const void *C, const float *D, const void *z, float *state,
+                              void *y, int64_t chunk_rows, ssm_stream_t stream_) {
+  if (!pl || chunk_rows < 0) return SSM_ERR_INVALID_ARG;
+  const ssm_scan_desc &d = pl->desc;
+  const uint32_t f = d.flags;
+  if (f & SSM_A_DIRECT) return SSM_ERR_INVALID_ARG;
+  if (f & SSM_CONV_X) return SSM_ERR_UNSUPPORTED;
+  const bool empty = d.batch * d.dim == 0;
+  if (!empty && (!x || !delta || !A || !B || !C || !state || !y)) return SSM_ERR_INVALID_ARG;
+  if (((f & SSM_HAS_Z) != 0) != (z != nullptr) || ((f & SSM_HAS_D) != 0) != (D != nullptr) ||
+      ((f & SSM_HAS_DELTA_BIAS) != 0) != (delta_bias != nullptr))
+    return SSM_ERR_INVALID_ARG;
+  if (empty) return SSM_OK;
+  DeviceGuard guard(pl->device);
+  if (!guard.ok) return SSM_ERR_CUDA;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  const int64_t Bn = d.batch;
+  const size_t ei = dtype_size(d.in_dtype), eo = dtype_size(d.out_dtype);
+  int64_t R = chunk_rows;
+  if (!R) {  // about four chunks, none under ~1 MB of copies
+    const int64_t per_row = d.dim * (3 * (int64_t)ei + (int64_t)eo) + 2 * d.dstate * (int64_t)ei;
+    R = std::max((Bn + 3) / 4, ((int64_t)1 << 20) / std::max<int64_t>(per_row, 1) + 1);
+  }
+  R = std::min(R, Bn);
+  if (!pl->step_pipe || pl->step_pipe->Lc != R) {
+    host_pipe_free(pl->step_pipe);
+    pl->step_pipe = nullptr;
+    const ssm_status st = step_pipe_build(pl, R, &pl->step_pipe);
+    if (st != SSM_OK) return st;
+  }
+  HostPipe &hp = *pl->step_pipe;
+  const int64_t nch = (Bn + R - 1) / R;
+  auto ck = [](cudaError_t e) { return e == cudaSuccess; };
+  auto run = [&]() -> ssm_status {
+    if (!ck(cudaEventRecord(hp.ev_start, stream)) || !ck(cudaStreamWaitEvent(hp.s_in, hp.ev_start, 0)) ||
+        !ck(cudaStreamWaitEvent(hp.s_out, hp.ev_start, 0)))
+      return SSM_ERR_CUDA;
+    for (int64_t c = 0; c < nch; ++c) {
+      const int s = (int)(c % kPipeSlots);
+      const int64_t b0 = c * R, rows = std::min(R, Bn - b0);
+      unsigned char *sb = hp.slots + s * hp.slot_bytes;
+      const size_t xo = (size_t)(b0 * d.dim) * ei, xn = (size_t)(rows * d.dim) * ei;
+      const size_t bo = (size_t)(b0 * d.dstate) * ei, bn = (size_t)(rows * d.dstate) * ei;
+      auto in = [&](size_t off, const void *src, size_t so, size_t n) {
+        return ck(cudaMemcpyAsync(sb + off, static_cast<const unsigned char *>(src) + so, n,
+                                  cudaMemcpyHostToDevice, hp.s_in));
+      };
+      if (c >= kPipeSlots && !ck(cudaStreamWaitEvent(hp.s_in, hp.ev_comp[s], 0))) return SSM_ERR_CUDA;
+      if (!in(0, x, xo, xn) || !in(hp.off_dt, delta, xo, xn) || (z && !in(hp.off_z, z, xo, xn)) ||
+          !in(hp.off_B, B, bo, bn) || !in(hp.off_C, C, bo, bn) ||
+          !ck(cudaEventRecord(hp.ev_in[s], hp.s_in)))
+        return SSM_ERR_CUDA;
+      if (!ck(cudaStreamWaitEvent(stream, hp.ev_in[s], 0)) ||
+          (c >= kPipeSlots && !ck(cudaStreamWaitEvent(stream, hp.ev_out[s], 0))))
+        return SSM_ERR_CUDA;
+      ssm::StepParams p{};
+      p.Bsz = (int)rows; p.D = (int)d.dim; p.N = (int)d.dstate;
+      p.softplus = f & SSM_DELTA_SOFTPLUS;
+      p.has_z = f & SSM_HAS_Z;
+      p.has_D = f & SSM_HAS_D;
+      p.has_bias = f & SSM_HAS_DELTA_BIAS;
+      p.zoh = f & SSM_ZOH;
+      p.in_bf16 = d.in_dtype == SSM_BF16;
+      p.out_bf16 = d.out_dtype == SSM_BF16;
+      p.x = sb; p.dt = sb + hp.off_dt; p.z = z ? sb + hp.off_z : nullptr;
+      p.B = sb + hp.off_B; p.C = sb + hp.off_C;
+      p.A = A; p.Dv = D; p.bias = delta_bias;
+      p.state = state + (size_t)(b0 * d.dim * d.dstate);
+      p.y = sb + hp.off_y;
+      if (ssm::launch_step(p, stream) != cudaSuccess) return SSM_ERR_CUDA;
+      if (!ck(cudaEventRecord(hp.ev_comp[s], stream)) ||
+          !ck(cudaStreamWaitEvent(hp.s_out, hp.ev_comp[s], 0)) ||
+          !ck(cudaMemcpyAsync(static_cast<unsigned char *>(y) + (size_t)(b0 * d.dim) * eo,
+                              sb + hp.off_y, (size_t)(rows * d.dim) * eo, cudaMemcpyDeviceToHost,
+                              hp.s_out)) ||
+          !ck(cudaEventRecord(hp.ev_out[s], hp.s_out)))
+        return SSM_ERR_CUDA;
+    }
     return SSM_OK;
   };
   const ssm_status st = run();

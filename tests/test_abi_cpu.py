@@ -87,6 +87,7 @@ def test_null_arguments(lib):
     assert lib.ssm_scan_create(None, None, 0) == bnd.ERR_INVALID_ARG
     assert lib.ssm_scan_fwd(*([None] * 13)) == bnd.ERR_INVALID_ARG
     assert lib.ssm_scan_fwd_host(*([None] * 12), 0, None) == bnd.ERR_INVALID_ARG
+    assert lib.ssm_scan_step_host(*([None] * 11), 0, None) == bnd.ERR_INVALID_ARG
     assert lib.ssm_scan_step(*([None] * 12)) == bnd.ERR_INVALID_ARG
     assert lib.ssm_scan_get_status(None) == bnd.ERR_INVALID_ARG
     assert lib.ssm_scan_destroy(None) == bnd.ERR_INVALID_ARG

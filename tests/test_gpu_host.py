@@ -87,3 +87,33 @@ def test_host_refuses_conv_plans():
     rc = lib.ssm_scan_fwd_host(plan._h, None, None, None, None, None, None, None, None, None,
                                None, None, 0, None)
     assert rc == bnd.ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("chunk_rows", [0, 3, 64])
+def test_host_decode_steps_against_oracle(chunk_rows):
+    """ssm_scan_step_host: 20 decode steps with the token's inputs and y on
+    the host and the state resident on the device, batch in chunks of 3 rows
+    (the last holds 1), the library's choice, and one chunk; y at every step
+    and the final state against the oracle stepping the same tokens."""
+    import oracle
+    dec = synth.make_decode(Bsz=10, D=96, N=16, steps=20, seed=77)
+    bf, f32 = torch.bfloat16, torch.float32
+    up = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a)).to("cuda", dt)
+    pin = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a)).to(dt).pin_memory()
+    flags = bnd.flags_for(z=1, D=1, delta_bias=1)
+    plan = bnd.Plan(dec.Bsz, 1, dec.D, dec.N, bf, bf, flags)
+    A, Dv, bias = up(dec.A, f32), up(dec.Dskip, f32), up(dec.delta_bias, f32)
+    state = up(dec.h0, f32)
+    ostate = dec.h0.astype(np.float64)
+    orc = oracle.get()
+    for t in range(dec.steps):
+        tok = dec.token(t)
+        y = plan.step_host(state, pin(tok["x"], bf), pin(tok["delta"], bf), A, pin(tok["B"], bf),
+                           pin(tok["C"], bf), D=Dv, z=pin(tok["z"], bf), delta_bias=bias,
+                           chunk_rows=chunk_rows)
+        torch.cuda.synchronize()
+        ry, ostate = orc.step(ostate, tok["x"], tok["delta"], dec.A, tok["B"], tok["C"],
+                              D=dec.Dskip, z=tok["z"], delta_bias=dec.delta_bias)
+        assert gu.normwise(y.float().numpy(), ry) <= gu.TOL["bf16"], t
+    assert gu.normwise(state.cpu().numpy(), ostate) <= 1e-5
+    assert plan.status() == 0
