@@ -222,8 +222,8 @@ SSM_API ssm_status ssm_scan_fwd_host(ssm_scan_plan *plan, const void *x, const v
  * C and the output y in HOST memory, while the state and the parameters A,
  * D, delta_bias stay on the device (a server whose tokens arrive on the host
  * and whose state is resident).  The batch is streamed through the device in
- * chunks of `chunk_rows` rows (0 = the library's choice: about four chunks,
- * at least ~1 MB of copies each): the copy-in of chunk c+1, the step of chunk
+ * chunks of `chunk_rows` rows (0 = the library's choice: two chunks, at
+ * least ~2 MB of copies each): the copy-in of chunk c+1, the step of chunk
  * c and the copy-out of chunk c-1's y overlap on three streams.  Host buffers
  * should be page-locked for the copies to overlap.  Stream-ordered like
  * ssm_scan_fwd_host (the work starts behind `stream`'s earlier work and

@@ -1082,9 +1082,9 @@ ssm_status ssm_scan_step_host(ssm_scan_plan *pl, const void *x, const void *delt
   const int64_t Bn = d.batch;
   const size_t ei = dtype_size(d.in_dtype), eo = dtype_size(d.out_dtype);
   int64_t R = chunk_rows;
-  if (!R) {  // about four chunks, none under ~1 MB of copies
+  if (!R) {  // two chunks, none under ~2 MB of copies (measured best on (256, 5120, 16))
     const int64_t per_row = d.dim * (3 * (int64_t)ei + (int64_t)eo) + 2 * d.dstate * (int64_t)ei;
-    R = std::max((Bn + 3) / 4, ((int64_t)1 << 20) / std::max<int64_t>(per_row, 1) + 1);
+    R = std::max((Bn + 1) / 2, ((int64_t)2 << 20) / std::max<int64_t>(per_row, 1) + 1);
   }
   R = std::min(R, Bn);
   if (!pl->step_pipe || pl->step_pipe->Lc != R) {
