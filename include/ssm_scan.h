@@ -339,9 +339,8 @@ SSM_API ssm_status ssm_scan_step(ssm_scan_plan *plan, const void *x, const void 
  * with SSM_ERR_UNSUPPORTED before anything is launched.  All calls share the
  * scratch, so calls that overlap on the GPU (other streams or threads) race
  * and give wrong results.  The first call on a device looks the scratch
- * address up (cudaGetSymbolAddress); make that first call before any stream
- * capture (a new CUDA context on the device, e.g. after cudaDeviceReset,
- * makes the next call look it up again).  A device-side wait that runs out
+ * address up (cudaGetSymbolAddress); a new CUDA context on the device (e.g.
+ * after cudaDeviceReset) makes the next call look it up again.  A device-side wait that runs out
  * is recorded in the scratch (outputs of that call are then unspecified) and
  * reported by ssm_scan_noalloc_status.  Nothing is allocated; inputs and
  * outputs are the caller's device buffers. */
