@@ -28,6 +28,7 @@ bounded sample of the same workload.
 from __future__ import annotations
 
 import argparse
+import copy
 import hashlib
 import json
 import os
@@ -853,6 +854,11 @@ def main():
                     sub = run_fwd(name, k, w, args, rank, world, device, peaks,
                                   args.e2e_steps)
                 res["workloads"][name] = sub
+            # the backward pass (ssm_scan_bwd) on the 130M layer, about 0.5 s timed
+            bargs = copy.copy(args)
+            bargs.bwd = True
+            res["workloads"]["mamba130m_layer_backward"] = run_fwd(
+                "mamba130m_layer", 500, 10, bargs, rank, world, device, peaks, 0)
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:
