@@ -250,3 +250,37 @@ def test_parts_past_a_short_last_segment(shape, segments):
     assert plan.status() == 0
     ry, rh = gu.run_oracle(inp)
     gu.assert_parity(gy, ry, gh, rh, gu.TOL["bf16"], str(info))
+
+
+def test_segment_layouts_sweep():
+    """Many (length, segments, stage, grid) layouts on a small row set: every
+    stage scanned once whatever the segments' and parts' lengths (short last
+    segments, parts past a segment's end, more CTAs than items), parity and
+    status 0 with a 200 ms wait bound."""
+    failures, ran = [], 0
+    for L in (130, 257, 700, 1031, 2500, 4099):
+        inp = synth.make_fwd(1, L, 64, 16, seed=80 + L % 97, has_h0=True)
+        ry, rh = gu.run_oracle(inp)
+        dev = gu.upload(inp)
+        for M in (2, 4, 8, 16):
+            for tt in (32, 64):
+                for grid in (0, 37):
+                    plan = gu.make_plan(inp)
+                    try:
+                        plan.set_config(segments=M, tile_t=tt, grid=grid)
+                    except bnd.SsmError:
+                        plan.close()
+                        continue
+                    info = plan.info()
+                    plan.set_debug(wait_timeout_ns=200_000_000)
+                    gy, gh = gu.run_gpu(inp, plan, dev)
+                    st = plan.status()
+                    plan.close()
+                    ran += 1
+                    try:
+                        assert st == 0, f"status {st}"
+                        gu.assert_parity(gy, ry, gh, rh, gu.TOL["bf16"], f"L={L} {info}")
+                    except AssertionError as e:
+                        failures.append(str(e))
+    assert ran >= 24, ran
+    assert not failures, "\n".join(failures[:10])
