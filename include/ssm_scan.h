@@ -135,7 +135,8 @@ typedef struct {
   int scan_loop;       /* 1 + variant options: bit 0 software-pipelined scan loop,
                           bit 1 registers capped for five CTAs per SM, bit 2 B and C
                           widened to fp32 once per CTA (bf16 inputs), bit 3 a quarter of
-                          the state exponentials on the FMA pipe */
+                          the state exponentials on the FMA pipe, bit 4 (with bit 0) the
+                          pipelined loop prepares two tokens ahead */
   int carry_lanes_per_chan; /* lanes per channel of the carry pass (segments > 1) */
   int carry_loop;      /* 1 + the carry pass's variant options (segments > 1) */
   int bwd_warps_per_cta; /* scan warps of the fused backward kernel (0: ssm_scan_bwd
@@ -157,8 +158,9 @@ typedef struct {
                          loads issued before this token's update), bit 1 = registers
                          capped so five CTAs fit on an SM, bit 2 = the load warp widens
                          each stage's B and C to fp32 once for the CTA (bf16 inputs),
-                         bit 3 = a quarter of the state exponentials on the FMA pipe;
-                         values above 16 are refused */
+                         bit 3 = a quarter of the state exponentials on the FMA pipe,
+                         bit 4 = (with bit 0) two tokens prepared ahead instead of one;
+                         values above 32 are refused */
   int carry_lanes_per_chan; /* carry pass of a segmented scan: lanes per channel (0 = free) */
   int carry_loop;     /* carry pass: 1 + its variant options, as scan_loop (0 = free) */
   int bwd_warps_per_cta; /* fused backward kernel: 2 or 4 scan warps (0 = free) */

@@ -123,13 +123,17 @@ double warps_weight(int warps) { return warps == 2 ? 0.8 : 1.0; }
 // the exponentials on the FMA pipe (bit 3) took 4-27 % longer, in the carry
 // pass too although its special-function pipe is the busiest (82 %): the
 // polynomial's eight instructions per exponential cost more issue than the
-// relief is worth.
+// relief is worth.  Preparing two tokens ahead in the pipelined loop (bit 4)
+// gained a further 3.7 % on the 130M layer and 1.4 % on the 1.4B layer
+// (three or four tokens ahead under a four-CTA register cap gained less:
+// 2.6 / 1.4 % and 0.6 / -0.6 %); on the long sequence's segmented 4-lane,
+// 32-token scan every pipelined form was slower than the plain loop.
 double opt_weight(int opt, int lpc, int tt, int segments) {
   if (opt == 0) return 1.0;
   if (opt & 4) return 0.9;
   if (opt & 8) return 0.9;
   if (segments > 1 || lpc != 8 || tt != 64) return 0.97;
-  return opt == 1 ? 1.05 : opt == 2 ? 1.04 : 1.03;
+  return opt == 17 ? 1.08 : opt == 1 ? 1.05 : opt == 2 ? 1.04 : 1.03;
 }
 // With segments, the 131k-token rows favoured 4 lanes x 32-token stages over
 // 8 lanes x 64-token stages by about 10 % more than the layer shapes do.

@@ -157,7 +157,8 @@ struct ItemPos {
 // bit 2 (bf16 inputs): the load warp widens each stage's B and C to fp32 in
 // shared memory once for the CTA, instead of every lane widening the values
 // it reads at every token; bit 3: a quarter of the state exponentials on the
-// FMA pipe (one channel per lane, even states per lane).
+// FMA pipe (one channel per lane, even states per lane); bit 4 (with bit 0):
+// the pipelined loop prepares two tokens ahead instead of one.
 template <typename InT, typename OutT, int NS, int LPC, int KC, int WARPS, int TT, bool ZOH,
           bool CARRY, bool CONV, int OPT>
 __global__ void __launch_bounds__((WARPS + 1) * 32, (OPT & 2) ? 5 : 0)
@@ -475,9 +476,12 @@ __global__ void __launch_bounds__((WARPS + 1) * 32, (OPT & 2) ? 5 : 0)
           // Software-pipelined form: the exponentials, input terms and C of
           // token t + 1 are formed (loads, ex2) before token t's state update
           // consumes those of token t, so the special-function latency and
-          // the shared-memory loads overlap the update chain.
+          // the shared-memory loads overlap the update chain (option bit 4:
+          // tokens t + 1 and t + 2, in registers: the special-function and
+          // shared-memory latencies get two tokens' work to hide behind).
           constexpr int NP = NPL / 2;
-          float2 an[NP], bn[NP], cn[NP];
+          constexpr int PD = (OPT & 16) ? 2 : 1;  // tokens prepared ahead
+          float2 an[PD][NP], bn[PD][NP], cn[PD][NP];
           auto prep = [&](int t, float2 (&a)[NP], float2 (&bx)[NP], float2 (&cc)[NP]) {
             const float4 dp = *reinterpret_cast<const float4 *>(prow + (t & ~1));
             const float2 dd = (t & 1) ? make_float2(dp.z, dp.w) : make_float2(dp.x, dp.y);
@@ -494,17 +498,22 @@ __global__ void __launch_bounds__((WARPS + 1) * 32, (OPT & 2) ? 5 : 0)
               cc[k] = make_float2(cv[2 * k], cv[2 * k + 1]);
             }
           };
-          prep(0, an, bn, cn);
+#pragma unroll
+          for (int i = 0; i < PD; ++i) prep(i, an[i], bn[i], cn[i]);
 #pragma unroll
           for (int tt = 0; tt < TT; tt += LPC) {
             float yp[LPC];
 #pragma unroll
             for (int j = 0; j < LPC; ++j) {
-              const int t = tt + j;
+              const int t = tt + j, sl = t % PD;
               float2 ac[NP], bc[NP], ccur[NP];
 #pragma unroll
-              for (int k = 0; k < NP; ++k) { ac[k] = an[k]; bc[k] = bn[k]; ccur[k] = cn[k]; }
-              if (t + 1 < TT) prep(t + 1, an, bn, cn);
+              for (int k = 0; k < NP; ++k) {
+                ac[k] = an[sl][k];
+                bc[k] = bn[sl][k];
+                ccur[k] = cn[sl][k];
+              }
+              if (t + PD < TT) prep(t + PD, an[sl], bn[sl], cn[sl]);
               float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
               for (int k = 0; k < NP; ++k) {

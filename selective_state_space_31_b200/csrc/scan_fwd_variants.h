@@ -2,7 +2,8 @@
 // X(NS, LPC, KC, WARPS, TT, ZOH, CARRY, CONV, OPT), one list per dtype pair and dstate
 // (OPT bit 0: software-pipelined scan loop; bit 1: five CTAs per SM; bit 2:
 // B and C widened to fp32 once per CTA by the load warp, bf16 inputs only;
-// bit 3: a quarter of the state exponentials on the FMA pipe).
+// bit 3: a quarter of the state exponentials on the FMA pipe; bit 4: the
+// pipelined loop prepares two tokens ahead).
 // Only these shapes exist in the library; the planner chooses among them.
 // Row tiles need DT = WARPS * (32 / LPC) * KC channels whose bytes are a
 // multiple of 16 (TMA rows); two channels per lane need an even NPL.
@@ -16,6 +17,7 @@
   X(16, 4, 1, 4, 32, false, false, false, 3) X(16, 8, 1, 4, 64, false, false, false, 3)  \
   X(16, 8, 1, 4, 64, false, false, false, 5) X(16, 4, 1, 4, 32, false, false, false, 4)  \
   X(16, 4, 1, 4, 32, false, false, false, 8)                                              \
+  X(16, 8, 1, 4, 64, false, false, false, 17)                                             \
   X(16, 1, 1, 4, 32, false, false, false, 0) X(16, 2, 1, 4, 32, false, false, false, 0)                      \
   X(16, 4, 1, 4, 32, false, false, false, 0) X(16, 4, 1, 4, 64, false, false, false, 0)                      \
   X(16, 8, 1, 4, 32, false, false, false, 0) X(16, 8, 1, 4, 64, false, false, false, 0)                      \

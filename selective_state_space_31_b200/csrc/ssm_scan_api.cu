@@ -362,8 +362,8 @@ ssm_status ssm_scan_get_info(const ssm_scan_plan *pl, ssm_scan_info *info) {
 ssm_status ssm_scan_set_config(ssm_scan_plan *pl, const ssm_scan_config *cfg) {
   if (!pl || !cfg) return SSM_ERR_INVALID_ARG;
   if (cfg->lanes_per_chan < 0 || cfg->warps_per_cta < 0 || cfg->grid < 0 || cfg->tile_t < 0 ||
-      cfg->chans_per_lane < 0 || cfg->segments < 0 || cfg->scan_loop < 0 || cfg->scan_loop > 16 ||
-      cfg->carry_lanes_per_chan < 0 || cfg->carry_loop < 0 || cfg->carry_loop > 16 ||
+      cfg->chans_per_lane < 0 || cfg->segments < 0 || cfg->scan_loop < 0 || cfg->scan_loop > 32 ||
+      cfg->carry_lanes_per_chan < 0 || cfg->carry_loop < 0 || cfg->carry_loop > 32 ||
       (cfg->bwd_warps_per_cta != 0 && cfg->bwd_warps_per_cta != 2 && cfg->bwd_warps_per_cta != 4) ||
       (cfg->bwd_segments != 0 && cfg->bwd_segments != 1 && cfg->bwd_segments != 2 &&
        cfg->bwd_segments != 4 && cfg->bwd_segments != 8 && cfg->bwd_segments != 16) ||
